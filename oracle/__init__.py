@@ -1,0 +1,225 @@
+"""Oracle for the KV-cache attention step -- TEST INFRASTRUCTURE ONLY.
+
+A plain fp64 CPU statement of what the hot path computes (``oracle.c``),
+plus thin numpy marshalling.  Only ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this package; the
+product package never does and shares no code with it.
+
+What each function follows (pages cited by title and section):
+
+* ``kv_bytes`` -- "9. 推理：从生成到性能优化" (goclawai.cn/llm/inference),
+  section 9.3 "KV Cache": the KV-bytes formula.
+* ``append_contig`` / ``append_paged`` / ``gather_paged`` -- the same page,
+  9.3 (past K/V never change; the new token's K/V are appended) and 9.6
+  (paged KV managed in blocks); "llm-perf-lab" README (preallocated
+  append/commit cache).
+* ``attend`` -- the naive definition: "项目 9-16" roadmap page, project 11
+  (CachedSelfAttention: scores q.K^T * scale, softmax over past+new, times
+  V) and project 15 (naive attention materialises the scores), with the
+  causal-within-chunk and GQA readings stated in ``oracle.c``.
+* ``attend_chunked`` -- "llm-perf-lab" README: chunked attention equals naive
+  attention for any chunk size.
+
+Pins (closed forms, library routines, exhaustive checks, page values) live in
+``tests/test_oracle_pins.py``; planted-mistake checks in
+``tests/test_oracle_mutants.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+HERE = Path(__file__).resolve().parent
+SRC = HERE / "oracle.c"
+LIB = HERE / "liboracle.so"
+
+FP16 = 0
+BF16 = 1
+
+_lib = None
+_lib_path = None
+
+
+def build(src: Path = SRC, out: Path = LIB, defines: tuple[str, ...] = ()) -> Path:
+    """Compile the oracle with gcc (-O2, OpenMP).  Returns the .so path."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-D_GNU_SOURCE", *[f"-D{d}" for d in defines], str(src), "-o", str(out), "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    I64 = ctypes.c_int64
+    D = ctypes.c_double
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = I
+    lib.oracle_decode.argtypes = [P, P, I64, I]
+    lib.oracle_decode.restype = None
+    lib.oracle_round.argtypes = [P, P, I64, I]
+    lib.oracle_round.restype = None
+    lib.oracle_kv_bytes.argtypes = [I64] * 6
+    lib.oracle_kv_bytes.restype = ctypes.c_uint64
+    lib.oracle_append_contig.argtypes = [I, I, I, I, I, P, P, P]
+    lib.oracle_append_contig.restype = None
+    lib.oracle_append_paged.argtypes = [I, I, I, I, I, I, P, P, P, P]
+    lib.oracle_append_paged.restype = None
+    lib.oracle_gather_paged.argtypes = [I, I, I, I, I, I, P, P, P, P]
+    lib.oracle_gather_paged.restype = None
+    lib.oracle_attend.argtypes = [I, I, I, I, I, I, P, P, P, I, P, D, P, I]
+    lib.oracle_attend.restype = None
+    lib.oracle_attend_chunked.argtypes = [I, I, I, I, I, I, P, P, P, I, P, D, I, P, I]
+    lib.oracle_attend_chunked.restype = None
+    return lib
+
+
+def load(path: Path | None = None) -> ctypes.CDLL:
+    """Load (building first if needed) the oracle library."""
+    global _lib, _lib_path
+    path = Path(path) if path is not None else LIB
+    if _lib is not None and _lib_path == path:
+        return _lib
+    if path == LIB and (not LIB.exists() or LIB.stat().st_mtime < SRC.stat().st_mtime):
+        build()
+    lib = _bind(ctypes.CDLL(str(path)))
+    if path == LIB:
+        _lib, _lib_path = lib, path
+    return lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected uint16 bit patterns, got {a.dtype}")
+    return a
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def dtype_code(name: str) -> int:
+    return {"fp16": FP16, "float16": FP16, "bf16": BF16, "bfloat16": BF16}[name]
+
+
+class Oracle:
+    """numpy-level wrappers over one oracle library (the real one or a planted mutant)."""
+
+    def __init__(self, lib: ctypes.CDLL | None = None):
+        self.lib = lib if lib is not None else load()
+
+    # -- storage formats -------------------------------------------------
+    def decode(self, bits, dtype: int) -> np.ndarray:
+        bits = _u16(bits)
+        out = np.empty(bits.shape, dtype=np.float64)
+        self.lib.oracle_decode(_ptr(bits), _ptr(out), bits.size, dtype)
+        return out
+
+    def round(self, x, dtype: int) -> np.ndarray:
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty(x.shape, dtype=np.uint16)
+        self.lib.oracle_round(_ptr(x), _ptr(out), x.size, dtype)
+        return out
+
+    # -- KV bytes ---------------------------------------------------------
+    def kv_bytes(self, layers, kv_heads, head_dim, seq_len, bytes_per_elem, batch) -> int:
+        return int(self.lib.oracle_kv_bytes(layers, kv_heads, head_dim, seq_len,
+                                            bytes_per_elem, batch))
+
+    # -- append / gather ------------------------------------------------
+    def append_contig(self, cache, new_kv, seq_lens) -> None:
+        """cache (B,H_kv,T_cap,D) uint16, updated in place; new_kv (B,H_kv,T_new,D)."""
+        new_kv = _u16(new_kv)
+        assert cache.dtype == np.uint16 and cache.flags["C_CONTIGUOUS"]
+        B, H_kv, T_cap, D = cache.shape
+        T_new = new_kv.shape[2]
+        sl = _i32(seq_lens)
+        assert new_kv.shape == (B, H_kv, T_new, D)
+        assert np.all(sl + T_new <= T_cap) and np.all(sl >= 0)
+        self.lib.oracle_append_contig(B, H_kv, T_new, D, T_cap, _ptr(new_kv), _ptr(sl),
+                                      _ptr(cache))
+
+    def append_paged(self, pool, new_kv, seq_lens, block_table) -> None:
+        """pool (num_pages,H_kv,P,D) uint16, updated in place."""
+        new_kv = _u16(new_kv)
+        assert pool.dtype == np.uint16 and pool.flags["C_CONTIGUOUS"]
+        num_pages, H_kv, P, D = pool.shape
+        B, _, T_new, _ = new_kv.shape
+        sl = _i32(seq_lens)
+        bt = _i32(block_table)
+        max_pages = bt.shape[1]
+        last = (sl + T_new - 1) // P
+        assert np.all(last < max_pages)
+        rows = np.arange(B)
+        for j in range(int(T_new)):
+            pages = bt[rows, (sl + j) // P]
+            assert np.all((pages >= 0) & (pages < num_pages))
+        self.lib.oracle_append_paged(B, H_kv, T_new, D, P, max_pages, _ptr(new_kv),
+                                     _ptr(sl), _ptr(bt), _ptr(pool))
+
+    def gather_paged(self, pool, block_table, n_visible, T_cap: int) -> np.ndarray:
+        """Logical (B,H_kv,T_cap,D) view of the first n_visible[b] positions (rest zero)."""
+        pool = _u16(pool)
+        num_pages, H_kv, P, D = pool.shape
+        bt = _i32(block_table)
+        nv = _i32(n_visible)
+        B, max_pages = bt.shape
+        assert np.all(nv <= T_cap)
+        assert np.all((nv + P - 1) // P <= max_pages)
+        out = np.zeros((B, H_kv, T_cap, D), dtype=np.uint16)
+        self.lib.oracle_gather_paged(B, H_kv, D, P, max_pages, T_cap, _ptr(pool), _ptr(bt),
+                                     _ptr(nv), _ptr(out))
+        return out
+
+    # -- attention --------------------------------------------------------
+    def _check_attend(self, q, K, V, seq_lens):
+        q, K, V = _u16(q), _u16(K), _u16(V)
+        B, H_q, T_new, D = q.shape
+        Bk, H_kv, T_cap, Dk = K.shape
+        assert K.shape == V.shape and Bk == B and Dk == D
+        assert H_q % H_kv == 0
+        sl = _i32(seq_lens)
+        assert sl.shape == (B,) and np.all(sl + T_new <= T_cap)
+        return q, K, V, sl, B, H_q, H_kv, T_new, D, T_cap
+
+    def attend(self, q, K, V, seq_lens, scale: float, dtype: int, nthreads: int = 0):
+        """fp64 output (B,H_q,T_new,D) of exact attention over each request's visible rows."""
+        q, K, V, sl, B, H_q, H_kv, T_new, D, T_cap = self._check_attend(q, K, V, seq_lens)
+        out = np.empty((B, H_q, T_new, D), dtype=np.float64)
+        self.lib.oracle_attend(B, H_q, H_kv, T_new, D, T_cap, _ptr(q), _ptr(K), _ptr(V),
+                               dtype, _ptr(sl), float(scale), _ptr(out), int(nthreads))
+        return out
+
+    def attend_chunked(self, q, K, V, seq_lens, scale: float, dtype: int, chunk: int,
+                       nthreads: int = 0):
+        q, K, V, sl, B, H_q, H_kv, T_new, D, T_cap = self._check_attend(q, K, V, seq_lens)
+        assert chunk >= 1
+        out = np.empty((B, H_q, T_new, D), dtype=np.float64)
+        self.lib.oracle_attend_chunked(B, H_q, H_kv, T_new, D, T_cap, _ptr(q), _ptr(K),
+                                       _ptr(V), dtype, _ptr(sl), float(scale), int(chunk),
+                                       _ptr(out), int(nthreads))
+        return out
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def threads_used(nthreads: int = 0) -> int:
+    """The OpenMP thread count ``attend`` uses for ``nthreads`` (0 = OpenMP's default)."""
+    return nthreads if nthreads > 0 else int(load().oracle_max_threads())

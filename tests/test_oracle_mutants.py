@@ -1,0 +1,85 @@
+"""Plant plausible mistakes in a copy of the oracle and show that the pins catch them.
+
+Each mutant is built from ``oracle/oracle.c`` with one textual replacement
+(the replaced text must occur, or the test fails), compiled with gcc into a
+temporary directory and run through every check in ``tests/oracle_pins.py``.
+A mutant that passes every check would mean the pins cannot see that
+mistake.  CPU only.
+"""
+import ctypes
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+# (name, text in oracle.c, replacement, occurrence: 0 = first only, -1 = all)
+MUTANTS = [
+    ("mask_drops_own_row", "int n = seq_lens[b] + i + 1;\n        const uint16_t* Kb",
+     "int n = seq_lens[b] + i;\n        const uint16_t* Kb", 0),
+    ("mask_sees_next_row", "int n = seq_lens[b] + i + 1;\n        const uint16_t* Kb",
+     "int n = seq_lens[b] + i + 2;\n        const uint16_t* Kb", 0),
+    ("mask_ignores_chunk_row", "int n = seq_lens[b] + i + 1;\n        const uint16_t* Kb",
+     "int n = seq_lens[b] + T_new;\n        const uint16_t* Kb", 0),
+    ("gqa_modulo_mapping", "int g = h / group;", "int g = h % H_kv;", 0),
+    ("scale_dropped", "s[j] = scale * dot;", "s[j] = dot;", 0),
+    ("denominator_is_count", "double pj = s[j] / denom;", "double pj = s[j] / (double)n;", 0),
+    ("exp_sign_flipped", "s[j] = exp(s[j] - mx);", "s[j] = exp(mx - s[j]);", 0),
+    ("values_read_from_K", "const uint16_t* vrow = Vbase + (int64_t)j * D;",
+     "const uint16_t* vrow = Kbase + (int64_t)j * D;", 0),
+    ("keys_reversed", "const uint16_t* krow = Kbase + (int64_t)j * D;",
+     "const uint16_t* krow = Kbase + (int64_t)(n - 1 - j) * D;", 0),
+    ("q_rows_transposed", "attend_row(D, n, q + r * D,",
+     "attend_row(D, n, q + (((int64_t)b * T_new + i) * H_q + h) * D,", 0),
+    ("dot_drops_last_dim", "for (int d = 0; d < D; ++d)\n            dot += qd[d]",
+     "for (int d = 0; d < D - 1; ++d)\n            dot += qd[d]", 0),
+    ("append_contig_off_by_one", "int64_t pos = (int64_t)seq_lens[b] + i;",
+     "int64_t pos = (int64_t)seq_lens[b] + i + 1;", 0),
+    ("append_paged_slot_swapped",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint16_t* src = new_kv",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos % P];\n                int64_t slot = pos / P;\n                const uint16_t* src = new_kv", 0),
+    ("gather_ignores_table",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint16_t* src = pool",
+     "int64_t page = pos / P;\n                int64_t slot = pos % P;\n                const uint16_t* src = pool", 0),
+    ("fp16_bias_wrong", "expo - 25", "expo - 24", 0),
+    ("fp16_subnormal_scale", "ldexp((double)mant, -24)", "ldexp((double)mant, -25)", 0),
+    ("rounding_ties_away", "nearbyint(a / quantum)", "round(a / quantum)", 0),
+    ("kv_bytes_without_k_and_v", "return (uint64_t)2 *", "return (uint64_t)1 *", 0),
+    ("chunked_no_rescale_of_sum", "l *= alpha;", "l *= 1.0;", 0),
+    ("chunked_no_rescale_of_acc", "acc[d] *= alpha;", "acc[d] *= 1.0;", 0),
+]
+
+
+def _mutate(src: str, old: str, new: str, occurrence: int) -> str:
+    assert old in src, f"mutation target not found: {old!r}"
+    if occurrence == -1:
+        return src.replace(old, new)
+    return src.replace(old, new, 1)
+
+
+@pytest.mark.parametrize("name,old,new,occ", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new, occ):
+    src = oracle.SRC.read_text()
+    mutated = _mutate(src, old, new, occ)
+    assert mutated != src
+    c = tmp_path / f"oracle_{name}.c"
+    c.write_text(mutated)
+    so = oracle.build(c, tmp_path / f"liboracle_{name}.so")
+    o = oracle.Oracle(oracle.load(so))
+    caught = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(o)
+        except (AssertionError, FloatingPointError, ValueError, ZeroDivisionError) as e:
+            caught.append(check.__name__)
+    assert caught, f"mutant {name} passed every pin"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    c = tmp_path / "oracle_copy.c"
+    shutil.copy(oracle.SRC, c)
+    o = oracle.Oracle(oracle.load(oracle.build(c, tmp_path / "liboracle_copy.so")))
+    for check in oracle_pins.ALL_CHECKS:
+        check(o)
