@@ -1,0 +1,412 @@
+"""Benchmark of the KV-cache decode step on B200 (one JSON line on rank 0).
+
+Workload (default): 32-layer GQA decode -- B=16 requests, H_q=32, H_kv=8,
+D=128, bf16, contiguous cache, T_past=4096, one new token per request.  A
+step is one decode layer-step for all 32 layers: kvc_append + kvc_attend per
+layer (split-K attend + log-sum-exp combine inside), 8.6 GB of K/V read per
+step, far above the 126 MB L2, so consecutive steps cannot hit in L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvc|reference]
+
+`value` is whole-job KV HBM GB/s: algorithmic bytes of all ranks' steps
+(K/V read, q read, out written, appended K/V written) over the max-over-ranks
+device time.  `e2e` is the same metric through the C ABI with pinned host
+buffers, the host->device copy of q/k_new/v_new and the device->host copy of
+out inside the timed region.  `--impl reference` times the fp64 CPU oracle
+(the only reference implementation there is) on a bounded sample.
+Multi-GPU runs are independent replicas (weak scaling): the decode step has
+no cross-request exchange, so no collective is on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import workloads as W  # noqa: E402
+
+METRIC = ("decode-attention KV HBM GB/s (% of B200 peak) and tokens/s per layer-step")
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.f.flush()
+        rows = [r.split(",") for r in Path(self.f.name).read_text().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for k, name in enumerate(names):
+                    if r[5 + k].strip().lower() == "active":
+                        reasons.add(name)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline
+# ---------------------------------------------------------------------------
+
+def oracle_sample(case: W.Case, layer: int, requests: list[int]):
+    """Inputs for the oracle on a sample of the workload (generated on the host)."""
+    import oracle
+    sel = np.asarray(requests)
+    L = case.seq_lens[sel]
+    T_cap = int(L.max()) + case.T_new
+    shape = (len(sel), case.H_kv, T_cap, case.D)
+    K = W.normal_bits(shape, case.dtype, case.seed, "cpu_k", layer, std=case.kv_std)
+    V = W.normal_bits(shape, case.dtype, case.seed, "cpu_v", layer, std=case.kv_std)
+    q = W.normal_bits((len(sel), case.H_q, case.T_new, case.D), case.dtype, case.seed,
+                      "cpu_q", layer, std=case.q_std)
+    return q, K, V, L, oracle.dtype_code(case.dtype)
+
+
+def sample_bytes(case: W.Case, requests) -> int:
+    L = case.seq_lens[np.asarray(requests)]
+    kv = int((L.astype(np.int64) + case.T_new).sum()) * 2 * case.H_kv * case.D * case.elt
+    qo = 2 * len(requests) * case.H_q * case.T_new * case.D * case.elt
+    app = 2 * len(requests) * case.H_kv * case.T_new * case.D * case.elt
+    return kv + qo + app
+
+
+def time_oracle(case: W.Case, requests: list[int], layers: list[int]) -> tuple[float, int]:
+    """Wall time of the oracle's attend over the sample (inputs prepared outside)."""
+    import oracle
+    o = oracle.get()
+    total, nbytes = 0.0, 0
+    for layer in layers:
+        q, K, V, L, dt = oracle_sample(case, layer, requests)
+        t0 = time.perf_counter()
+        o.attend(q, K, V, L, case.scale, dt)
+        total += time.perf_counter() - t0
+        nbytes += sample_bytes(case, requests)
+    return total, nbytes
+
+
+def cpu_baseline(case: W.Case, budget_s: float = 12.0) -> dict:
+    import oracle
+    reqs = list(range(case.B))
+    layers, t, nb = [], 0.0, 0
+    for layer in range(case.layers):
+        dt, b = time_oracle(case, reqs, [layer])
+        layers.append(layer)
+        t += dt
+        nb += b
+        if t >= budget_s:
+            break
+    return {"value": nb / t / 1e9, "unit": "GB/s", "cores": oracle.threads_used(),
+            "kind": "oracle",
+            "sample": f"{len(layers)} of {case.layers} layers x all {case.B} requests "
+                      f"({case.name}), fp64 C oracle, {t:.1f} s"}
+
+
+def run_reference(args, case: W.Case) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    reqs = [0, 1]  # two requests of one layer per step: a bounded sample
+    for w in range(args.warmup):
+        time_oracle(case, reqs, [w % case.layers])
+    tot, nb = 0.0, 0
+    for s in range(args.steps):
+        dt, b = time_oracle(case, reqs, [s % case.layers])
+        tot += dt
+        nb += b
+    value = nb / tot / 1e9
+    cores = oracle.threads_used()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": case.name, "layers": case.layers, "B": case.B,
+                   "H_q": case.H_q, "H_kv": case.H_kv, "D": case.D, "T_past": 4096,
+                   "T_new": case.T_new, "cache": "contiguous"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: 2 of {case.B} requests of one layer "
+                                   f"({case.name}), fp64 C oracle"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_kvc(args, case: W.Case) -> None:
+    import torch
+    import torch.distributed as dist
+    import kv_cache_decode_03_b200 as kvc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    c = case
+    tdt = {"fp16": torch.float16, "bf16": torch.bfloat16}[c.dtype]
+    cache = kvc.KVCache(c.B, c.H_kv, c.D, c.max_T, c.dtype, num_layers=c.layers)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(c.seed * 1000 + rank)
+    for layer in range(c.layers):
+        for which in ("k", "v"):
+            pool = cache.pool(layer, which)
+            pool.normal_(0.0, c.kv_std, generator=gen)
+    qs = torch.randn((c.layers, c.B, c.H_q, c.T_new, c.D), device="cuda", dtype=tdt,
+                     generator=gen) * c.q_std
+    ks = torch.randn((c.layers, c.B, c.H_kv, c.T_new, c.D), device="cuda", dtype=tdt,
+                     generator=gen) * c.kv_std
+    vs = torch.randn((c.layers, c.B, c.H_kv, c.T_new, c.D), device="cuda", dtype=tdt,
+                     generator=gen) * c.kv_std
+    outs = torch.empty((c.layers, c.B, c.H_q, c.T_new, c.D), device="cuda", dtype=tdt)
+    seq = torch.from_numpy(c.seq_lens).cuda()
+    cache.reserve(c.H_q, c.T_new)
+    ns, split_tokens = cache.plan(c.H_q, c.T_new)
+    stream = torch.cuda.Stream()
+    scale = c.scale
+
+    def step(q=qs, k=ks, v=vs, o=outs):
+        for layer in range(c.layers):
+            cache.append(layer, k[layer], v[layer], seq, stream=stream)
+            cache.attend(layer, q[layer], seq, scale=scale, out=o[layer], stream=stream)
+
+    launches_per_step = c.layers * (2 + (1 if ns > 1 else 0))
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        stream.synchronize()
+        if cache.get_error() != kvc.KVC_OK:
+            raise RuntimeError("device error during warm-up")
+
+        # one step captured in a CUDA graph: the decode loop replays it
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        for _ in range(3):
+            graph.replay()
+        stream.synchronize()
+
+    # ---- timed region: K graph replays, device time by CUDA events
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms)
+    clocks = clk.summary()
+
+    # ---- eager (no graph) step time, for reference
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(max(3, args.steps // 4)):
+            step()
+        e1.record(stream)
+    e1.synchronize()
+    ms_eager = e0.elapsed_time(e1) / max(3, args.steps // 4)
+
+    # ---- per-call attend duration (split-K attend + combine) for the roofline
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(c.layers)]
+    durs = []
+    with torch.cuda.stream(stream):
+        for _ in range(max(2, args.steps // 10)):
+            for layer in range(c.layers):
+                cache.append(layer, ks[layer], vs[layer], seq, stream=stream)
+                evs[layer][0].record(stream)
+                cache.attend(layer, qs[layer], seq, scale=scale, out=outs[layer], stream=stream)
+                evs[layer][1].record(stream)
+            stream.synchronize()
+            durs += [a.elapsed_time(b) for a, b in evs]
+    attend_ms = statistics.mean(durs)
+    if cache.get_error() != kvc.KVC_OK:
+        raise RuntimeError("device error in the timed region")
+
+    # ---- e2e: pinned host buffers, copies inside the timed region
+    hq = qs.cpu().pin_memory()
+    hk = ks.cpu().pin_memory()
+    hv = vs.cpu().pin_memory()
+    ho = torch.empty(outs.shape, dtype=tdt).pin_memory()
+    dq, dk, dv = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
+    e2e_steps = max(3, args.steps // 4)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            step(dq, dk, dv, outs)
+            ho.copy_(outs, non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * c.elt
+    d2h = ho.numel() * c.elt
+
+    step_bytes = c.layers * c.algorithmic_bytes()
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    attend_bytes = c.kv_read_bytes() + 2 * c.B * c.H_q * c.T_new * c.D * c.elt
+    achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    tok_layer_step = world * c.B * c.T_new / (ms * 1e-3 / c.layers)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(c)
+
+    graph.reset()
+    del graph
+    cache.close()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": c.dtype, "data": "synthetic",
+            "config": {"workload": c.name, "layers": c.layers, "B": c.B, "H_q": c.H_q,
+                       "H_kv": c.H_kv, "D": c.D, "T_past": int(c.seq_lens[0]),
+                       "T_new": c.T_new, "cache": "contiguous",
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (8.6 GB of K/V per step)",
+                       "split_k": {"num_splits": ns, "split_tokens": split_tokens},
+                       "timing": "CUDA graph of one 32-layer step, CUDA events"},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "tokens_per_s_per_layer_step": tok_layer_step,
+            "ms_per_step_eager": ms_eager,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "kvc_attend (split-K attend + LSE combine), per call",
+                         "peak_source": peak_kind},
+            "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+WORKLOADS = {
+    "gqa_32layer": lambda: W.gqa_32layer(32),
+}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
+    ap.add_argument("--workload", default="gqa_32layer", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (a smaller case for profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    case = WORKLOADS[args.workload]()
+    if args.layers:
+        case.layers = args.layers
+    if args.impl == "reference":
+        run_reference(args, case)
+    else:
+        run_kvc(args, case)
+
+
+if __name__ == "__main__":
+    main()

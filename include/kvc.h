@@ -1,0 +1,166 @@
+/*
+ * kvc.h -- C ABI of the B200 (sm_100a) KV-cache attention library (libkvc.so).
+ *
+ * The library holds a per-layer K/V cache in device memory and runs the two
+ * steps of one decode (or speculative-verify) layer-step on it:
+ *
+ *   kvc_append  writes the new tokens' K and V into the cache, and
+ *   kvc_attend  attends the new query rows over every cached position.
+ *
+ * Sources (web pages, cited by title and section):
+ *   "9. 推理：从生成到性能优化" (goclawai.cn/llm/inference):
+ *       9.3 "KV Cache" -- past K/V never change; each step projects only the
+ *           new token and appends it; the KV-bytes formula;
+ *       9.6 -- a paged cache managed in fixed-size blocks;
+ *       9.7 -- flash attention is exact attention up to rounding.
+ *   "项目 9-16: Decoding、KV Cache、长上下文与推理系统" (sshipanoo.com):
+ *       project 11 -- K/V are (B, H, T, D), new K/V go after the past along
+ *           T, scores are q.K^T * scale followed by softmax and a product
+ *           with V; project 12 -- MQA/GQA query heads share K/V heads.
+ *   "llm-perf-lab" README -- a preallocated cache with two-phase
+ *       append/commit; speculative decoding verifies gamma drafted tokens in
+ *       one pass and rolls the cache back to the accepted prefix.
+ *
+ * Conventions shared by every call:
+ *   - Element type: fp16 or bf16 (kvc_dtype), the same for q, K, V and out.
+ *     Arithmetic is fp32 with exact (max-subtracted) softmax.
+ *   - All tensor arguments are DEVICE pointers owned by the caller, C-contiguous,
+ *     16-byte aligned.  `stream` is a cudaStream_t (NULL = legacy default stream);
+ *     every call is asynchronous on it.
+ *   - seq_lens: device int32[B]; seq_lens[b] is the committed length L_b of request
+ *     b BEFORE the new tokens.  The library never modifies it: committing T_new
+ *     tokens (append/commit) means the caller adds T_new to seq_lens after the step;
+ *     rolling back after a rejected speculative draft means lowering it.
+ *   - GQA: query head h reads KV head h / (H_q / H_kv).  MHA: H_q == H_kv.  MQA: H_kv == 1.
+ *   - Causality: new row i (0 <= i < T_new) of request b sees positions 0 .. L_b + i.
+ *   - Paged cache: pool[page][H_kv][page_size][D] for K and for V of each layer;
+ *     logical position p of request b lives in page block_table[b*max_pages + p/page_size],
+ *     slot p % page_size.  block_table is device int32[B][max_pages]; entries that a
+ *     call does not reach are never read.  Several requests may list the same physical
+ *     page (shared prefix); appends must target pages owned by one request.
+ *   - Contiguous cache: per layer K and V are (B, H_kv, max_T, D).
+ *   - Host-side argument errors return a status before anything is launched.
+ *     Device-side violations (a page id outside [0, num_pages), a position past the
+ *     capacity, a pipeline wait that ran out) never trap: the offending write or read
+ *     is skipped, a sticky error word in the cache is set, and kvc_get_error reports it.
+ *   - A cache handle is not thread-safe; calls on one handle must be serialised.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVC_OK = 0,
+    KVC_ERR_INVALID_ARG = 1, /* bad shape, null pointer, misalignment, layer out of range */
+    KVC_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement (e.g. D=96) */
+    KVC_ERR_OOM = 3,         /* device allocation failed */
+    KVC_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch error, no device) */
+    KVC_ERR_BOUNDS = 5,      /* device side: page id or position outside the cache */
+    KVC_ERR_TIMEOUT = 6      /* device side: a bounded pipeline wait gave up */
+} kvc_status;
+
+typedef enum { KVC_FP16 = 0, KVC_BF16 = 1 } kvc_dtype;
+
+typedef struct kvc_cache kvc_cache;
+
+/*
+ * kvc_create -- allocate a cache of `num_layers` layers on the current device.
+ *   B          batch size (requests) the cache serves; every later call uses B requests.
+ *   H_kv, D    KV heads and head dim; D must be 32, 64 or 128.
+ *   max_T      per-request capacity in tokens (contiguous: allocated; paged: a bound
+ *              that appends are checked against).
+ *   page_size  0 = contiguous cache; otherwise tokens per page (a power of two, 1..1024).
+ *   num_pages  paged pool size in pages (per layer; K and V each); must be 0 if contiguous.
+ * The pools are zero-filled.  Returns KVC_ERR_OOM if device memory runs out.
+ * Ownership: the handle owns the pools and any workspace; release with kvc_destroy.
+ */
+kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int page_size,
+                      int num_layers, int num_pages, kvc_cache** out);
+
+/* kvc_destroy -- free the pools, workspace and handle (synchronises the device). NULL is ok. */
+kvc_status kvc_destroy(kvc_cache* cache);
+
+/*
+ * kvc_bytes -- bytes held by the K and V pools, following the KV-bytes formula of
+ * "9. 推理" section 9.3: 2 x layers x kv_heads x head_dim x T x bytes x batch, where
+ * T x batch is max_T x B for a contiguous cache and num_pages x page_size for a paged
+ * one.  Page tables and workspace are not counted (the page excludes them too).
+ */
+size_t kvc_bytes(const kvc_cache* cache);
+
+/* kvc_bytes_formula -- the same formula as a pure function (no cache needed). */
+size_t kvc_bytes_formula(int layers, int kv_heads, int head_dim, long long seq_len,
+                         int bytes_per_elem, int batch);
+
+/*
+ * kvc_append -- write the new tokens of one layer into the cache ("9. 推理" 9.3;
+ * "项目 9-16" project 11's concatenation, done in place).
+ *   k_new, v_new  device (B, H_kv, T_new, D) in the cache dtype.
+ *   T_new         tokens per request (>= 1).
+ *   block_table   device int32 (B, max_pages) for a paged cache, NULL for a contiguous one.
+ *   seq_lens      device int32 (B): new token i of request b goes to position seq_lens[b]+i.
+ * Writes are bit-exact copies.  Positions >= max_T, or whose page id is outside the pool,
+ * are skipped and flag KVC_ERR_BOUNDS.
+ */
+kvc_status kvc_append(kvc_cache* cache, int layer, const void* k_new, const void* v_new,
+                      int T_new, const int32_t* block_table, int max_pages,
+                      const int32_t* seq_lens, void* stream);
+
+/*
+ * kvc_attend -- exact-softmax attention of the new query rows of one layer over every
+ * cached position ("项目 9-16" projects 11/15; "9. 推理" 9.7).
+ *   q      device (B, H_q, T_new, D); H_q must be a multiple of H_kv.
+ *   T_new  1 for decode, gamma for a speculative-verify chunk (causal within the chunk).
+ *   block_table, max_pages, seq_lens as for kvc_append (the appended rows are visible).
+ *   scale  multiplies q.k (callers normally pass 1/sqrt(D)).
+ *   out    device (B, H_q, T_new, D), written in the cache dtype.
+ * Must follow the kvc_append of the same tokens on the same stream.  Uses a workspace
+ * owned by the cache for split-K partial results; it grows on demand (a device
+ * allocation, so the first call with a larger shape should precede any stream capture;
+ * kvc_reserve sizes it up front).
+ */
+kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
+                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                      float scale, void* out, void* stream);
+
+/*
+ * kvc_reserve -- size the attend workspace for up to `H_q` query heads, `T_new` new rows
+ * and `max_pages` block-table columns, so that later kvc_attend calls allocate nothing.
+ */
+kvc_status kvc_reserve(kvc_cache* cache, int H_q, int T_new, int max_pages);
+
+/*
+ * kvc_get_error -- synchronise the device, return the sticky device error (KVC_OK,
+ * KVC_ERR_BOUNDS or KVC_ERR_TIMEOUT) and clear it.
+ */
+kvc_status kvc_get_error(kvc_cache* cache);
+
+/* kvc_status_string -- static, human-readable name of a status. */
+const char* kvc_status_string(kvc_status status);
+
+/* kvc_k_pool / kvc_v_pool -- device address of a layer's K / V pool (NULL if out of range);
+ * for initialising history and for bit-exact inspection. */
+void* kvc_k_pool(kvc_cache* cache, int layer);
+void* kvc_v_pool(kvc_cache* cache, int layer);
+
+/* kvc_layer_pool_bytes -- bytes of one layer's K (equally V) pool. */
+size_t kvc_layer_pool_bytes(const kvc_cache* cache);
+
+/*
+ * kvc_plan_splits -- number of split-K slices kvc_attend would use per (request, KV head)
+ * for these arguments, and the tokens each slice covers (for measurement and tests).
+ */
+kvc_status kvc_plan_splits(const kvc_cache* cache, int H_q, int T_new, int max_pages,
+                           int* num_splits, int* split_tokens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H */

@@ -1,0 +1,419 @@
+// kvc_api.cu -- host side of libkvc: the cache object, argument checks, the
+// split-K planner and kernel dispatch behind the C ABI of include/kvc.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "append.cuh"
+#include "attend_simt.cuh"
+#include "combine.cuh"
+#include "kvc.h"
+
+struct kvc_cache {
+  int B, H_kv, D, max_T, page_size, page_shift, num_layers, num_pages;
+  kvc_dtype dtype;
+  bool paged;
+  size_t layer_bytes;  // one layer's K (equally V) pool
+  char* pool;          // layers x {K, V}
+  int* d_err;
+  float* ws;           // split-K workspace
+  size_t ws_bytes;
+  int device;
+  int num_sms;
+};
+
+namespace {
+
+constexpr int kEltBytes = 2;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int log2_exact(int v) {
+  int s = 0;
+  while ((1 << s) < v) ++s;
+  return (1 << s) == v ? s : -1;
+}
+
+kvc_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return KVC_OK;
+  if (e == cudaErrorMemoryAllocation) return KVC_ERR_OOM;
+  return KVC_ERR_CUDA;
+}
+
+int tile_tokens(int D) {
+  switch (D) {
+    case 32: return kvc::SimtCfg<32>::kTile;
+    case 64: return kvc::SimtCfg<64>::kTile;
+    default: return kvc::SimtCfg<128>::kTile;
+  }
+}
+
+// ------------------------------------------------------------ attend plan
+struct Plan {
+  int R;             // query rows per CTA
+  int row_blocks;    // CTAs per KV head along the rows
+  int split_tokens;  // tokens per split-K slice
+  int num_splits;
+  size_t ws_bytes;
+};
+
+template <int D, int R, typename T, bool PAGED>
+int simt_occupancy() {
+  static int occ = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const size_t smem = kvc::SimtCfg<D>::template smem_bytes<R>();
+    cudaFuncSetAttribute(kvc::attend_simt_kernel<D, R, T, PAGED>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kvc::attend_simt_kernel<D, R, T, PAGED>, kvc::SimtCfg<D>::kThreads, smem) !=
+        cudaSuccess)
+      n = 1;
+    occ = std::max(1, n);
+  });
+  return occ;
+}
+
+template <int D, typename T, bool PAGED>
+int occupancy_for(int R) {
+  switch (R) {
+    case 1: return simt_occupancy<D, 1, T, PAGED>();
+    case 2: return simt_occupancy<D, 2, T, PAGED>();
+    default: return simt_occupancy<D, 4, T, PAGED>();
+  }
+}
+
+template <int D, typename T>
+int occupancy_for(int R, bool paged) {
+  return paged ? occupancy_for<D, T, true>(R) : occupancy_for<D, T, false>(R);
+}
+
+template <typename T>
+int occupancy_for(int D, int R, bool paged) {
+  switch (D) {
+    case 32: return occupancy_for<32, T>(R, paged);
+    case 64: return occupancy_for<64, T>(R, paged);
+    default: return occupancy_for<128, T>(R, paged);
+  }
+}
+
+int occupancy(const kvc_cache* c, int R) {
+  return c->dtype == KVC_BF16 ? occupancy_for<__nv_bfloat16>(c->D, R, c->paged)
+                              : occupancy_for<__half>(c->D, R, c->paged);
+}
+
+Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
+  Plan pl{};
+  const int rows = (H_q / c->H_kv) * T_new;
+  pl.R = rows == 1 ? 1 : (rows == 2 ? 2 : 4);
+  pl.row_blocks = kvc::ceil_div(rows, pl.R);
+  const int tile = tile_tokens(c->D);
+  long long cap = c->max_T;
+  if (c->paged) cap = std::min<long long>(cap, (long long)max_pages * c->page_size);
+  cap = std::max<long long>(cap, 1);
+  const long long units = (long long)c->B * c->H_kv * pl.row_blocks;
+  const long long target = 2LL * c->num_sms * occupancy(c, pl.R);  // ~2 waves
+  const long long max_ns = (cap + tile - 1) / tile;
+  long long ns = std::min(std::max((target + units - 1) / units, 1LL), max_ns);
+  long long S = (cap + ns - 1) / ns;
+  S = (S + tile - 1) / tile * tile;
+  ns = (cap + S - 1) / S;
+  pl.split_tokens = (int)S;
+  pl.num_splits = (int)ns;
+  pl.ws_bytes = ns > 1 ? (size_t)c->B * H_q * T_new * ns * (c->D + 1) * sizeof(float) : 0;
+  return pl;
+}
+
+kvc_status ensure_workspace(kvc_cache* c, size_t bytes) {
+  if (bytes <= c->ws_bytes) return KVC_OK;
+  if (c->ws) {
+    cudaError_t e = cudaFree(c->ws);  // synchronises: no launch still reads it
+    c->ws = nullptr;
+    c->ws_bytes = 0;
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  void* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return KVC_ERR_OOM;
+  }
+  c->ws = static_cast<float*>(p);
+  c->ws_bytes = bytes;
+  return KVC_OK;
+}
+
+// --------------------------------------------------------------- dispatch
+template <int D, int R, typename T, bool PAGED>
+kvc_status launch_attend_simt(const kvc::AttendParams& p, cudaStream_t stream) {
+  using C = kvc::SimtCfg<D>;
+  simt_occupancy<D, R, T, PAGED>();  // sets the shared-memory attribute once
+  const size_t smem = C::template smem_bytes<R>();
+  dim3 grid(p.num_splits, p.H_kv * p.row_blocks, p.B);
+  kvc::attend_simt_kernel<D, R, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p);
+  if (p.num_splits > 1) {
+    const long long rows = (long long)p.B * p.H_q * p.T_new;
+    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+    kvc::combine_kernel<D, T><<<blocks, 256, 0, stream>>>(p);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D, typename T, bool PAGED>
+kvc_status dispatch_r(const kvc::AttendParams& p, int R, cudaStream_t s) {
+  switch (R) {
+    case 1: return launch_attend_simt<D, 1, T, PAGED>(p, s);
+    case 2: return launch_attend_simt<D, 2, T, PAGED>(p, s);
+    default: return launch_attend_simt<D, 4, T, PAGED>(p, s);
+  }
+}
+
+template <int D, typename T>
+kvc_status dispatch_paged(const kvc::AttendParams& p, int R, bool paged, cudaStream_t s) {
+  return paged ? dispatch_r<D, T, true>(p, R, s) : dispatch_r<D, T, false>(p, R, s);
+}
+
+template <typename T>
+kvc_status dispatch_d(const kvc::AttendParams& p, int D, int R, bool paged, cudaStream_t s) {
+  switch (D) {
+    case 32: return dispatch_paged<32, T>(p, R, paged, s);
+    case 64: return dispatch_paged<64, T>(p, R, paged, s);
+    default: return dispatch_paged<128, T>(p, R, paged, s);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvc_status_string(kvc_status s) {
+  switch (s) {
+    case KVC_OK: return "KVC_OK";
+    case KVC_ERR_INVALID_ARG: return "KVC_ERR_INVALID_ARG";
+    case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED";
+    case KVC_ERR_OOM: return "KVC_ERR_OOM";
+    case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
+    case KVC_ERR_BOUNDS: return "KVC_ERR_BOUNDS";
+    case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT";
+  }
+  return "KVC_ERR_UNKNOWN";
+}
+
+size_t kvc_bytes_formula(int layers, int kv_heads, int head_dim, long long seq_len,
+                         int bytes_per_elem, int batch) {
+  return (size_t)2 * (size_t)layers * (size_t)kv_heads * (size_t)head_dim * (size_t)seq_len *
+         (size_t)bytes_per_elem * (size_t)batch;
+}
+
+kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int page_size,
+                      int num_layers, int num_pages, kvc_cache** out) {
+  if (!out) return KVC_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (B <= 0 || H_kv <= 0 || max_T <= 0 || num_layers <= 0 || page_size < 0 || num_pages < 0)
+    return KVC_ERR_INVALID_ARG;
+  if (dtype != KVC_FP16 && dtype != KVC_BF16) return KVC_ERR_INVALID_ARG;
+  if (D != 32 && D != 64 && D != 128) return KVC_ERR_UNSUPPORTED;
+  const bool paged = page_size > 0;
+  int shift = 0;
+  if (paged) {
+    shift = log2_exact(page_size);
+    if (shift < 0 || page_size > 1024 || num_pages <= 0) return KVC_ERR_INVALID_ARG;
+  } else if (num_pages != 0) {
+    return KVC_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KVC_ERR_CUDA;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KVC_ERR_CUDA;
+  }
+  const size_t layer_bytes =
+      paged ? (size_t)num_pages * H_kv * page_size * D * kEltBytes
+            : (size_t)B * H_kv * max_T * D * kEltBytes;
+  kvc_cache* c = new kvc_cache();
+  c->B = B;
+  c->H_kv = H_kv;
+  c->D = D;
+  c->max_T = max_T;
+  c->page_size = page_size;
+  c->page_shift = shift;
+  c->num_layers = num_layers;
+  c->num_pages = num_pages;
+  c->dtype = dtype;
+  c->paged = paged;
+  c->layer_bytes = layer_bytes;
+  c->device = dev;
+  c->num_sms = sms;
+  void* pool = nullptr;
+  if (cudaMalloc(&pool, 2 * layer_bytes * (size_t)num_layers) != cudaSuccess) {
+    cudaGetLastError();
+    delete c;
+    return KVC_ERR_OOM;
+  }
+  c->pool = static_cast<char*>(pool);
+  void* err = nullptr;
+  if (cudaMalloc(&err, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(pool);
+    delete c;
+    return KVC_ERR_OOM;
+  }
+  c->d_err = static_cast<int*>(err);
+  if (cudaMemset(c->pool, 0, 2 * layer_bytes * (size_t)num_layers) != cudaSuccess ||
+      cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(c->pool);
+    cudaFree(c->d_err);
+    delete c;
+    return KVC_ERR_CUDA;
+  }
+  *out = c;
+  return KVC_OK;
+}
+
+kvc_status kvc_destroy(kvc_cache* c) {
+  if (!c) return KVC_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaFree(c->pool);
+  cudaFree(c->d_err);
+  if (c->ws) cudaFree(c->ws);
+  delete c;
+  return cuda_status(e);
+}
+
+size_t kvc_bytes(const kvc_cache* c) {
+  if (!c) return 0;
+  if (c->paged)
+    return kvc_bytes_formula(c->num_layers, c->H_kv, c->D,
+                             (long long)c->num_pages * c->page_size, kEltBytes, 1);
+  return kvc_bytes_formula(c->num_layers, c->H_kv, c->D, c->max_T, kEltBytes, c->B);
+}
+
+size_t kvc_layer_pool_bytes(const kvc_cache* c) { return c ? c->layer_bytes : 0; }
+
+void* kvc_k_pool(kvc_cache* c, int layer) {
+  if (!c || layer < 0 || layer >= c->num_layers) return nullptr;
+  return c->pool + (size_t)(2 * layer) * c->layer_bytes;
+}
+
+void* kvc_v_pool(kvc_cache* c, int layer) {
+  if (!c || layer < 0 || layer >= c->num_layers) return nullptr;
+  return c->pool + (size_t)(2 * layer + 1) * c->layer_bytes;
+}
+
+kvc_status kvc_append(kvc_cache* c, int layer, const void* k_new, const void* v_new, int T_new,
+                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                      void* stream) {
+  if (!c || layer < 0 || layer >= c->num_layers || T_new <= 0) return KVC_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !seq_lens || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned4(seq_lens))
+    return KVC_ERR_INVALID_ARG;
+  if (c->paged && (!block_table || !aligned4(block_table) || max_pages <= 0))
+    return KVC_ERR_INVALID_ARG;
+  if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
+  kvc::AppendParams p{};
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_pool = kvc_k_pool(c, layer);
+  p.v_pool = kvc_v_pool(c, layer);
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.B = c->B;
+  p.H_kv = c->H_kv;
+  p.T_new = T_new;
+  p.D = c->D;
+  p.max_T = c->max_T;
+  p.max_pages = max_pages;
+  p.page_shift = c->page_shift;
+  p.num_pages = c->num_pages;
+  p.err = c->d_err;
+  const long long vecs = (long long)c->B * c->H_kv * T_new * (c->D / 8);
+  const unsigned blocks = (unsigned)((vecs + 255) / 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c->paged) kvc::append_kernel<true><<<blocks, 256, 0, s>>>(p);
+  else kvc::append_kernel<false><<<blocks, 256, 0, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+kvc_status kvc_plan_splits(const kvc_cache* c, int H_q, int T_new, int max_pages,
+                           int* num_splits, int* split_tokens) {
+  if (!c || H_q <= 0 || T_new <= 0 || H_q % c->H_kv != 0) return KVC_ERR_INVALID_ARG;
+  if (c->paged && max_pages <= 0) return KVC_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c, H_q, T_new, max_pages);
+  if (num_splits) *num_splits = pl.num_splits;
+  if (split_tokens) *split_tokens = pl.split_tokens;
+  return KVC_OK;
+}
+
+kvc_status kvc_reserve(kvc_cache* c, int H_q, int T_new, int max_pages) {
+  if (!c || H_q <= 0 || T_new <= 0 || H_q % c->H_kv != 0) return KVC_ERR_INVALID_ARG;
+  if (c->paged && max_pages <= 0) return KVC_ERR_INVALID_ARG;
+  return ensure_workspace(c, make_plan(c, H_q, T_new, max_pages).ws_bytes);
+}
+
+kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new,
+                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                      float scale, void* out, void* stream) {
+  if (!c || layer < 0 || layer >= c->num_layers || T_new <= 0 || H_q <= 0 ||
+      H_q % c->H_kv != 0)
+    return KVC_ERR_INVALID_ARG;
+  if (!q || !out || !seq_lens || !aligned16(q) || !aligned16(out) || !aligned4(seq_lens))
+    return KVC_ERR_INVALID_ARG;
+  if (c->paged && (!block_table || !aligned4(block_table) || max_pages <= 0))
+    return KVC_ERR_INVALID_ARG;
+  if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
+  if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c, H_q, T_new, max_pages);
+  kvc_status st = ensure_workspace(c, pl.ws_bytes);
+  if (st != KVC_OK) return st;
+  kvc::AttendParams p{};
+  p.k_pool = kvc_k_pool(c, layer);
+  p.v_pool = kvc_v_pool(c, layer);
+  p.q = q;
+  p.out = out;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.max_pages = max_pages;
+  p.B = c->B;
+  p.H_q = H_q;
+  p.H_kv = c->H_kv;
+  p.T_new = T_new;
+  p.group = H_q / c->H_kv;
+  p.rows = p.group * T_new;
+  p.max_T = c->max_T;
+  p.page_shift = c->page_shift;
+  p.num_pages = c->num_pages;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.split_tokens = pl.split_tokens;
+  p.num_splits = pl.num_splits;
+  p.row_blocks = pl.row_blocks;
+  p.ws_o = c->ws;
+  p.ws_lse = c->ws ? c->ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D : nullptr;
+  p.err = c->d_err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return c->dtype == KVC_BF16 ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
+                              : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
+}
+
+kvc_status kvc_get_error(kvc_cache* c) {
+  if (!c) return KVC_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return KVC_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, c->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  if (h != 0 && cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess) return KVC_ERR_CUDA;
+  return static_cast<kvc_status>(h);
+}
+
+}  // extern "C"

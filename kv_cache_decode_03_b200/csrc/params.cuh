@@ -1,0 +1,44 @@
+// params.cuh -- launch parameter blocks shared by the host planner and the kernels.
+#pragma once
+
+#include <stdint.h>
+
+namespace kvc {
+
+struct AppendParams {
+  const void* k_new;  // (B, H_kv, T_new, D)
+  const void* v_new;
+  void* k_pool;       // this layer's pools
+  void* v_pool;
+  const int32_t* seq_lens;     // (B)
+  const int32_t* block_table;  // (B, max_pages) or null
+  int B, H_kv, T_new, D;
+  int max_T;       // logical capacity per request
+  int max_pages;   // block-table columns
+  int page_shift;  // log2(page_size) (paged)
+  int num_pages;
+  int* err;
+};
+
+struct AttendParams {
+  const void* k_pool;  // this layer's pools
+  const void* v_pool;
+  const void* q;       // (B, H_q, T_new, D)
+  void* out;           // (B, H_q, T_new, D)
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  int max_pages;
+  int B, H_q, H_kv, T_new, group, rows;  // rows = group * T_new (query rows per KV head)
+  int max_T;                             // logical capacity per request
+  int page_shift;                        // log2(page_size) (paged)
+  int num_pages;
+  float scale_log2;   // scale * log2(e): scores are kept in base-2 units
+  int split_tokens;   // tokens per split-K slice (a multiple of the tile)
+  int num_splits;     // slices in the grid
+  int row_blocks;     // CTAs per KV head along the query rows
+  float* ws_o;        // (B, H_q, T_new, num_splits, D) normalised partial outputs
+  float* ws_lse;      // (B, H_q, T_new, num_splits) base-2 log-sum-exp of each slice
+  int* err;
+};
+
+}  // namespace kvc

@@ -1,0 +1,316 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, on identical seeded inputs.
+
+Bars: cache contents bit-exact after every append (the whole pool is compared,
+so slots the append must not touch are checked too); attention output within
+|gpu - oracle| <= 2e-3 + 1e-2 |oracle| per element (fp32 accumulation,
+bf16/fp16 output), with max_abs_err reported.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_decode_03_b200 as kvc
+import workloads as W
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU, skipped there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+def run_case(case: W.Case, layer: int = 0, requests=None, check_pools: bool = True,
+             nthreads: int = 0, twice: bool = False):
+    """Append + attend on the GPU; compare pools bit-exactly and outputs within tolerance."""
+    g = H.GpuRun(case, layers=layer + 1)
+    try:
+        kp0, vp0 = case.k_pool(layer), case.v_pool(layer)
+        g.load_pools(layer, kp0, vp0)
+        g.append(layer, case.k_new(layer), case.v_new(layer))
+        q = case.q(layer)
+        out = g.attend(layer, q)
+        if twice:
+            out2 = g.attend(layer, q)
+            torch.cuda.synchronize()
+            assert torch.equal(out.view(torch.int16), out2.view(torch.int16)), "nondeterministic"
+        assert g.cache.get_error() == kvc.KVC_OK
+        kref, vref = H.oracle_pools_after_append(case, layer, kp0, vp0)
+        if check_pools:
+            kg, vg = g.pools(layer)
+            assert np.array_equal(kg, kref), "K pool differs from the oracle's image"
+            assert np.array_equal(vg, vref), "V pool differs from the oracle's image"
+        sel, ref = H.oracle_attend(case, kref, vref, q, requests, nthreads)
+        got = H.out_to_f64(out)[sel]
+        return H.compare(got, ref, case.name)
+    finally:
+        g.close()
+
+
+# ---------------------------------------------------------------------------
+# small grid: every head dim, dtype, layout and row grouping; ragged lengths
+# that span several tiles and slices
+# ---------------------------------------------------------------------------
+
+HEADS = [(4, 4, 1), (8, 2, 1), (8, 1, 3), (6, 2, 2), (3, 3, 5), (8, 8, 4)]
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("heads", HEADS, ids=lambda h: f"hq{h[0]}_hkv{h[1]}_t{h[2]}")
+def test_small_grid(D, dtype, paged, heads):
+    H_q, H_kv, T_new = heads
+    seed = 1000 + D + 7 * H_q + 13 * T_new + (1 if dtype == "bf16" else 0)
+    if paged:
+        case = W.paged_case("grid", 3, H_q, H_kv, D, dtype, T_new, 0, 700, 16, seed=seed,
+                            pool_seed=seed + 1)
+    else:
+        L = W.rng(seed, "L").integers(0, 700, size=3, endpoint=True)
+        case = W.contig_case("grid", 3, H_q, H_kv, D, dtype, T_new, L, seed=seed,
+                             max_T=int(L.max()) + T_new + 5)
+    run_case(case)
+
+
+@pytest.mark.parametrize("P", [1, 8, 64, 256])
+def test_page_sizes(P):
+    case = W.paged_case(f"pages{P}", 4, 8, 2, 64, "bf16", 2, 0, 900, P, seed=50 + P,
+                        pool_seed=60 + P, share_frac=0.5, share_tokens=4 * P)
+    run_case(case)
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+
+def test_empty_past_single_position():
+    case = W.contig_case("empty", 2, 4, 2, 128, "bf16", 1, 0, seed=5, max_T=1)
+    run_case(case)
+
+
+def test_empty_past_chunk():
+    case = W.contig_case("empty_chunk", 2, 8, 2, 64, "fp16", 7, [0, 3], seed=6, max_T=16)
+    run_case(case)
+
+
+def test_full_capacity():
+    """Append fills the very last slot of the capacity."""
+    case = W.contig_case("full", 2, 8, 8, 64, "bf16", 3, [997, 1], seed=7, max_T=1000)
+    run_case(case)
+
+
+def test_long_context_many_splits():
+    case = W.paged_case("long", 2, 16, 2, 128, "bf16", 4, 20000, 40000, 16, seed=8,
+                        pool_seed=9)
+    run_case(case)
+
+
+def test_mqa_wide_group():
+    case = W.paged_case("mqa", 2, 32, 1, 128, "bf16", 8, 100, 3000, 16, seed=10, pool_seed=11)
+    run_case(case)
+
+
+def test_deterministic():
+    case = W.paged_case("det", 4, 32, 8, 128, "bf16", 1, 500, 5000, 16, seed=12, pool_seed=13)
+    run_case(case, twice=True)
+
+
+# ---------------------------------------------------------------------------
+# the named workloads
+# ---------------------------------------------------------------------------
+
+def test_mha_b1_h16_d32_decode():
+    run_case(W.mha_small(512), twice=True)
+
+
+def test_mha_b1_token_by_token_matches_full_causal():
+    """64 appends of one token into an empty cache, each followed by a decode attend,
+    equal the rows of one full causal attention over the 64 tokens."""
+    import oracle
+    base = W.mha_small(512)
+    T = 64
+    case = W.contig_case("tbt", 1, 16, 16, 32, "fp16", 1, 0, seed=base.seed, max_T=T)
+    K = W.normal_bits((1, 16, T, 32), "fp16", case.seed, "tbt_k")
+    V = W.normal_bits((1, 16, T, 32), "fp16", case.seed, "tbt_v")
+    Q = W.normal_bits((1, 16, T, 32), "fp16", case.seed, "tbt_q")
+    g = H.GpuRun(case)
+    try:
+        rows = []
+        for t in range(T):
+            sl = torch.full((1,), t, dtype=torch.int32, device="cuda")
+            g.append(0, np.ascontiguousarray(K[:, :, t:t + 1]),
+                     np.ascontiguousarray(V[:, :, t:t + 1]), seq_lens=sl)
+            rows.append(H.out_to_f64(g.attend(0, np.ascontiguousarray(Q[:, :, t:t + 1]),
+                                              seq_lens=sl)))
+        assert g.cache.get_error() == kvc.KVC_OK
+        kg, vg = g.pools(0)
+        assert np.array_equal(kg, K) and np.array_equal(vg, V)
+    finally:
+        g.close()
+    full = oracle.get().attend(Q, K, V, np.zeros(1, np.int32), case.scale, oracle.FP16)
+    H.compare(np.concatenate(rows, axis=2), full, "token-by-token")
+
+
+@pytest.mark.parametrize("T_past", W.MHA_SWEEP_T)
+def test_mha_b4_h12_d64_decode(T_past):
+    run_case(W.mha_sweep(T_past))
+
+
+@pytest.mark.parametrize("chunk", W.PREFILL_CHUNKS)
+@pytest.mark.parametrize("T", W.MHA_SWEEP_T)
+def test_mha_b4_h12_d64_chunked_prefill(T, chunk):
+    """Build the cache chunk by chunk (append + causal attend of each chunk); every
+    emitted row equals full causal attention (all rows up to 1024 tokens, sampled
+    rows beyond)."""
+    import oracle
+    B, Hh, D = 4, 12, 64
+    case = W.contig_case("prefill", B, Hh, Hh, D, "fp16", 1, 0, seed=2, max_T=T)
+    K = W.normal_bits((B, Hh, T, D), "fp16", 2, "prefill_k", T)
+    V = W.normal_bits((B, Hh, T, D), "fp16", 2, "prefill_v", T)
+    Q = W.normal_bits((B, Hh, T, D), "fp16", 2, "prefill_q", T)
+    g = H.GpuRun(case)
+    out = np.empty((B, Hh, T, D))
+    try:
+        for s0 in range(0, T, chunk):
+            n = min(chunk, T - s0)
+            sl = torch.full((B,), s0, dtype=torch.int32, device="cuda")
+            g.append(0, np.ascontiguousarray(K[:, :, s0:s0 + n]),
+                     np.ascontiguousarray(V[:, :, s0:s0 + n]), seq_lens=sl)
+            o = g.cache.attend(0, H.to_device(np.ascontiguousarray(Q[:, :, s0:s0 + n]), "fp16"),
+                               sl, scale=case.scale)
+            out[:, :, s0:s0 + n] = H.out_to_f64(o)
+        assert g.cache.get_error() == kvc.KVC_OK
+        kg, vg = g.pools(0)
+        assert np.array_equal(kg, K) and np.array_equal(vg, V)
+    finally:
+        g.close()
+    o = oracle.get()
+    if T <= 1024:
+        ref = o.attend(Q, K, V, np.zeros(B, np.int32), case.scale, oracle.FP16)
+        H.compare(out, ref, f"prefill T={T} chunk={chunk}")
+        return
+    picks = sorted(set([0, 1, chunk - 1, chunk, T - 1] +
+                       list(W.rng(T, chunk, "rows").integers(0, T, size=12))))
+    for t in picks:
+        ref = o.attend(np.ascontiguousarray(Q[:, :, t:t + 1]), K, V,
+                       np.full(B, t, np.int32), case.scale, oracle.FP16)
+        H.compare(out[:, :, t:t + 1], ref, f"prefill T={T} chunk={chunk} row={t}")
+
+
+def test_gqa_b16_l4096_one_layer_full():
+    """One layer of the 32-layer GQA decode at full size, every request checked."""
+    run_case(W.gqa_32layer(layers=1))
+
+
+def test_gqa_b16_l4096_layer_offsets():
+    """Layers are independent pools: layer 3 of a 4-layer cache gives the same check."""
+    case = W.gqa_32layer(layers=4)
+    run_case(case, layer=3, requests=[0, 7, 15])
+
+
+def test_paged_gqa_b64_full():
+    """Paged GQA decode at full size (64 requests, 16 sharing the prefix pages);
+    pools bit-exact, 16 requests (all sharers among them) checked against the oracle."""
+    case = W.paged_gqa()
+    sh = list(case.shared_requests[:8])
+    others = [b for b in range(case.B) if b not in case.shared_requests][:8]
+    run_case(case, requests=sorted(sh + others))
+
+
+@pytest.mark.parametrize("gamma", [2, 4, 8])
+@pytest.mark.parametrize("H_kv", [8, 1])
+def test_spec_verify_full(gamma, H_kv):
+    """Speculative-verify chunks over 8K-32K paged contexts, causal within the chunk."""
+    case = W.spec_verify(gamma, H_kv)
+    run_case(case, requests=[0, 13, 31])
+
+
+# ---------------------------------------------------------------------------
+# errors: host-side rejections and device-side bounds flags (no fault, no trap)
+# ---------------------------------------------------------------------------
+
+def test_host_rejections():
+    c = kvc.KVCache(2, 2, 64, 64, "bf16")
+    try:
+        q = torch.zeros(2, 3, 1, 64, dtype=torch.bfloat16, device="cuda")  # 3 % 2 != 0
+        sl = torch.zeros(2, dtype=torch.int32, device="cuda")
+        with pytest.raises(kvc.KvcError) as e:
+            c.attend(0, q, sl)
+        assert e.value.status == kvc.KVC_ERR_INVALID_ARG
+        buf = torch.zeros(2 * 2 * 1 * 64 + 1, dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(kvc.KvcError) as e:  # misaligned by 2 bytes
+            kvc.kvc_append(c.handle, 0, buf.data_ptr() + 2, buf.data_ptr(), 1, 0, 0,
+                           sl.data_ptr(), 0)
+        assert e.value.status == kvc.KVC_ERR_INVALID_ARG
+        with pytest.raises(kvc.KvcError) as e:
+            kvc.kvc_attend(c.handle, 5, q.data_ptr(), 2, 1, 0, 0, sl.data_ptr(), 1.0,
+                           q.data_ptr(), 0)
+        assert e.value.status == kvc.KVC_ERR_INVALID_ARG
+    finally:
+        c.close()
+
+
+def test_device_bounds_flag_on_bad_page_id():
+    case = W.paged_case("badpage", 2, 8, 2, 64, "bf16", 1, 40, 60, 16, seed=20, pool_seed=21)
+    bt = case.block_table.copy()
+    bt[1, 1] = case.num_pages + 5  # outside the pool
+    case.block_table = bt
+    g = H.GpuRun(case)
+    try:
+        g.load_pools(0)
+        g.attend(0, case.q(0))
+        assert g.cache.get_error() == kvc.KVC_ERR_BOUNDS
+        assert g.cache.get_error() == kvc.KVC_OK  # cleared
+        bt[1, 1] = -1
+        g.block_table = torch.from_numpy(bt).cuda()
+        g.append(0, case.k_new(0), case.v_new(0))
+        g.attend(0, case.q(0))
+        assert g.cache.get_error() == kvc.KVC_OK  # page 1 is not reached by append
+    finally:
+        g.close()
+
+
+def test_device_bounds_flag_on_capacity_overflow():
+    case = W.contig_case("overflow", 2, 4, 4, 32, "fp16", 2, [10, 15], seed=22, max_T=16)
+    g = H.GpuRun(case)
+    try:
+        g.load_pools(0)
+        before = g.pools(0)
+        g.append(0, case.k_new(0), case.v_new(0))  # request 1 would write slot 16
+        assert g.cache.get_error() == kvc.KVC_ERR_BOUNDS
+        after = g.pools(0)
+        # request 0's rows landed, request 1's overflow row did not, nothing else moved
+        kref = before[0].copy()
+        kref[0, :, 10:12] = case.k_new(0)[0]
+        kref[1, :, 15] = case.k_new(0)[1, :, 0]
+        assert np.array_equal(after[0], kref)
+        g.attend(0, case.q(0))
+        assert g.cache.get_error() == kvc.KVC_ERR_BOUNDS
+    finally:
+        g.close()
+
+
+def test_kv_bytes_of_a_cache_follows_the_formula():
+    c = kvc.KVCache(1, 32, 128, 4096, "fp16", num_layers=32)
+    try:
+        assert c.nbytes == 2 * 1024 ** 3
+    finally:
+        c.close()
+    c = kvc.KVCache(1, 8, 128, 4096, "fp16", num_layers=32)
+    try:
+        assert c.nbytes == 512 * 1024 ** 2
+    finally:
+        c.close()
+    c = kvc.KVCache(16, 8, 128, 4097, "bf16", num_layers=2)
+    try:
+        assert c.nbytes == kvc.kvc_bytes_formula(2, 8, 128, 4097, 2, 16)
+    finally:
+        c.close()
+    c = kvc.KVCache(4, 8, 128, 8208, "bf16", page_size=16, num_layers=1, num_pages=1000)
+    try:
+        assert c.nbytes == kvc.kvc_bytes_formula(1, 8, 128, 16 * 1000, 2, 1)
+    finally:
+        c.close()

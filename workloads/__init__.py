@@ -221,8 +221,8 @@ def paged_case(name: str, B: int, H_q: int, H_kv: int, D: int, dtype: str, T_new
         # a request that shares the prefix holds at least the prefix, so the
         # appended rows (positions >= L_b) fall in its private pages
         L[shared] = np.maximum(L[shared], share_tokens)
-    max_pages = -(-(L_hi + T_new) // page_size)
     need = -(-(L.astype(np.int64) + T_new) // page_size)
+    max_pages = max(-(-(L_hi + T_new) // page_size), int(need.max()))
     bt, num_pages = _page_table(B, need, max_pages, shared, shared_pages, pool_seed)
     return Case(name=name, B=B, H_q=H_q, H_kv=H_kv, D=D, dtype=dtype, T_new=T_new,
                 seq_lens=L, seed=seed, layers=layers, page_size=page_size,
