@@ -251,7 +251,7 @@ def run_kvc(args, case: W.Case) -> None:
             cache.append(layer, k[layer], v[layer], seq, stream=stream)
             cache.attend(layer, q[layer], seq, scale=scale, out=o[layer], stream=stream)
 
-    launches_per_step = c.layers * (2 + (1 if ns > 1 else 0))
+    launches_per_step = c.layers * 2  # append + attend (the slice merge is fused)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):

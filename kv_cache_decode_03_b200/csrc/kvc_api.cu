@@ -1,15 +1,18 @@
 // kvc_api.cu -- host side of libkvc: the cache object, argument checks, the
 // split-K planner and kernel dispatch behind the C ABI of include/kvc.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "append.cuh"
-#include "attend_simt.cuh"
-#include "combine.cuh"
+#include "attend_decode.cuh"
+#include "attend_mma.cuh"
 #include "kvc.h"
 
 struct kvc_cache {
@@ -19,8 +22,11 @@ struct kvc_cache {
   size_t layer_bytes;  // one layer's K (equally V) pool
   char* pool;          // layers x {K, V}
   int* d_err;
-  float* ws;           // split-K workspace
+  float* ws;           // split-K workspace: partial outputs, lse, slice tickets
   size_t ws_bytes;
+  bool tma;                        // tensor maps built: the tensor-core path is available
+  std::vector<CUtensorMap> tmk;    // per layer: K pool as a 2-D (rows, D) tensor
+  std::vector<CUtensorMap> tmv;
   int device;
   int num_sms;
 };
@@ -28,6 +34,12 @@ struct kvc_cache {
 namespace {
 
 constexpr int kEltBytes = 2;
+
+// Split-K sizing: aim for this many waves of resident CTAs, so that the last
+// wave's imbalance is a small fraction of the pass.
+#ifndef KVC_SPLIT_WAVES
+#define KVC_SPLIT_WAVES 4
+#endif
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -46,18 +58,121 @@ kvc_status cuda_status(cudaError_t e) {
 
 int tile_tokens(int D) {
   switch (D) {
-    case 32: return kvc::SimtCfg<32>::kTile;
-    case 64: return kvc::SimtCfg<64>::kTile;
-    default: return kvc::SimtCfg<128>::kTile;
+    case 32: return kvc::DecodeCfg<32>::kTile;
+    case 64: return kvc::DecodeCfg<64>::kTile;
+    default: return kvc::DecodeCfg<128>::kTile;
   }
+}
+
+// ------------------------------------------------------------- tensor maps
+// The pools are addressed by TMA as 2-D tensors of rows x D elements: rows are
+// (b, g, position) for a contiguous cache and (page, g, slot) for a paged one.
+// Boxes are 64 elements (128 bytes, the swizzle span) by up to 64 rows.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* m, void* base, kvc_dtype dtype, int D, long long rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * kEltBytes};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = fn(m,
+                        dtype == KVC_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+void build_tmaps(kvc_cache* c) {
+  c->tma = false;
+  if (c->D != 64 && c->D != 128) return;
+  if (c->paged && c->page_size < 8) return;  // boxes must start on 1024-byte swizzle atoms
+  const long long rows = c->paged ? (long long)c->num_pages * c->H_kv * c->page_size
+                                  : (long long)c->B * c->H_kv * c->max_T;
+  if (rows + 64 >= (1LL << 31)) return;  // TMA coordinates are 32-bit
+  const int box_rows = c->paged ? std::min(c->page_size, 64) : 64;
+  c->tmk.resize(c->num_layers);
+  c->tmv.resize(c->num_layers);
+  for (int l = 0; l < c->num_layers; ++l) {
+    if (!make_tmap(&c->tmk[l], c->pool + (size_t)(2 * l) * c->layer_bytes, c->dtype, c->D,
+                   rows, box_rows) ||
+        !make_tmap(&c->tmv[l], c->pool + (size_t)(2 * l + 1) * c->layer_bytes, c->dtype, c->D,
+                   rows, box_rows))
+      return;
+  }
+  c->tma = true;
+}
+
+template <int D, int NT, typename T, bool PAGED>
+int mma_occupancy() {
+  static int occ = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const size_t smem = kvc::MmaCfg<D>::template smem_bytes<NT>();
+    cudaFuncSetAttribute(kvc::attend_mma_kernel<D, NT, T, PAGED>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kvc::attend_mma_kernel<D, NT, T, PAGED>, kvc::MmaCfg<D>::kThreads, smem) !=
+        cudaSuccess)
+      n = 1;
+    occ = std::max(1, n);
+  });
+  return occ;
+}
+
+template <int D, typename T, bool PAGED>
+int mma_occ_nt(int NT) {
+  switch (NT) {
+    case 1: return mma_occupancy<D, 1, T, PAGED>();
+    case 2: return mma_occupancy<D, 2, T, PAGED>();
+    default: return mma_occupancy<D, 4, T, PAGED>();
+  }
+}
+
+template <typename T>
+int mma_occ(int D, int NT, bool paged) {
+  if (D == 64) return paged ? mma_occ_nt<64, T, true>(NT) : mma_occ_nt<64, T, false>(NT);
+  return paged ? mma_occ_nt<128, T, true>(NT) : mma_occ_nt<128, T, false>(NT);
+}
+
+int mma_scratch_floats(int D, int NT) {
+  if (D == 64)
+    return NT == 1 ? kvc::MmaCfg<64>::scratch_floats<1>()
+                   : NT == 2 ? kvc::MmaCfg<64>::scratch_floats<2>()
+                             : kvc::MmaCfg<64>::scratch_floats<4>();
+  return NT == 1 ? kvc::MmaCfg<128>::scratch_floats<1>()
+                 : NT == 2 ? kvc::MmaCfg<128>::scratch_floats<2>()
+                           : kvc::MmaCfg<128>::scratch_floats<4>();
 }
 
 // ------------------------------------------------------------ attend plan
 struct Plan {
+  bool mma;          // tensor-core kernel (else the CUDA-core kernel)
+  int NT;            // mma: 8-row n-tiles per CTA
   int R;             // query rows per CTA
   int row_blocks;    // CTAs per KV head along the rows
   int split_tokens;  // tokens per split-K slice
   int num_splits;
+  size_t ws_partial_floats;  // partial outputs + lse
+  size_t ws_counters;        // slice tickets
   size_t ws_bytes;
 };
 
@@ -66,12 +181,12 @@ int simt_occupancy() {
   static int occ = 0;
   static std::once_flag once;
   std::call_once(once, [] {
-    const size_t smem = kvc::SimtCfg<D>::template smem_bytes<R>();
-    cudaFuncSetAttribute(kvc::attend_simt_kernel<D, R, T, PAGED>,
+    const size_t smem = kvc::DecodeCfg<D>::template smem_bytes<R>();
+    cudaFuncSetAttribute(kvc::attend_decode_kernel<D, R, T, PAGED>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, kvc::attend_simt_kernel<D, R, T, PAGED>, kvc::SimtCfg<D>::kThreads, smem) !=
+            &n, kvc::attend_decode_kernel<D, R, T, PAGED>, kvc::DecodeCfg<D>::kThreads, smem) !=
         cudaSuccess)
       n = 1;
     occ = std::max(1, n);
@@ -110,25 +225,44 @@ int occupancy(const kvc_cache* c, int R) {
 Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
   Plan pl{};
   const int rows = (H_q / c->H_kv) * T_new;
-  pl.R = rows == 1 ? 1 : (rows == 2 ? 2 : 4);
+  // Three or more query rows per K/V row make q.k and p.v a dense contraction
+  // worth the tensor cores; one or two rows stay on CUDA cores.
+  pl.mma = c->tma && rows >= 3;
+  int tile, occ, scratch = 1 << 30;
+  if (pl.mma) {
+    pl.NT = rows <= 8 ? 1 : (rows <= 16 ? 2 : 4);
+    pl.R = pl.NT * 8;
+    tile = 64;
+    occ = c->dtype == KVC_BF16 ? mma_occ<__nv_bfloat16>(c->D, pl.NT, c->paged)
+                               : mma_occ<__half>(c->D, pl.NT, c->paged);
+    scratch = mma_scratch_floats(c->D, pl.NT);
+  } else {
+    pl.NT = 0;
+    pl.R = rows == 1 ? 1 : (rows == 2 ? 2 : 4);
+    tile = tile_tokens(c->D);
+    occ = occupancy(c, pl.R);
+  }
   pl.row_blocks = kvc::ceil_div(rows, pl.R);
-  const int tile = tile_tokens(c->D);
   long long cap = c->max_T;
   if (c->paged) cap = std::min<long long>(cap, (long long)max_pages * c->page_size);
   cap = std::max<long long>(cap, 1);
   const long long units = (long long)c->B * c->H_kv * pl.row_blocks;
-  const long long target = 2LL * c->num_sms * occupancy(c, pl.R);  // ~2 waves
-  const long long max_ns = (cap + tile - 1) / tile;
+  const long long target = (long long)KVC_SPLIT_WAVES * c->num_sms * occ;
+  // the merging CTA keeps one weight per (row, slice) in shared memory
+  const long long max_ns = std::min<long long>((cap + tile - 1) / tile, scratch / pl.R);
   long long ns = std::min(std::max((target + units - 1) / units, 1LL), max_ns);
   long long S = (cap + ns - 1) / ns;
   S = (S + tile - 1) / tile * tile;
   ns = (cap + S - 1) / S;
   pl.split_tokens = (int)S;
   pl.num_splits = (int)ns;
-  pl.ws_bytes = ns > 1 ? (size_t)c->B * H_q * T_new * ns * (c->D + 1) * sizeof(float) : 0;
+  pl.ws_partial_floats = ns > 1 ? (size_t)c->B * H_q * T_new * ns * (c->D + 1) : 0;
+  pl.ws_counters = ns > 1 ? (size_t)c->B * c->H_kv * pl.row_blocks : 0;
+  pl.ws_bytes = pl.ws_partial_floats * sizeof(float) + pl.ws_counters * sizeof(int);
   return pl;
 }
 
+// Grow the workspace to `bytes` (zero-filled: slice tickets must start at 0).
 kvc_status ensure_workspace(kvc_cache* c, size_t bytes) {
   if (bytes <= c->ws_bytes) return KVC_OK;
   if (c->ws) {
@@ -143,24 +277,55 @@ kvc_status ensure_workspace(kvc_cache* c, size_t bytes) {
     cudaGetLastError();
     return KVC_ERR_OOM;
   }
+  if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(p);
+    return KVC_ERR_CUDA;
+  }
   c->ws = static_cast<float*>(p);
   c->ws_bytes = bytes;
   return KVC_OK;
 }
 
 // --------------------------------------------------------------- dispatch
+template <int D, int NT, typename T, bool PAGED>
+kvc_status launch_attend_mma(const kvc::AttendParams& p, const CUtensorMap& tk,
+                             const CUtensorMap& tv, cudaStream_t stream) {
+  using C = kvc::MmaCfg<D>;
+  mma_occupancy<D, NT, T, PAGED>();  // sets the shared-memory attribute once
+  const size_t smem = C::template smem_bytes<NT>();
+  dim3 grid(p.num_splits, p.H_kv * p.row_blocks, p.B);
+  kvc::attend_mma_kernel<D, NT, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p, tk, tv);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D, typename T, bool PAGED>
+kvc_status dispatch_mma_nt(const kvc::AttendParams& p, int NT, const CUtensorMap& tk,
+                           const CUtensorMap& tv, cudaStream_t s) {
+  switch (NT) {
+    case 1: return launch_attend_mma<D, 1, T, PAGED>(p, tk, tv, s);
+    case 2: return launch_attend_mma<D, 2, T, PAGED>(p, tk, tv, s);
+    default: return launch_attend_mma<D, 4, T, PAGED>(p, tk, tv, s);
+  }
+}
+
+template <typename T>
+kvc_status dispatch_mma(const kvc::AttendParams& p, int D, int NT, bool paged,
+                        const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  if (D == 64)
+    return paged ? dispatch_mma_nt<64, T, true>(p, NT, tk, tv, s)
+                 : dispatch_mma_nt<64, T, false>(p, NT, tk, tv, s);
+  return paged ? dispatch_mma_nt<128, T, true>(p, NT, tk, tv, s)
+               : dispatch_mma_nt<128, T, false>(p, NT, tk, tv, s);
+}
+
 template <int D, int R, typename T, bool PAGED>
 kvc_status launch_attend_simt(const kvc::AttendParams& p, cudaStream_t stream) {
-  using C = kvc::SimtCfg<D>;
+  using C = kvc::DecodeCfg<D>;
   simt_occupancy<D, R, T, PAGED>();  // sets the shared-memory attribute once
   const size_t smem = C::template smem_bytes<R>();
   dim3 grid(p.num_splits, p.H_kv * p.row_blocks, p.B);
-  kvc::attend_simt_kernel<D, R, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p);
-  if (p.num_splits > 1) {
-    const long long rows = (long long)p.B * p.H_q * p.T_new;
-    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
-    kvc::combine_kernel<D, T><<<blocks, 256, 0, stream>>>(p);
-  }
+  kvc::attend_decode_kernel<D, R, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -277,6 +442,7 @@ kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int pa
     delete c;
     return KVC_ERR_CUDA;
   }
+  build_tmaps(c);
   *out = c;
   return KVC_OK;
 }
@@ -399,8 +565,14 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   p.row_blocks = pl.row_blocks;
   p.ws_o = c->ws;
   p.ws_lse = c->ws ? c->ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D : nullptr;
+  p.counters = c->ws ? reinterpret_cast<int*>(c->ws + pl.ws_partial_floats) : nullptr;
   p.err = c->d_err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.mma)
+    return c->dtype == KVC_BF16
+               ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
+                                             c->tmv[layer], s)
+               : dispatch_mma<__half>(p, c->D, pl.NT, c->paged, c->tmk[layer], c->tmv[layer], s);
   return c->dtype == KVC_BF16 ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
                               : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
 }
@@ -412,7 +584,12 @@ kvc_status kvc_get_error(kvc_cache* c) {
   int h = 0;
   if (cudaMemcpy(&h, c->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return KVC_ERR_CUDA;
-  if (h != 0 && cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess) return KVC_ERR_CUDA;
+  if (h != 0) {
+    if (cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess) return KVC_ERR_CUDA;
+    // A launch that gave up may have left slice tickets behind: clear them all.
+    if (c->ws && cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) return KVC_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return KVC_ERR_CUDA;
+  }
   return static_cast<kvc_status>(h);
 }
 

@@ -38,6 +38,7 @@ struct AttendParams {
   int row_blocks;     // CTAs per KV head along the query rows
   float* ws_o;        // (B, H_q, T_new, num_splits, D) normalised partial outputs
   float* ws_lse;      // (B, H_q, T_new, num_splits) base-2 log-sum-exp of each slice
+  int* counters;      // (B, H_kv, row_blocks) slice tickets, zero between launches
   int* err;
 };
 

@@ -255,6 +255,7 @@ def test_host_rejections():
 
 def test_device_bounds_flag_on_bad_page_id():
     case = W.paged_case("badpage", 2, 8, 2, 64, "bf16", 1, 40, 60, 16, seed=20, pool_seed=21)
+    good = case.block_table.copy()
     bt = case.block_table.copy()
     bt[1, 1] = case.num_pages + 5  # outside the pool
     case.block_table = bt
@@ -267,8 +268,13 @@ def test_device_bounds_flag_on_bad_page_id():
         bt[1, 1] = -1
         g.block_table = torch.from_numpy(bt).cuda()
         g.append(0, case.k_new(0), case.v_new(0))
+        assert g.cache.get_error() == kvc.KVC_OK  # append never reaches logical page 1
         g.attend(0, case.q(0))
-        assert g.cache.get_error() == kvc.KVC_OK  # page 1 is not reached by append
+        assert g.cache.get_error() == kvc.KVC_ERR_BOUNDS  # attend does
+        # the rejected page left the slice tickets clean: a valid table works again
+        g.block_table = torch.from_numpy(good).cuda()
+        g.attend(0, case.q(0))
+        assert g.cache.get_error() == kvc.KVC_OK
     finally:
         g.close()
 
