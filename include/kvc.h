@@ -153,8 +153,11 @@ void* kvc_v_pool(kvc_cache* cache, int layer);
 size_t kvc_layer_pool_bytes(const kvc_cache* cache);
 
 /*
- * kvc_plan_splits -- number of split-K slices kvc_attend would use per (request, KV head)
- * for these arguments, and the tokens each slice covers (for measurement and tests).
+ * kvc_plan_splits -- how kvc_attend would divide the work for these arguments (for
+ * measurement and tests).  Fixed-size split-K: *num_splits slices of *split_tokens tokens
+ * per (request, KV head).  Persistent stream-K (up to 16 query rows per KV head with the
+ * tensor-core path): *num_splits is the number of persistent CTAs, each streaming an equal
+ * share of all K/V tiles, and *split_tokens is 0.
  */
 kvc_status kvc_plan_splits(const kvc_cache* cache, int H_q, int T_new, int max_pages,
                            int* num_splits, int* split_tokens);

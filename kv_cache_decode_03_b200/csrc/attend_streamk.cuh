@@ -1,0 +1,563 @@
+// attend_streamk.cuh -- N2 + N3 (tensor-core, persistent): stream-K split attention.
+//
+// Same contract and the same per-tile arithmetic as attend_mma.cuh (mma.m16n8k16
+// with tokens as M, query rows as N; fp32 online softmax), organised so that no
+// SM waits for work or for memory between pieces of work:
+//
+// * Work is counted in 64-token tiles of "segments" s = (request b, KV head g,
+//   row block rb), in that order; segment s has ceil((L_b + i_max + 1) / 64)
+//   tiles, where i_max is the largest new-row index of the row block.  Each of
+//   the G persistent CTAs takes the contiguous tile range
+//   [c*W/G, (c+1)*W/G) of the W tiles in total, so every CTA streams the same
+//   number of K/V bytes to within one tile, whatever the mix of lengths.
+//   Every CTA computes the per-request tile counts and their prefix sums from
+//   seq_lens itself (a block scan), so the host needs no lengths.
+// * Lane 0 of warp 0 keeps the 3-stage TMA ring full across segment
+//   boundaries; the first tile of each segment piece also carries that
+//   segment's q rows (one bulk copy into a per-stage q slot).
+// * When a piece ends, the four warps merge their partial results inside the
+//   stage they just consumed, while the other stages keep streaming.  A piece
+//   that covers its whole segment writes the output directly.  A CTA has at
+//   most two partial pieces (its first and its last); they go to slots
+//   (c, 0) and (c, 1) of the workspace, and the last CTA of a segment to
+//   finish merges the segment's pieces by log-sum-exp ("9. 推理" 9.7:
+//   exact up to rounding); an atomic ticket after a release fence decides
+//   who is last, so nothing ever waits on another CTA.
+#pragma once
+
+#include <cuda.h>
+#include <math.h>
+
+#include "attend_mma.cuh"
+#include "device_common.cuh"
+#include "params.cuh"
+#include "splitk_epilogue.cuh"
+
+namespace kvc {
+
+template <int D>
+struct StreamKCfg {
+  static constexpr int kWarps = 4;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kTile = 64;
+  static constexpr int kHalves = D / 64;
+  static constexpr int kBoxBytes = kTile * 128;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kStages = 3;
+  static constexpr int kKSteps = D / 16;
+  static constexpr int kMTiles = D / 16;
+  static constexpr int kRing = 2 * kStages * kTileBytes;
+
+  template <int NT>
+  static constexpr size_t smem_bytes() {
+    return 1024 + kRing                                 // aligned K and V rings
+           + kStages * NT * 8 * D * 2                   // q slots
+           + kWarps * NT * 8 * 2 * sizeof(float)        // warp m and l
+           + 2 * kStages * sizeof(uint64_t) + 64;       // barriers, flags
+  }
+  // the block scan of per-request tile counts uses the ring before the first copy
+  static constexpr int kMaxBatch = kRing / (int)sizeof(int) - 1;
+};
+
+// Row-block geometry: new-row indices covered by row block rb.
+struct RowBlock {
+  int imin, imax;
+};
+
+__device__ __forceinline__ RowBlock row_block(int rb, int R, int rows, int T_new) {
+  const int r0 = rb * R;
+  const int r1 = min(r0 + R, rows) - 1;
+  if (r1 - r0 + 1 >= T_new) return {0, T_new - 1};
+  const int i0 = r0 % T_new, i1 = r1 % T_new;
+  return i1 >= i0 ? RowBlock{i0, i1} : RowBlock{0, T_new - 1};
+}
+
+__device__ __forceinline__ bool length_ok(const AttendParams& p, int L, bool paged) {
+  return L >= 0 && L + p.T_new <= p.max_T &&
+         (!paged || ((L + p.T_new - 1) >> p.page_shift) < p.max_pages);
+}
+
+template <int R>
+__device__ __forceinline__ int request_tiles(const AttendParams& p, int L) {
+  int t = 0;
+  for (int rb = 0; rb < p.row_blocks; ++rb)
+    t += ceil_div(L + row_block(rb, R, p.rows, p.T_new).imax + 1, 64);
+  return t * p.H_kv;
+}
+
+// Walks tiles in the global order: request, KV head, row block, tile.
+template <int R>
+struct TileCursor {
+  int b, g, rb, L, k, seg_tiles;
+  long long seg_start;  // global index of the segment's first tile
+
+  __device__ __forceinline__ void enter_segment(const AttendParams& p) {
+    seg_tiles = ceil_div(L + row_block(rb, R, p.rows, p.T_new).imax + 1, 64);
+  }
+  __device__ __forceinline__ void next(const AttendParams& p, bool paged) {
+    if (++k < seg_tiles) return;
+    seg_start += seg_tiles;
+    k = 0;
+    if (++rb == p.row_blocks) {
+      rb = 0;
+      if (++g == p.H_kv) {
+        g = 0;
+        do {  // requests whose length is invalid contribute no tiles
+          ++b;
+          L = b < p.B ? p.seq_lens[b] : 0;
+        } while (b < p.B && !length_ok(p, L, paged));
+      }
+    }
+    enter_segment(p);
+  }
+};
+
+template <int D, int NT, typename T, bool PAGED>
+__global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
+    attend_streamk_kernel(const AttendParams p, const __grid_constant__ CUtensorMap tmk,
+                          const __grid_constant__ CUtensorMap tmv) {
+  using C = StreamKCfg<D>;
+  constexpr int W = C::kWarps;
+  constexpr int NTH = C::kThreads;
+  constexpr int R = NT * 8;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sk = smem;
+  unsigned char* sv = smem + C::kStages * C::kTileBytes;
+  unsigned char* sq = smem + C::kRing;  // [stage][R][D]
+  float* red_m = reinterpret_cast<float*>(sq + C::kStages * R * D * 2);
+  float* red_l = red_m + W * R;
+  uint64_t* full = reinterpret_cast<uint64_t*>(red_l + W * R);
+  uint64_t* empty = full + C::kStages;
+  int* flags = reinterpret_cast<int*>(empty + C::kStages);  // [0] abort, [1] last, [4..7] scan
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int c = blockIdx.x;
+
+  // ---------------------------------------------- per-request tile prefix
+  int* P = reinterpret_cast<int*>(smem);  // [B + 1], in the ring before any copy
+  {
+    const int per = ceil_div(p.B, NTH);
+    const int b_lo = min(p.B, tid * per), b_hi = min(p.B, b_lo + per);
+    int sum = 0;
+    for (int b = b_lo; b < b_hi; ++b) {
+      const int L = p.seq_lens[b];
+      int t = 0;
+      if (length_ok(p, L, PAGED)) t = request_tiles<R>(p, L);
+      else flag_error(p.err, KVC_ERR_BOUNDS);
+      P[b] = t;
+      sum += t;
+    }
+    int incl = sum;  // inclusive scan across the block
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int* wsum = flags + 4;  // [W]
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += wsum[w];
+    int run = base + incl - sum;
+    for (int b = b_lo; b < b_hi; ++b) {
+      const int t = P[b];
+      P[b] = run;
+      run += t;
+    }
+    if (tid == NTH - 1) P[p.B] = base + incl;
+    __syncthreads();
+  }
+  const long long Wt = P[p.B];
+  const int G = (int)(Wt < (long long)gridDim.x ? Wt : (long long)gridDim.x);
+  if (c >= G) return;
+  const long long lo = (long long)c * Wt / G;
+  const long long hi = (long long)(c + 1) * Wt / G;
+  const int ntiles = (int)(hi - lo);
+
+  // starting position: request (binary search), KV head, row block
+  TileCursor<R> cur;
+  {
+    int a = 0, z = p.B;  // largest b with P[b] <= lo
+    while (z - a > 1) {
+      const int mid = (a + z) >> 1;
+      if (P[mid] <= lo) a = mid;
+      else z = mid;
+    }
+    while (P[a + 1] == P[a]) ++a;  // skip requests with no tiles
+    cur.b = a;
+    cur.L = p.seq_lens[a];
+    int local = (int)(lo - P[a]);
+    const int per_g = (P[a + 1] - P[a]) / p.H_kv;
+    cur.g = local / per_g;
+    local -= cur.g * per_g;
+    cur.rb = 0;
+    while (true) {
+      const int t = ceil_div(cur.L + row_block(cur.rb, R, p.rows, p.T_new).imax + 1, 64);
+      if (local < t) {
+        cur.seg_tiles = t;
+        break;
+      }
+      local -= t;
+      ++cur.rb;
+    }
+    cur.k = local;
+    cur.seg_start = lo - local;
+  }
+  __syncthreads();  // P is dead: the ring may now be filled
+
+  if (tid == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+#pragma unroll
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], W);
+    }
+    flags[0] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // ------------------------------------------------------- tile producer
+  const bool producer = (tid == 0);
+  const uint64_t pol = l2_policy_evict_first();
+  TileCursor<R> pc = cur;  // producer's own cursor
+  int issued = 0;
+  auto issue = [&]() {
+    const int st = issued % C::kStages;
+    const bool first = (issued == 0) || (pc.k == 0);
+    const int r0 = pc.rb * R;
+    const int nr = min(R, p.rows - r0);
+    const uint32_t qbytes = first ? (uint32_t)nr * D * 2 : 0u;
+    mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes + qbytes);
+    if (first) {
+      const char* qsrc = static_cast<const char*>(p.q) +
+                         ((((size_t)pc.b * p.H_q + (size_t)pc.g * p.group) * p.T_new) + r0) *
+                             D * 2;
+      bulk_g2s(sq + st * R * D * 2, qsrc, qbytes, &full[st]);
+    }
+    unsigned char* dk = sk + st * C::kTileBytes;
+    unsigned char* dv = sv + st * C::kTileBytes;
+    const int t0 = pc.k * C::kTile;
+    if (!PAGED) {
+      const int y = (pc.b * p.H_kv + pc.g) * p.max_T + t0;
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h) {
+        tma_load_2d(dk + h * C::kBoxBytes, &tmk, h * 64, y, &full[st], pol);
+        tma_load_2d(dv + h * C::kBoxBytes, &tmv, h * 64, y, &full[st], pol);
+      }
+    } else {
+      const int Pg = 1 << p.page_shift;
+      const int box_rows = Pg < C::kTile ? Pg : C::kTile;
+      const int n_seg = pc.L + row_block(pc.rb, R, p.rows, p.T_new).imax + 1;
+      const int32_t* bt = p.block_table + (size_t)pc.b * p.max_pages;
+      const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
+#pragma unroll 1
+      for (int t = t0; t < t0 + C::kTile; t += box_rows) {
+        int y = beyond;
+        if (t < n_seg) {
+          const int page = bt[t >> p.page_shift];
+          if (page >= 0 && page < p.num_pages)
+            y = (page * p.H_kv + pc.g) * Pg + (t & (Pg - 1));
+          else
+            flag_error(p.err, KVC_ERR_BOUNDS);
+        }
+        const int off = (t - t0) * 128;
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) {
+          tma_load_2d(dk + h * C::kBoxBytes + off, &tmk, h * 64, y, &full[st], pol);
+          tma_load_2d(dv + h * C::kBoxBytes + off, &tmv, h * 64, y, &full[st], pol);
+        }
+      }
+    }
+    ++issued;
+    pc.next(p, PAGED);
+  };
+  if (producer)
+    while (issued < min(C::kStages, ntiles)) issue();
+
+  // Bounded waits that keep every thread on the same control path: a wait that
+  // runs out flags the error and the CTA abort word, and from then on waits
+  // return at once; the CTA finishes its loop (on garbage) instead of
+  // stranding threads at a named barrier.
+  volatile int* abort_word = flags;
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*abort_word) return false;
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t_start = global_timer_ns();
+#pragma unroll 1
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (*abort_word) return false;
+      if (global_timer_ns() - t_start > kWaitLimitNs) {
+        flag_error(p.err, KVC_ERR_TIMEOUT);
+        *abort_word = 1;
+        return false;
+      }
+    }
+  };
+
+  // ------------------------------------------------------------- consumers
+  const int mi = lane >> 3;
+  const int wrow = warp * 16;
+  const int k_row = wrow + (mi & 1) * 8 + (lane & 7);
+  const int k_cs = mi >> 1;
+  const int v_row = wrow + (mi >> 1) * 8 + (lane & 7);
+  const int v_cs = mi & 1;
+  const uint32_t sk_addr = smem_addr(sk);
+  const uint32_t sv_addr = smem_addr(sv);
+
+  uint32_t qb[C::kKSteps][NT][2];
+  int vis[NT][2];
+  int r0 = 0, nr = 0, vis_min = 0, piece_first_j = 0;
+  float m[NT][2], l[NT][2];
+  float o[C::kMTiles][NT][4];
+
+#pragma unroll 1
+  for (int j = 0; j < ntiles; ++j) {
+    const int st = j % C::kStages;
+    if (producer && j >= 1 && issued < ntiles) {
+      wait(&empty[(j - 1) % C::kStages], ((j - 1) / C::kStages) & 1);
+      issue();
+    }
+    wait(&full[st], (j / C::kStages) & 1);
+
+    if (j == 0 || cur.k == 0) {  // a new piece: its q rows, visibility, fresh state
+      piece_first_j = j;
+      r0 = cur.rb * R;
+      nr = min(R, p.rows - r0);
+      vis_min = cur.L + row_block(cur.rb, R, p.rows, p.T_new).imin + 1;
+      const unsigned char* qs = sq + st * R * D * 2;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int row = nt * 8 + (lane >> 2);
+#pragma unroll
+        for (int kk = 0; kk < C::kKSteps; ++kk) {
+          if (row < nr) {
+            const unsigned char* src = qs + row * D * 2 + (kk * 16 + (lane & 3) * 2) * 2;
+            qb[kk][nt][0] = *reinterpret_cast<const uint32_t*>(src);
+            qb[kk][nt][1] = *reinterpret_cast<const uint32_t*>(src + 16);
+          } else {
+            qb[kk][nt][0] = 0u;
+            qb[kk][nt][1] = 0u;
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int rr = nt * 8 + (lane & 3) * 2 + cc;
+          vis[nt][cc] = rr < nr ? cur.L + (r0 + rr) % p.T_new + 1 : 0;
+          m[nt][cc] = -INFINITY;
+          l[nt][cc] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+      }
+    }
+
+    const uint32_t kb = sk_addr + st * C::kTileBytes;
+    const uint32_t vb = sv_addr + st * C::kTileBytes;
+    const int t0 = cur.k * C::kTile;
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < C::kKSteps; ++kk) {
+      uint32_t a[4];
+      ldmatrix_x4(a, kb + swz<D>(k_row, 2 * kk + k_cs));
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_16816<T>(sacc[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+    }
+    const int tok0 = t0 + wrow + (lane >> 2);
+    const bool unmasked = (t0 + C::kTile <= vis_min);
+    bool grew = false;
+    float alpha[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float s0 = sacc[nt][cc] * p.scale_log2;
+        float s1 = sacc[nt][2 + cc] * p.scale_log2;
+        if (!unmasked) {
+          s0 = (tok0 < vis[nt][cc]) ? s0 : -INFINITY;
+          s1 = (tok0 + 8 < vis[nt][cc]) ? s1 : -INFINITY;
+        }
+        float mx = fmaxf(s0, s1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m[nt][cc], mx);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[nt][cc] = exp2f(m[nt][cc] - mu);
+        grew |= (m_new > m[nt][cc]);
+        m[nt][cc] = m_new;
+        const float p0 = exp2f(s0 - mu);
+        const float p1 = exp2f(s1 - mu);
+        l[nt][cc] = fmaf(l[nt][cc], alpha[nt][cc], p0 + p1);
+        sacc[nt][cc] = p0;
+        sacc[nt][2 + cc] = p1;
+      }
+    }
+    if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+      for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          o[mt][nt][0] *= alpha[nt][0];
+          o[mt][nt][1] *= alpha[nt][1];
+          o[mt][nt][2] *= alpha[nt][0];
+          o[mt][nt][3] *= alpha[nt][1];
+        }
+    }
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      pb[nt][0] = movmatrix_trans(Elt<T>::pack2(sacc[nt][0], sacc[nt][1]));
+      pb[nt][1] = movmatrix_trans(Elt<T>::pack2(sacc[nt][2], sacc[nt][3]));
+    }
+#pragma unroll
+    for (int mt = 0; mt < C::kMTiles; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a, vb + swz<D>(v_row, 2 * mt + v_cs));
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+    }
+
+    const bool piece_end = (j == ntiles - 1) || (cur.k == cur.seg_tiles - 1);
+    if (!piece_end) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      cur.next(p, PAGED);
+      continue;
+    }
+
+    // -------------------------------------------- end of a segment piece
+    // The four warps merge inside this stage's K/V buffers (every warp is
+    // done reading them after the barrier); other stages keep streaming.
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        l[nt][cc] += __shfl_xor_sync(0xffffffffu, l[nt][cc], 4);
+        l[nt][cc] += __shfl_xor_sync(0xffffffffu, l[nt][cc], 8);
+        l[nt][cc] += __shfl_xor_sync(0xffffffffu, l[nt][cc], 16);
+      }
+    named_barrier_sync(1, NTH);
+    float* red_acc = reinterpret_cast<float*>(sk + st * C::kTileBytes);
+    float* red_acc_hi = reinterpret_cast<float*>(sv + st * C::kTileBytes);
+    auto acc_at = [&](int w, int row, int d) -> float* {
+      // W*R*D floats spread over this stage's K then V buffers
+      const int idx = (w * R + row) * D + d;
+      constexpr int kHalfFloats = C::kTileBytes / 4;
+      return idx < kHalfFloats ? red_acc + idx : red_acc_hi + (idx - kHalfFloats);
+    };
+#pragma unroll
+    for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = nt * 8 + (lane & 3) * 2 + (e & 1);
+          const int d = mt * 16 + (lane >> 2) + (e >> 1) * 8;
+          *acc_at(warp, row, d) = o[mt][nt][e];
+        }
+    if (lane < 4) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int row = nt * 8 + lane * 2 + cc;
+          red_m[warp * R + row] = m[nt][cc];
+          red_l[warp * R + row] = l[nt][cc];
+        }
+    }
+    named_barrier_sync(1, NTH);
+
+    const bool whole = (piece_first_j == j - cur.k) && (cur.k == cur.seg_tiles - 1);
+    const int slot = (piece_first_j == 0) ? 0 : 1;
+    T* out = static_cast<T*>(p.out);
+    const size_t row_base =
+        ((size_t)cur.b * p.H_q + (size_t)cur.g * p.group) * p.T_new + r0;
+    float* wso = p.ws_o + ((size_t)c * 2 + slot) * R * D;
+    float* wsl = p.ws_lse + ((size_t)c * 2 + slot) * R;
+#pragma unroll 1
+    for (int idx = tid; idx < R * D; idx += NTH) {
+      const int rr = idx / D;
+      const int d = idx - rr * D;
+      if (rr >= nr) break;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W; ++w) M = fmaxf(M, red_m[w * R + rr]);
+      float lsum = 0.f, ov = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          const float f = exp2f(red_m[w * R + rr] - M);
+          lsum = fmaf(red_l[w * R + rr], f, lsum);
+          ov = fmaf(*acc_at(w, rr, d), f, ov);
+        }
+      }
+      if (whole) {
+        store_elt<T>(out + (row_base + rr) * D + d, ov / lsum);
+      } else {
+        wso[rr * D + d] = M == -INFINITY ? 0.f : ov / lsum;
+        if (d == 0) wsl[rr] = M == -INFINITY ? -INFINITY : M + log2f(lsum);
+      }
+    }
+    if (!whole) {
+      // hand the piece to the segment's last finisher
+      __threadfence();
+      named_barrier_sync(1, NTH);
+      const long long s0 = cur.seg_start, s1 = cur.seg_start + cur.seg_tiles - 1;
+      const int cf = (int)(((s0 + 1) * G - 1) / Wt);  // CTA holding the segment's first tile
+      const int cl = (int)(((s1 + 1) * G - 1) / Wt);
+      int* ticket = p.counters + ((size_t)cur.b * p.H_kv + cur.g) * p.row_blocks + cur.rb;
+      if (tid == 0) flags[1] = (atomicAdd(ticket, 1) == cl - cf);
+      named_barrier_sync(1, NTH);
+      if (flags[1]) {
+        __threadfence();
+        const bool cf_mid = ((long long)cf * Wt / G) < s0;  // cf began in an earlier segment
+#pragma unroll 1
+        for (int idx = tid; idx < R * D; idx += NTH) {
+          const int rr = idx / D;
+          const int d = idx - rr * D;
+          if (rr >= nr) break;
+          float M = -INFINITY;
+          for (int cc = cf; cc <= cl; ++cc) {
+            const int sl = (cc == cf && cf_mid) ? 1 : 0;
+            M = fmaxf(M, __ldcg(p.ws_lse + ((size_t)cc * 2 + sl) * R + rr));
+          }
+          float den = 0.f, ov = 0.f;
+          for (int cc = cf; cc <= cl; ++cc) {
+            const int sl = (cc == cf && cf_mid) ? 1 : 0;
+            const float ls = __ldcg(p.ws_lse + ((size_t)cc * 2 + sl) * R + rr);
+            const float w = (ls == -INFINITY) ? 0.f : exp2f(ls - M);
+            den += w;
+            ov = fmaf(w, __ldcg(p.ws_o + (((size_t)cc * 2 + sl) * R + rr) * D + d), ov);
+          }
+          store_elt<T>(out + (row_base + rr) * D + d, ov / den);
+        }
+        if (tid == 0) *ticket = 0;
+      }
+    }
+    named_barrier_sync(1, NTH);  // the stage's buffers are free again
+    if (lane == 0) mbar_arrive(&empty[st]);
+    cur.next(p, PAGED);
+  }
+  // After an abort, do not retire while copies may still be landing.
+  if (producer && *abort_word)
+#pragma unroll 1
+    for (int j = max(0, issued - C::kStages); j < issued; ++j)
+      if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.err)) break;
+}
+
+}  // namespace kvc

@@ -13,6 +13,7 @@
 #include "append.cuh"
 #include "attend_decode.cuh"
 #include "attend_mma.cuh"
+#include "attend_streamk.cuh"
 #include "kvc.h"
 
 struct kvc_cache {
@@ -22,8 +23,10 @@ struct kvc_cache {
   size_t layer_bytes;  // one layer's K (equally V) pool
   char* pool;          // layers x {K, V}
   int* d_err;
-  float* ws;           // split-K workspace: partial outputs, lse, slice tickets
+  float* ws;           // split-K workspace: partial outputs and lse
   size_t ws_bytes;
+  int* tickets;        // slice tickets, zero between launches (own allocation, so that
+  size_t n_tickets;    // partial layouts of different plans can never overwrite them)
   bool tma;                        // tensor maps built: the tensor-core path is available
   std::vector<CUtensorMap> tmk;    // per layer: K pool as a 2-D (rows, D) tensor
   std::vector<CUtensorMap> tmv;
@@ -153,6 +156,37 @@ int mma_occ(int D, int NT, bool paged) {
   return paged ? mma_occ_nt<128, T, true>(NT) : mma_occ_nt<128, T, false>(NT);
 }
 
+template <int D, int NT, typename T, bool PAGED>
+int streamk_occupancy() {
+  static int occ = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const size_t smem = kvc::StreamKCfg<D>::template smem_bytes<NT>();
+    cudaFuncSetAttribute(kvc::attend_streamk_kernel<D, NT, T, PAGED>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kvc::attend_streamk_kernel<D, NT, T, PAGED>, kvc::StreamKCfg<D>::kThreads,
+            smem) != cudaSuccess)
+      n = 1;
+    occ = std::max(1, n);
+  });
+  return occ;
+}
+
+template <typename T>
+int streamk_occ(int D, int NT, bool paged) {
+  if (D == 64)
+    return paged ? (NT == 1 ? streamk_occupancy<64, 1, T, true>()
+                            : streamk_occupancy<64, 2, T, true>())
+                 : (NT == 1 ? streamk_occupancy<64, 1, T, false>()
+                            : streamk_occupancy<64, 2, T, false>());
+  return paged ? (NT == 1 ? streamk_occupancy<128, 1, T, true>()
+                          : streamk_occupancy<128, 2, T, true>())
+               : (NT == 1 ? streamk_occupancy<128, 1, T, false>()
+                          : streamk_occupancy<128, 2, T, false>());
+}
+
 int mma_scratch_floats(int D, int NT) {
   if (D == 64)
     return NT == 1 ? kvc::MmaCfg<64>::scratch_floats<1>()
@@ -166,6 +200,8 @@ int mma_scratch_floats(int D, int NT) {
 // ------------------------------------------------------------ attend plan
 struct Plan {
   bool mma;          // tensor-core kernel (else the CUDA-core kernel)
+  bool streamk;      // mma: persistent stream-K kernel (grid = resident CTAs)
+  int grid;          // streamk: persistent CTAs
   int NT;            // mma: 8-row n-tiles per CTA
   int R;             // query rows per CTA
   int row_blocks;    // CTAs per KV head along the rows
@@ -243,6 +279,22 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
     occ = occupancy(c, pl.R);
   }
   pl.row_blocks = kvc::ceil_div(rows, pl.R);
+  // Persistent stream-K for up to 16 rows per KV head: the per-CTA partial
+  // slots need no split size and every CTA streams the same bytes.
+  const int max_batch = c->D == 64 ? kvc::StreamKCfg<64>::kMaxBatch
+                                   : kvc::StreamKCfg<128>::kMaxBatch;
+  if (pl.mma && pl.NT <= 2 && c->B <= max_batch) {
+    pl.streamk = true;
+    const int socc = c->dtype == KVC_BF16 ? streamk_occ<__nv_bfloat16>(c->D, pl.NT, c->paged)
+                                          : streamk_occ<__half>(c->D, pl.NT, c->paged);
+    pl.grid = c->num_sms * socc;
+    pl.split_tokens = 1 << 30;  // unused by the stream-K kernel
+    pl.num_splits = 1;
+    pl.ws_partial_floats = (size_t)pl.grid * 2 * pl.R * (c->D + 1);
+    pl.ws_counters = (size_t)c->B * c->H_kv * pl.row_blocks;
+    pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
+    return pl;
+  }
   long long cap = c->max_T;
   if (c->paged) cap = std::min<long long>(cap, (long long)max_pages * c->page_size);
   cap = std::max<long long>(cap, 1);
@@ -258,12 +310,32 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
   pl.num_splits = (int)ns;
   pl.ws_partial_floats = ns > 1 ? (size_t)c->B * H_q * T_new * ns * (c->D + 1) : 0;
   pl.ws_counters = ns > 1 ? (size_t)c->B * c->H_kv * pl.row_blocks : 0;
-  pl.ws_bytes = pl.ws_partial_floats * sizeof(float) + pl.ws_counters * sizeof(int);
+  pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
   return pl;
 }
 
-// Grow the workspace to `bytes` (zero-filled: slice tickets must start at 0).
-kvc_status ensure_workspace(kvc_cache* c, size_t bytes) {
+// Grow the tickets to `n` (zero-filled) and the partial workspace to `bytes`.
+kvc_status ensure_workspace(kvc_cache* c, size_t bytes, size_t n) {
+  if (n > c->n_tickets) {
+    if (c->tickets) {
+      cudaError_t e = cudaFree(c->tickets);  // synchronises
+      c->tickets = nullptr;
+      c->n_tickets = 0;
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+    void* t = nullptr;
+    if (cudaMalloc(&t, n * sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      return KVC_ERR_OOM;
+    }
+    if (cudaMemset(t, 0, n * sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(t);
+      return KVC_ERR_CUDA;
+    }
+    c->tickets = static_cast<int*>(t);
+    c->n_tickets = n;
+  }
   if (bytes <= c->ws_bytes) return KVC_OK;
   if (c->ws) {
     cudaError_t e = cudaFree(c->ws);  // synchronises: no launch still reads it
@@ -276,11 +348,6 @@ kvc_status ensure_workspace(kvc_cache* c, size_t bytes) {
   if (e != cudaSuccess) {
     cudaGetLastError();
     return KVC_ERR_OOM;
-  }
-  if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(p);
-    return KVC_ERR_CUDA;
   }
   c->ws = static_cast<float*>(p);
   c->ws_bytes = bytes;
@@ -317,6 +384,33 @@ kvc_status dispatch_mma(const kvc::AttendParams& p, int D, int NT, bool paged,
                  : dispatch_mma_nt<64, T, false>(p, NT, tk, tv, s);
   return paged ? dispatch_mma_nt<128, T, true>(p, NT, tk, tv, s)
                : dispatch_mma_nt<128, T, false>(p, NT, tk, tv, s);
+}
+
+template <int D, int NT, typename T, bool PAGED>
+kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, cudaStream_t stream) {
+  using C = kvc::StreamKCfg<D>;
+  streamk_occupancy<D, NT, T, PAGED>();  // sets the shared-memory attribute once
+  const size_t smem = C::template smem_bytes<NT>();
+  kvc::attend_streamk_kernel<D, NT, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p, tk, tv);
+  return cuda_status(cudaGetLastError());
+}
+
+template <typename T>
+kvc_status dispatch_streamk(const kvc::AttendParams& p, int D, int NT, bool paged, int grid,
+                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  if (D == 64) {
+    if (paged)
+      return NT == 1 ? launch_attend_streamk<64, 1, T, true>(p, grid, tk, tv, s)
+                     : launch_attend_streamk<64, 2, T, true>(p, grid, tk, tv, s);
+    return NT == 1 ? launch_attend_streamk<64, 1, T, false>(p, grid, tk, tv, s)
+                   : launch_attend_streamk<64, 2, T, false>(p, grid, tk, tv, s);
+  }
+  if (paged)
+    return NT == 1 ? launch_attend_streamk<128, 1, T, true>(p, grid, tk, tv, s)
+                   : launch_attend_streamk<128, 2, T, true>(p, grid, tk, tv, s);
+  return NT == 1 ? launch_attend_streamk<128, 1, T, false>(p, grid, tk, tv, s)
+                 : launch_attend_streamk<128, 2, T, false>(p, grid, tk, tv, s);
 }
 
 template <int D, int R, typename T, bool PAGED>
@@ -453,6 +547,7 @@ kvc_status kvc_destroy(kvc_cache* c) {
   cudaFree(c->pool);
   cudaFree(c->d_err);
   if (c->ws) cudaFree(c->ws);
+  if (c->tickets) cudaFree(c->tickets);
   delete c;
   return cuda_status(e);
 }
@@ -516,15 +611,16 @@ kvc_status kvc_plan_splits(const kvc_cache* c, int H_q, int T_new, int max_pages
   if (!c || H_q <= 0 || T_new <= 0 || H_q % c->H_kv != 0) return KVC_ERR_INVALID_ARG;
   if (c->paged && max_pages <= 0) return KVC_ERR_INVALID_ARG;
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
-  if (num_splits) *num_splits = pl.num_splits;
-  if (split_tokens) *split_tokens = pl.split_tokens;
+  if (num_splits) *num_splits = pl.streamk ? pl.grid : pl.num_splits;
+  if (split_tokens) *split_tokens = pl.streamk ? 0 : pl.split_tokens;
   return KVC_OK;
 }
 
 kvc_status kvc_reserve(kvc_cache* c, int H_q, int T_new, int max_pages) {
   if (!c || H_q <= 0 || T_new <= 0 || H_q % c->H_kv != 0) return KVC_ERR_INVALID_ARG;
   if (c->paged && max_pages <= 0) return KVC_ERR_INVALID_ARG;
-  return ensure_workspace(c, make_plan(c, H_q, T_new, max_pages).ws_bytes);
+  const Plan pl = make_plan(c, H_q, T_new, max_pages);
+  return ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
 }
 
 kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new,
@@ -540,7 +636,7 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
   if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
-  kvc_status st = ensure_workspace(c, pl.ws_bytes);
+  kvc_status st = ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
   if (st != KVC_OK) return st;
   kvc::AttendParams p{};
   p.k_pool = kvc_k_pool(c, layer);
@@ -564,10 +660,18 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   p.num_splits = pl.num_splits;
   p.row_blocks = pl.row_blocks;
   p.ws_o = c->ws;
-  p.ws_lse = c->ws ? c->ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D : nullptr;
-  p.counters = c->ws ? reinterpret_cast<int*>(c->ws + pl.ws_partial_floats) : nullptr;
+  p.ws_lse = !c->ws ? nullptr
+             : pl.streamk ? c->ws + (size_t)pl.grid * 2 * pl.R * c->D
+                          : c->ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
+  p.counters = c->tickets;
   p.err = c->d_err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.streamk)
+    return c->dtype == KVC_BF16
+               ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
+                                                 c->tmk[layer], c->tmv[layer], s)
+               : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
+                                          c->tmv[layer], s);
   if (pl.mma)
     return c->dtype == KVC_BF16
                ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
@@ -587,7 +691,8 @@ kvc_status kvc_get_error(kvc_cache* c) {
   if (h != 0) {
     if (cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess) return KVC_ERR_CUDA;
     // A launch that gave up may have left slice tickets behind: clear them all.
-    if (c->ws && cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) return KVC_ERR_CUDA;
+    if (c->tickets && cudaMemset(c->tickets, 0, c->n_tickets * sizeof(int)) != cudaSuccess)
+      return KVC_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return KVC_ERR_CUDA;
   }
   return static_cast<kvc_status>(h);

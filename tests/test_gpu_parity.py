@@ -320,3 +320,27 @@ def test_kv_bytes_of_a_cache_follows_the_formula():
         assert c.nbytes == kvc.kvc_bytes_formula(1, 8, 128, 16 * 1000, 2, 1)
     finally:
         c.close()
+
+
+def test_alternating_plans_share_one_cache():
+    """Decode (persistent stream-K), a 32-row verify chunk (fixed split-K) and decode
+    again on the same cache: each kernel's slice tickets must be left clean for the next."""
+    import oracle
+    base = W.paged_case("alt", 6, 32, 8, 128, "bf16", 8, 300, 6000, 16, seed=31, pool_seed=32)
+    g = H.GpuRun(base)
+    try:
+        kp, vp = base.k_pool(0), base.v_pool(0)
+        g.load_pools(0, kp, vp)
+        o = oracle.get()
+        vis = base.seq_lens.astype(np.int64) + base.T_new
+        K = o.gather_paged(kp, base.block_table, vis, int(vis.max()))
+        V = o.gather_paged(vp, base.block_table, vis, int(vis.max()))
+        for T_new in (1, 8, 1, 4, 1):
+            q = W.normal_bits((base.B, base.H_q, T_new, base.D), "bf16", 31, "alt_q", T_new)
+            out = g.cache.attend(0, H.to_device(q, "bf16"), g.seq_lens, g.block_table,
+                                 scale=base.scale)
+            assert g.cache.get_error() == kvc.KVC_OK
+            ref = o.attend(q, K, V, base.seq_lens, base.scale, oracle.BF16)
+            H.compare(H.out_to_f64(out), ref, f"T_new={T_new}")
+    finally:
+        g.close()
