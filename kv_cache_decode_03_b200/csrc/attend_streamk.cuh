@@ -33,6 +33,10 @@
 #include "params.cuh"
 #include "splitk_epilogue.cuh"
 
+#ifndef KVC_SK_STAGES
+#define KVC_SK_STAGES 3
+#endif
+
 namespace kvc {
 
 template <int D>
@@ -43,7 +47,7 @@ struct StreamKCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = kTile * 128;
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStages = 3;
+  static constexpr int kStages = KVC_SK_STAGES;
   static constexpr int kKSteps = D / 16;
   static constexpr int kMTiles = D / 16;
   static constexpr int kRing = 2 * kStages * kTileBytes;

@@ -38,6 +38,12 @@ namespace {
 
 constexpr int kEltBytes = 2;
 
+// TMA L2 promotion: a 128-byte box column pulls the neighbouring half of the
+// 256-byte K/V row into L2, where the other column's load finds it.
+#ifndef KVC_TMA_L2_PROMOTION
+#define KVC_TMA_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
 // Split-K sizing: aim for this many waves of resident CTAs, so that the last
 // wave's imbalance is a small fraction of the pass.
 #ifndef KVC_SPLIT_WAVES
@@ -98,7 +104,7 @@ bool make_tmap(CUtensorMap* m, void* base, kvc_dtype dtype, int D, long long row
                         dtype == KVC_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                         2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_SWIZZLE_128B, KVC_TMA_L2_PROMOTION,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
