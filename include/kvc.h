@@ -62,7 +62,8 @@ typedef enum {
     KVC_ERR_OOM = 3,         /* device allocation failed */
     KVC_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch error, no device) */
     KVC_ERR_BOUNDS = 5,      /* device side: page id or position outside the cache */
-    KVC_ERR_TIMEOUT = 6      /* device side: a bounded pipeline wait gave up */
+    KVC_ERR_TIMEOUT = 6,     /* device side: a bounded pipeline wait gave up */
+    KVC_ERR_SCRATCH = 7      /* kvc_attend_noalloc: the call needs more than its fixed scratch */
 } kvc_status;
 
 typedef enum { KVC_FP16 = 0, KVC_BF16 = 1 } kvc_dtype;
@@ -128,6 +129,28 @@ kvc_status kvc_append(kvc_cache* cache, int layer, const void* k_new, const void
 kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
                       const int32_t* block_table, int max_pages, const int32_t* seq_lens,
                       float scale, void* out, void* stream);
+
+/*
+ * kvc_attend_noalloc -- kvc_attend without any device allocation.  The pages have no
+ * counterpart of this call: it exists for callers that cannot let a library allocate
+ * device memory -- code recording a step inside CUDA stream capture (cudaMalloc cannot
+ * be captured), engines whose caching allocator owns almost all device memory (a side
+ * allocation can fail or fragment its pool), and latency-bound loops that cannot afford
+ * the device synchronisation that cudaFree implies.
+ *   Arguments, layouts and results are those of kvc_attend.  The split-K scratch
+ *   (partial results and slice tickets) lives in one fixed 16 MiB device array that the
+ *   library holds on every GPU that loads it, until the process exits.  A call whose plan
+ *   needs more scratch than that returns KVC_ERR_SCRATCH before launching anything
+ *   (decode with up to 16 query rows per KV head needs about 2.5 MB on a 148-SM B200).
+ *   The first call on a device looks up the array's device address (once per device);
+ *   make that first call before any stream capture.  Each call clears the tickets it
+ *   uses with an asynchronous memset on `stream`.  Every call shares the one array, so
+ *   calls whose executions overlap on the GPU (other streams, other threads, other cache
+ *   handles on the same device) race with each other and must be serialised by the caller.
+ */
+kvc_status kvc_attend_noalloc(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
+                              const int32_t* block_table, int max_pages,
+                              const int32_t* seq_lens, float scale, void* out, void* stream);
 
 /*
  * kvc_reserve -- size the attend workspace for up to `H_q` query heads, `T_new` new rows

@@ -24,6 +24,7 @@ KVC_ERR_OOM = 3
 KVC_ERR_CUDA = 4
 KVC_ERR_BOUNDS = 5
 KVC_ERR_TIMEOUT = 6
+KVC_ERR_SCRATCH = 7
 
 KVC_FP16 = 0
 KVC_BF16 = 1
@@ -58,6 +59,7 @@ def library() -> ctypes.CDLL:
         "kvc_bytes_formula": ([I, I, I, LL, I, I], SZ),
         "kvc_append": ([P, I, P, P, I, P, I, P, P], I),
         "kvc_attend": ([P, I, P, I, I, P, I, P, F, P, P], I),
+        "kvc_attend_noalloc": ([P, I, P, I, I, P, I, P, F, P, P], I),
         "kvc_reserve": ([P, I, I, I], I),
         "kvc_get_error": ([P], I),
         "kvc_status_string": ([I], ctypes.c_char_p),
@@ -120,6 +122,16 @@ def kvc_attend(cache: int, layer: int, q: int, H_q: int, T_new: int, block_table
                max_pages: int, seq_lens: int, scale: float, out: int, stream: int) -> None:
     _check(library().kvc_attend(cache, layer, q, H_q, T_new, block_table or None, max_pages,
                                 seq_lens, scale, out, stream or None), "kvc_attend")
+
+
+def kvc_attend_noalloc(cache: int, layer: int, q: int, H_q: int, T_new: int, block_table: int,
+                       max_pages: int, seq_lens: int, scale: float, out: int,
+                       stream: int) -> None:
+    """kvc_attend with its split-K scratch in the library's fixed device array (no
+    device allocation; see include/kvc.h for who needs this and the limits)."""
+    _check(library().kvc_attend_noalloc(cache, layer, q, H_q, T_new, block_table or None,
+                                        max_pages, seq_lens, scale, out, stream or None),
+           "kvc_attend_noalloc")
 
 
 def kvc_reserve(cache: int, H_q: int, T_new: int, max_pages: int = 0) -> None:

@@ -465,6 +465,7 @@ const char* kvc_status_string(kvc_status s) {
     case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
     case KVC_ERR_BOUNDS: return "KVC_ERR_BOUNDS";
     case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT";
+    case KVC_ERR_SCRATCH: return "KVC_ERR_SCRATCH";
   }
   return "KVC_ERR_UNKNOWN";
 }
@@ -705,3 +706,109 @@ kvc_status kvc_get_error(kvc_cache* c) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free attend.
+//
+// Some callers cannot let a library allocate device memory: code that records
+// a decode step inside CUDA stream capture (cudaMalloc is not a capturable
+// operation), engines whose caching allocator owns nearly all of the device's
+// memory (a side allocation can fail or fragment its pool), and latency-bound
+// serving loops that cannot afford the device synchronisation cudaFree implies.
+// For them kvc_attend_noalloc runs the same kernels as kvc_attend with the
+// split-K scratch (partial results and slice tickets) in the fixed-size device
+// array below instead of the cache's growable workspace.
+static constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB on every device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static constexpr int kNoAllocMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device: looked up once per
+// device (the array's name is only a host-side stand-in in host code).
+static kvc_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+    cudaGetLastError();
+    return KVC_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return KVC_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return KVC_OK;
+}
+
+extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q, int H_q,
+                                         int T_new, const int32_t* block_table, int max_pages,
+                                         const int32_t* seq_lens, float scale, void* out,
+                                         void* stream) {
+  if (!c || layer < 0 || layer >= c->num_layers || T_new <= 0 || H_q <= 0 ||
+      H_q % c->H_kv != 0)
+    return KVC_ERR_INVALID_ARG;
+  if (!q || !out || !seq_lens || !aligned16(q) || !aligned16(out) || !aligned4(seq_lens))
+    return KVC_ERR_INVALID_ARG;
+  if (c->paged && (!block_table || !aligned4(block_table) || max_pages <= 0))
+    return KVC_ERR_INVALID_ARG;
+  if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
+  if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c, H_q, T_new, max_pages);
+  // [tickets, padded to 256 bytes][partial outputs][lse]
+  const size_t ticket_bytes = (pl.ws_counters * sizeof(int) + 255) & ~size_t(255);
+  if (ticket_bytes + pl.ws_bytes > kNoAllocScratchBytes) return KVC_ERR_SCRATCH;
+  void* base = nullptr;
+  kvc_status st = noalloc_scratch(&base);
+  if (st != KVC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents; tickets must start at zero.
+  if (pl.ws_counters &&
+      cudaMemsetAsync(base, 0, pl.ws_counters * sizeof(int), s) != cudaSuccess)
+    return cuda_status(cudaGetLastError());
+  float* ws = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + ticket_bytes);
+  kvc::AttendParams p{};
+  p.k_pool = kvc_k_pool(c, layer);
+  p.v_pool = kvc_v_pool(c, layer);
+  p.q = q;
+  p.out = out;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.max_pages = max_pages;
+  p.B = c->B;
+  p.H_q = H_q;
+  p.H_kv = c->H_kv;
+  p.T_new = T_new;
+  p.group = H_q / c->H_kv;
+  p.rows = p.group * T_new;
+  p.max_T = c->max_T;
+  p.page_shift = c->page_shift;
+  p.num_pages = c->num_pages;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.split_tokens = pl.split_tokens;
+  p.num_splits = pl.num_splits;
+  p.row_blocks = pl.row_blocks;
+  p.ws_o = ws;
+  p.ws_lse = pl.streamk ? ws + (size_t)pl.grid * 2 * pl.R * c->D
+                        : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
+  p.counters = static_cast<int*>(base);
+  p.err = c->d_err;
+  if (pl.streamk)
+    return c->dtype == KVC_BF16
+               ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
+                                                 c->tmk[layer], c->tmv[layer], s)
+               : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
+                                          c->tmv[layer], s);
+  if (pl.mma)
+    return c->dtype == KVC_BF16
+               ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
+                                             c->tmv[layer], s)
+               : dispatch_mma<__half>(p, c->D, pl.NT, c->paged, c->tmk[layer], c->tmv[layer], s);
+  return c->dtype == KVC_BF16 ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
+                              : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
+}
