@@ -40,6 +40,29 @@ import workloads as W  # noqa: E402
 METRIC = ("decode-attention KV HBM GB/s (% of B200 peak) and tokens/s per layer-step")
 
 
+def kernel_source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "kv_cache_decode_03_b200" / "csrc").glob("*")):
+        h.update(f.name.encode())
+        h.update(f.read_bytes())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if its sources still match."""
+    sha = kernel_source_sha256()
+    for f in sorted((ROOT / "profiles").glob("*.md")):
+        kv = {}
+        for line in f.read_text().splitlines():
+            if ":" in line and not line.startswith(("|", " ", "#")):
+                k, _, v = line.partition(":")
+                kv[k.strip()] = v.strip()
+        if kv.get("kernel") == kernel and kv.get("source_sha256") == sha:
+            return int(kv["dram_bytes_per_launch"])
+    return None
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -342,6 +365,7 @@ def run_kvc(args, case: W.Case) -> None:
     peak, peak_kind = peaks()
     tok_layer_step = world * c.B * c.T_new / (ms * 1e-3 / c.layers)
 
+    traffic = profiled_traffic(f"attend_streamk_kernel<{c.D},1,{c.dtype},contiguous>")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(c)
@@ -366,8 +390,8 @@ def run_kvc(args, case: W.Case) -> None:
             "tokens_per_s_per_layer_step": tok_layer_step,
             "ms_per_step_eager": ms_eager,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
-                         "kernel": "kvc_attend (split-K attend + LSE combine), per call",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "attend_streamk_kernel: one launch per kvc_attend call (split attend + merge)",
                          "peak_source": peak_kind},
             "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
