@@ -518,38 +518,25 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
       }
     }
     if (!whole) {
-      // hand the piece to the segment's last finisher
-      __threadfence();
+      // hand the piece to the segment's last finisher: the barrier orders every
+      // thread's partial stores before thread 0's fence and ticket
       named_barrier_sync(1, NTH);
       const long long s0 = cur.seg_start, s1 = cur.seg_start + cur.seg_tiles - 1;
-      const int cf = (int)(((s0 + 1) * G - 1) / Wt);  // CTA holding the segment's first tile
-      const int cl = (int)(((s1 + 1) * G - 1) / Wt);
+      RangeMap rm;
+      rm.W = Wt;
+      rm.G = G;
+      const long long rf = rm.of(s0), rl = rm.of(s1);
       int* ticket = p.counters + ((size_t)cur.b * p.H_kv + cur.g) * p.row_blocks + cur.rb;
-      if (tid == 0) flags[1] = (atomicAdd(ticket, 1) == cl - cf);
+      if (tid == 0) {
+        __threadfence();
+        const bool last = atomicAdd(ticket, 1) == (int)(rl - rf);
+        if (last) __threadfence();  // acquire the other pieces before the barrier
+        flags[1] = last;
+      }
       named_barrier_sync(1, NTH);
       if (flags[1]) {
-        __threadfence();
-        const bool cf_mid = ((long long)cf * Wt / G) < s0;  // cf began in an earlier segment
-#pragma unroll 1
-        for (int idx = tid; idx < R * D; idx += NTH) {
-          const int rr = idx / D;
-          const int d = idx - rr * D;
-          if (rr >= nr) break;
-          float M = -INFINITY;
-          for (int cc = cf; cc <= cl; ++cc) {
-            const int sl = (cc == cf && cf_mid) ? 1 : 0;
-            M = fmaxf(M, __ldcg(p.ws_lse + ((size_t)cc * 2 + sl) * R + rr));
-          }
-          float den = 0.f, ov = 0.f;
-          for (int cc = cf; cc <= cl; ++cc) {
-            const int sl = (cc == cf && cf_mid) ? 1 : 0;
-            const float ls = __ldcg(p.ws_lse + ((size_t)cc * 2 + sl) * R + rr);
-            const float w = (ls == -INFINITY) ? 0.f : exp2f(ls - M);
-            den += w;
-            ov = fmaf(w, __ldcg(p.ws_o + (((size_t)cc * 2 + sl) * R + rr) * D + d), ov);
-          }
-          store_elt<T>(out + (row_base + rr) * D + d, ov / den);
-        }
+        merge_pieces<T, D, R, NTH>(p, rm, rf, rl, s0, nr, row_base, red_acc, red_acc_hi,
+                                   C::kTileBytes / 4, [] { named_barrier_sync(1, NTH); });
         if (tid == 0) *ticket = 0;
       }
     }

@@ -208,6 +208,7 @@ struct Plan {
   bool mma;          // tensor-core kernel (else the CUDA-core kernel)
   bool streamk;      // mma: persistent stream-K kernel (grid = resident CTAs)
   int grid;          // streamk: persistent CTAs
+  size_t slots;      // streamk: partial-result slots (R rows x D each) in the workspace
   int NT;            // mma: 8-row n-tiles per CTA
   int R;             // query rows per CTA
   int row_blocks;    // CTAs per KV head along the rows
@@ -294,6 +295,7 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
     const int socc = c->dtype == KVC_BF16 ? streamk_occ<__nv_bfloat16>(c->D, pl.NT, c->paged)
                                           : streamk_occ<__half>(c->D, pl.NT, c->paged);
     pl.grid = c->num_sms * socc;
+    pl.slots = (size_t)pl.grid * 2;
     pl.split_tokens = 1 << 30;  // unused by the stream-K kernel
     pl.num_splits = 1;
     pl.ws_partial_floats = (size_t)pl.grid * 2 * pl.R * (c->D + 1);
@@ -668,7 +670,7 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   p.row_blocks = pl.row_blocks;
   p.ws_o = c->ws;
   p.ws_lse = !c->ws ? nullptr
-             : pl.streamk ? c->ws + (size_t)pl.grid * 2 * pl.R * c->D
+             : pl.streamk ? c->ws + pl.slots * pl.R * c->D
                           : c->ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
   p.counters = c->tickets;
   p.err = c->d_err;
@@ -794,7 +796,7 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
   p.num_splits = pl.num_splits;
   p.row_blocks = pl.row_blocks;
   p.ws_o = ws;
-  p.ws_lse = pl.streamk ? ws + (size_t)pl.grid * 2 * pl.R * c->D
+  p.ws_lse = pl.streamk ? ws + pl.slots * pl.R * c->D
                         : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
   p.counters = static_cast<int*>(base);
   p.err = c->d_err;
