@@ -121,9 +121,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 2)
   // after the tile loop the ring is free: warp partials, then merge weights
   float* red_acc = reinterpret_cast<float*>(smem);
 
-  const int s = blockIdx.x;
-  const int g = blockIdx.y / p.row_blocks;
-  const int rb = blockIdx.y - g * p.row_blocks;
+  // Row blocks vary fastest: the CTAs that read the same K/V slice for
+  // different query rows launch together, so L2 serves all but the first read.
+  const int s = blockIdx.x / p.row_blocks;
+  const int rb = blockIdx.x - s * p.row_blocks;
+  const int g = blockIdx.y;
   const int b = blockIdx.z;
   const int L = p.seq_lens[b];
   const int r0 = rb * R;

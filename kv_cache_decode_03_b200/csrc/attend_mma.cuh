@@ -96,9 +96,11 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
   int* flags = reinterpret_cast<int*>(empty + C::kStages);  // [0] abort, [1] last
   float* red_acc = reinterpret_cast<float*>(smem);         // ring, after the loop
 
-  const int s = blockIdx.x;
-  const int g = blockIdx.y / p.row_blocks;
-  const int rb = blockIdx.y - g * p.row_blocks;
+  // Row blocks vary fastest: the CTAs that read the same K/V slice for
+  // different query rows launch together, so L2 serves all but the first read.
+  const int s = blockIdx.x / p.row_blocks;
+  const int rb = blockIdx.x - s * p.row_blocks;
+  const int g = blockIdx.y;
   const int b = blockIdx.z;
   const int L = p.seq_lens[b];
   const int r0 = rb * R;
@@ -141,7 +143,8 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
 
   // ------------------------------------------------------- tile producer
   const bool producer = (threadIdx.x == 0);
-  const uint64_t pol = l2_policy_evict_first();
+  // K/V read once: evict first; read by several row blocks: keep them in L2
+  const uint64_t pol = p.row_blocks > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
   auto issue = [&](int j) {
     const int st = j % C::kStages;
     const int t0 = t_begin + j * C::kTile;

@@ -369,7 +369,7 @@ kvc_status launch_attend_mma(const kvc::AttendParams& p, const CUtensorMap& tk,
   using C = kvc::MmaCfg<D>;
   mma_occupancy<D, NT, T, PAGED>();  // sets the shared-memory attribute once
   const size_t smem = C::template smem_bytes<NT>();
-  dim3 grid(p.num_splits, p.H_kv * p.row_blocks, p.B);
+  dim3 grid(p.num_splits * p.row_blocks, p.H_kv, p.B);
   kvc::attend_mma_kernel<D, NT, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p, tk, tv);
   return cuda_status(cudaGetLastError());
 }
@@ -426,7 +426,7 @@ kvc_status launch_attend_simt(const kvc::AttendParams& p, cudaStream_t stream) {
   using C = kvc::DecodeCfg<D>;
   simt_occupancy<D, R, T, PAGED>();  // sets the shared-memory attribute once
   const size_t smem = C::template smem_bytes<R>();
-  dim3 grid(p.num_splits, p.H_kv * p.row_blocks, p.B);
+  dim3 grid(p.num_splits * p.row_blocks, p.H_kv, p.B);
   kvc::attend_decode_kernel<D, R, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p);
   return cuda_status(cudaGetLastError());
 }
