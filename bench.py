@@ -222,30 +222,55 @@ def run_reference(args, case: W.Case) -> None:
 # GPU arm
 # ---------------------------------------------------------------------------
 
+class Replicas:
+    """One process per GPU running an independent replica of the step.
+
+    The decode step has no cross-request exchange, so the only collectives are
+    plumbing around the timed region: a barrier on both sides and the max of
+    the ranks' device times (the whole job is as slow as its slowest rank)."""
+
+    def __init__(self, backend: str = "nccl", device=None):
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.device = device
+        self.dist = dist
+        if self.world > 1 and not dist.is_initialized():
+            import datetime
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+    def barrier(self) -> None:
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self) -> None:
+        if self.world > 1 and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
+def whole_job_gbs(world: int, bytes_per_rank_step: int, ms_per_step_max: float) -> float:
+    """Algorithmic bytes of all replicas' steps over the slowest rank's step time."""
+    return world * bytes_per_rank_step / (ms_per_step_max * 1e-3) / 1e9
+
+
 def run_kvc(args, case: W.Case) -> None:
     import torch
-    import torch.distributed as dist
     import kv_cache_decode_03_b200 as kvc
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    reps = Replicas("nccl", torch.device("cuda", local))
+    world, rank = reps.world, reps.rank
+    barrier, max_over_ranks = reps.barrier, reps.max_over_ranks
 
     c = case
     tdt = {"fp16": torch.float16, "bf16": torch.bfloat16}[c.dtype]
@@ -359,7 +384,7 @@ def run_kvc(args, case: W.Case) -> None:
     d2h = ho.numel() * c.elt
 
     step_bytes = c.layers * c.algorithmic_bytes()
-    value = world * step_bytes / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, ms)
     attend_bytes = c.kv_read_bytes() + 2 * c.B * c.H_q * c.T_new * c.D * c.elt
     achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
@@ -393,7 +418,7 @@ def run_kvc(args, case: W.Case) -> None:
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "attend_streamk_kernel: one launch per kvc_attend call (split attend + merge)",
                          "peak_source": peak_kind},
-            "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": whole_job_gbs(world, step_bytes, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
@@ -401,8 +426,7 @@ def run_kvc(args, case: W.Case) -> None:
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    reps.close()
 
 
 WORKLOADS = {
