@@ -2,9 +2,10 @@
 
 Workload (default): 32-layer GQA decode -- B=16 requests, H_q=32, H_kv=8,
 D=128, bf16, contiguous cache, T_past=4096, one new token per request.  A
-step is one decode layer-step for all 32 layers: kvc_append + kvc_attend per
-layer (split-K attend + log-sum-exp combine inside), 8.6 GB of K/V read per
-step, far above the 126 MB L2, so consecutive steps cannot hit in L2.
+step is one decode layer-step for all 32 layers: kvc_append_attend per layer
+(append, split attend and log-sum-exp merge in one launch on the persistent
+path), 8.6 GB of K/V read per step, far above the 126 MB L2, so consecutive
+steps cannot hit in L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvc|reference]
 
@@ -296,10 +297,11 @@ def run_kvc(args, case: W.Case) -> None:
 
     def step(q=qs, k=ks, v=vs, o=outs):
         for layer in range(c.layers):
-            cache.append(layer, k[layer], v[layer], seq, stream=stream)
-            cache.attend(layer, q[layer], seq, scale=scale, out=o[layer], stream=stream)
+            cache.append_attend(layer, k[layer], v[layer], q[layer], seq, scale=scale,
+                                out=o[layer], stream=stream)
 
-    launches_per_step = c.layers * 2  # append + attend (the slice merge is fused)
+    # one launch per layer on the persistent path (append, attend and merge fused)
+    launches_per_step = c.layers * (1 if split_tokens == 0 else 2)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -342,16 +344,16 @@ def run_kvc(args, case: W.Case) -> None:
     e1.synchronize()
     ms_eager = e0.elapsed_time(e1) / max(3, args.steps // 4)
 
-    # ---- per-call attend duration (split-K attend + combine) for the roofline
+    # ---- per-launch duration of the step's kernel (kvc_append_attend) for the roofline
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(c.layers)]
     durs = []
     with torch.cuda.stream(stream):
         for _ in range(max(2, args.steps // 10)):
             for layer in range(c.layers):
-                cache.append(layer, ks[layer], vs[layer], seq, stream=stream)
                 evs[layer][0].record(stream)
-                cache.attend(layer, qs[layer], seq, scale=scale, out=outs[layer], stream=stream)
+                cache.append_attend(layer, ks[layer], vs[layer], qs[layer], seq, scale=scale,
+                                    out=outs[layer], stream=stream)
                 evs[layer][1].record(stream)
             stream.synchronize()
             durs += [a.elapsed_time(b) for a, b in evs]
@@ -385,7 +387,8 @@ def run_kvc(args, case: W.Case) -> None:
 
     step_bytes = c.layers * c.algorithmic_bytes()
     value = whole_job_gbs(world, step_bytes, ms)
-    attend_bytes = c.kv_read_bytes() + 2 * c.B * c.H_q * c.T_new * c.D * c.elt
+    # K/V read + q read + out written + k_new/v_new read + their rows written to the cache
+    attend_bytes = c.algorithmic_bytes() + 2 * c.B * c.H_kv * c.T_new * c.D * c.elt
     achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
     tok_layer_step = world * c.B * c.T_new / (ms * 1e-3 / c.layers)
@@ -416,7 +419,8 @@ def run_kvc(args, case: W.Case) -> None:
             "ms_per_step_eager": ms_eager,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "attend_streamk_kernel: one launch per kvc_attend call (split attend + merge)",
+                         "kernel": "attend_streamk_kernel, fused: one launch per "
+                                   "kvc_append_attend call (append, split attend, merge)",
                          "peak_source": peak_kind},
             "e2e": {"value": whole_job_gbs(world, step_bytes, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -131,6 +131,20 @@ kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T
                       float scale, void* out, void* stream);
 
 /*
+ * kvc_append_attend -- kvc_append followed by kvc_attend for the same new tokens, in
+ * one launch where the kernel allows it ("9. 推理" 9.3: the new token's K/V join the
+ * cache and are attended in the same step).  Arguments are those of the two calls.
+ * With up to 16 query rows per KV head on the tensor-core path the attend kernel itself
+ * writes the new rows into the cache and uses them straight from k_new / v_new; in other
+ * cases the two kernels run back to back on `stream`.  Results (cache contents and out)
+ * are identical to calling kvc_append then kvc_attend.
+ */
+kvc_status kvc_append_attend(kvc_cache* cache, int layer, const void* k_new, const void* v_new,
+                             const void* q, int H_q, int T_new, const int32_t* block_table,
+                             int max_pages, const int32_t* seq_lens, float scale, void* out,
+                             void* stream);
+
+/*
  * kvc_attend_noalloc -- kvc_attend without any device allocation.  The pages have no
  * counterpart of this call: it exists for callers that cannot let a library allocate
  * device memory -- code recording a step inside CUDA stream capture (cudaMalloc cannot

@@ -60,6 +60,7 @@ def library() -> ctypes.CDLL:
         "kvc_append": ([P, I, P, P, I, P, I, P, P], I),
         "kvc_attend": ([P, I, P, I, I, P, I, P, F, P, P], I),
         "kvc_attend_noalloc": ([P, I, P, I, I, P, I, P, F, P, P], I),
+        "kvc_append_attend": ([P, I, P, P, P, I, I, P, I, P, F, P, P], I),
         "kvc_reserve": ([P, I, I, I], I),
         "kvc_get_error": ([P], I),
         "kvc_status_string": ([I], ctypes.c_char_p),
@@ -122,6 +123,14 @@ def kvc_attend(cache: int, layer: int, q: int, H_q: int, T_new: int, block_table
                max_pages: int, seq_lens: int, scale: float, out: int, stream: int) -> None:
     _check(library().kvc_attend(cache, layer, q, H_q, T_new, block_table or None, max_pages,
                                 seq_lens, scale, out, stream or None), "kvc_attend")
+
+
+def kvc_append_attend(cache: int, layer: int, k_new: int, v_new: int, q: int, H_q: int,
+                      T_new: int, block_table: int, max_pages: int, seq_lens: int, scale: float,
+                      out: int, stream: int) -> None:
+    _check(library().kvc_append_attend(cache, layer, k_new, v_new, q, H_q, T_new,
+                                       block_table or None, max_pages, seq_lens, scale, out,
+                                       stream or None), "kvc_append_attend")
 
 
 def kvc_attend_noalloc(cache: int, layer: int, q: int, H_q: int, T_new: int, block_table: int,
@@ -253,6 +262,25 @@ class KVCache:
         kvc_attend(self.handle, layer, self._dev(q, "q", self.torch_dtype), H_q, T_new, bt, mp,
                    self._dev(seq_lens, "seq_lens", torch.int32), float(scale),
                    self._dev(out, "out", self.torch_dtype), self._stream(stream))
+        return out
+
+    def append_attend(self, layer: int, k_new, v_new, q, seq_lens, block_table=None,
+                      scale: float | None = None, out=None, stream=None):
+        """kvc_append then kvc_attend for the same tokens, fused where possible."""
+        import torch
+        B, H_q, T_new, D = (int(x) for x in q.shape)
+        assert tuple(k_new.shape) == (self.B, self.H_kv, T_new, self.D) == tuple(v_new.shape)
+        if out is None:
+            out = torch.empty_like(q)
+        if scale is None:
+            scale = 1.0 / D ** 0.5
+        bt = 0 if block_table is None else self._dev(block_table, "block_table", torch.int32)
+        mp = 0 if block_table is None else int(block_table.shape[1])
+        kvc_append_attend(self.handle, layer, self._dev(k_new, "k_new", self.torch_dtype),
+                          self._dev(v_new, "v_new", self.torch_dtype),
+                          self._dev(q, "q", self.torch_dtype), H_q, T_new, bt, mp,
+                          self._dev(seq_lens, "seq_lens", torch.int32), float(scale),
+                          self._dev(out, "out", self.torch_dtype), self._stream(stream))
         return out
 
     def reserve(self, H_q: int, T_new: int, max_pages: int = 0) -> None:

@@ -366,6 +366,51 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
       }
     }
 
+    // Fused append: the tile that holds the new positions takes them from
+    // k_new / v_new (its copy from the pool may predate them) and the first row
+    // block writes them into the cache; every other tile is untouched.
+    if (p.k_new != nullptr) {
+      const int ta = cur.k * C::kTile;
+      const int n_lo = max(cur.L, ta), n_hi = min(cur.L + p.T_new, ta + C::kTile);
+      if (n_lo < n_hi) {  // the same decision in every thread of the CTA
+        constexpr int CH = D / 8;  // 16-byte chunks per row
+        unsigned char* dk = sk + st * C::kTileBytes;
+        unsigned char* dv = sv + st * C::kTileBytes;
+        char* kpool = static_cast<char*>(const_cast<void*>(p.k_pool));
+        char* vpool = static_cast<char*>(const_cast<void*>(p.v_pool));
+#pragma unroll 1
+        for (int idx = tid; idx < (n_hi - n_lo) * CH; idx += NTH) {
+          const int rr = idx / CH;
+          const int ch = idx - rr * CH;
+          const int pos = n_lo + rr;
+          const size_t src =
+              ((((size_t)cur.b * p.H_kv + cur.g) * p.T_new + (pos - cur.L)) * D + ch * 8) * 2;
+          const uint4 kv = ld_global_nc_v4(static_cast<const char*>(p.k_new) + src);
+          const uint4 vv = ld_global_nc_v4(static_cast<const char*>(p.v_new) + src);
+          const uint32_t off = swz<D>(pos - ta, ch);
+          st_shared_v4(dk + off, kv);
+          st_shared_v4(dv + off, vv);
+          if (cur.rb == 0) {
+            long long row;
+            if (PAGED) {
+              const int page = p.block_table[(size_t)cur.b * p.max_pages + (pos >> p.page_shift)];
+              if (page < 0 || page >= p.num_pages) {
+                flag_error(p.err, KVC_ERR_BOUNDS);
+                continue;
+              }
+              row = ((long long)page * p.H_kv + cur.g) * (1 << p.page_shift) +
+                    (pos & ((1 << p.page_shift) - 1));
+            } else {
+              row = ((long long)cur.b * p.H_kv + cur.g) * p.max_T + pos;
+            }
+            st_global_v4(kpool + (row * D + ch * 8) * 2, kv);
+            st_global_v4(vpool + (row * D + ch * 8) * 2, vv);
+          }
+        }
+        named_barrier_sync(1, NTH);
+      }
+    }
+
     const uint32_t kb = sk_addr + st * C::kTileBytes;
     const uint32_t vb = sv_addr + st * C::kTileBytes;
     const int t0 = cur.k * C::kTile;

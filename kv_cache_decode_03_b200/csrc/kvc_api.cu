@@ -814,3 +814,68 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
   return c->dtype == KVC_BF16 ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
                               : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
 }
+
+// ---------------------------------------------------------------------------
+// Append and attend in one call.  With the persistent stream-K kernel this is one
+// launch: the tile holding the new positions takes them from k_new / v_new and
+// the kernel writes them into the cache.  Other kernels run the append kernel
+// and then the attend kernel on the same stream.
+extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_new,
+                                        const void* v_new, const void* q, int H_q, int T_new,
+                                        const int32_t* block_table, int max_pages,
+                                        const int32_t* seq_lens, float scale, void* out,
+                                        void* stream) {
+  if (!c || layer < 0 || layer >= c->num_layers || T_new <= 0 || H_q <= 0 ||
+      H_q % c->H_kv != 0)
+    return KVC_ERR_INVALID_ARG;
+  if (!q || !out || !seq_lens || !k_new || !v_new || !aligned16(q) || !aligned16(out) ||
+      !aligned16(k_new) || !aligned16(v_new) || !aligned4(seq_lens))
+    return KVC_ERR_INVALID_ARG;
+  if (c->paged && (!block_table || !aligned4(block_table) || max_pages <= 0))
+    return KVC_ERR_INVALID_ARG;
+  if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
+  if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c, H_q, T_new, max_pages);
+  if (!pl.streamk) {
+    kvc_status st = kvc_append(c, layer, k_new, v_new, T_new, block_table, max_pages,
+                               seq_lens, stream);
+    if (st != KVC_OK) return st;
+    return kvc_attend(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, out,
+                      stream);
+  }
+  kvc_status st = ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
+  if (st != KVC_OK) return st;
+  kvc::AttendParams p{};
+  p.k_pool = kvc_k_pool(c, layer);
+  p.v_pool = kvc_v_pool(c, layer);
+  p.q = q;
+  p.out = out;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.max_pages = max_pages;
+  p.B = c->B;
+  p.H_q = H_q;
+  p.H_kv = c->H_kv;
+  p.T_new = T_new;
+  p.group = H_q / c->H_kv;
+  p.rows = p.group * T_new;
+  p.max_T = c->max_T;
+  p.page_shift = c->page_shift;
+  p.num_pages = c->num_pages;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.split_tokens = pl.split_tokens;
+  p.num_splits = pl.num_splits;
+  p.row_blocks = pl.row_blocks;
+  p.ws_o = c->ws;
+  p.ws_lse = c->ws + pl.slots * pl.R * c->D;
+  p.counters = c->tickets;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.err = c->d_err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return c->dtype == KVC_BF16
+             ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
+                                               c->tmv[layer], s)
+             : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
+                                        c->tmv[layer], s);
+}

@@ -39,6 +39,8 @@ struct AttendParams {
   float* ws_o;        // (B, H_q, T_new, num_splits, D) normalised partial outputs
   float* ws_lse;      // (B, H_q, T_new, num_splits) base-2 log-sum-exp of each slice
   int* counters;      // (B, H_kv, row_blocks) slice tickets, zero between launches
+  const void* k_new;  // fused append (stream-K kernel): (B, H_kv, T_new, D), else null
+  const void* v_new;
   int* err;
 };
 

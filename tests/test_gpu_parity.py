@@ -24,15 +24,22 @@ if not torch.cuda.is_available():  # collected on CPU, skipped there
 
 
 def run_case(case: W.Case, layer: int = 0, requests=None, check_pools: bool = True,
-             nthreads: int = 0, twice: bool = False):
-    """Append + attend on the GPU; compare pools bit-exactly and outputs within tolerance."""
+             nthreads: int = 0, twice: bool = False, fused: bool = False):
+    """Append + attend on the GPU (two calls, or kvc_append_attend when fused); compare
+    pools bit-exactly and outputs within tolerance."""
     g = H.GpuRun(case, layers=layer + 1)
     try:
         kp0, vp0 = case.k_pool(layer), case.v_pool(layer)
         g.load_pools(layer, kp0, vp0)
-        g.append(layer, case.k_new(layer), case.v_new(layer))
         q = case.q(layer)
-        out = g.attend(layer, q)
+        if fused:
+            out = g.cache.append_attend(layer, H.to_device(case.k_new(layer), case.dtype),
+                                        H.to_device(case.v_new(layer), case.dtype),
+                                        H.to_device(q, case.dtype), g.seq_lens, g.block_table,
+                                        scale=case.scale)
+        else:
+            g.append(layer, case.k_new(layer), case.v_new(layer))
+            out = g.attend(layer, q)
         if twice:
             out2 = g.attend(layer, q)
             torch.cuda.synchronize()
@@ -344,3 +351,27 @@ def test_alternating_plans_share_one_cache():
             H.compare(H.out_to_f64(out), ref, f"T_new={T_new}")
     finally:
         g.close()
+
+
+FUSED = {
+    # stream-K (fused in one launch): decode, contiguous and paged with shared prefixes
+    "gqa_contig_decode": lambda: W.contig_case("fz1", 5, 32, 8, 128, "bf16", 1,
+                                               [4095, 64, 127, 0, 3000], seed=41, max_T=4100),
+    "gqa_paged_shared": lambda: W.paged_case("fz2", 8, 32, 8, 128, "bf16", 1, 100, 3000, 16,
+                                             seed=42, pool_seed=43, share_frac=0.25,
+                                             share_tokens=512),
+    # a verify chunk whose new rows straddle a 64-token tile boundary
+    "gqa_verify_straddle": lambda: W.contig_case("fz3", 3, 16, 8, 128, "bf16", 4,
+                                                 [62, 125, 1021], seed=44, max_T=1100),
+    "d64_fp16_paged": lambda: W.paged_case("fz4", 4, 16, 4, 64, "fp16", 2, 0, 900, 16,
+                                           seed=45, pool_seed=46),
+    # other kernels: append then attend, two launches
+    "mha_simt": lambda: W.contig_case("fz5", 2, 8, 8, 64, "fp16", 1, [700, 33], seed=47),
+    "mqa_splitk": lambda: W.paged_case("fz6", 2, 32, 1, 128, "bf16", 4, 100, 2000, 16,
+                                       seed=48, pool_seed=49),
+}
+
+
+@pytest.mark.parametrize("name", list(FUSED))
+def test_append_attend_fused(name):
+    run_case(FUSED[name](), fused=True, twice=False)
