@@ -14,6 +14,7 @@
 #include "attend_decode.cuh"
 #include "attend_mma.cuh"
 #include "attend_streamk.cuh"
+#include "attend_tc.cuh"
 #include "kvc.h"
 
 struct kvc_cache {
@@ -42,6 +43,11 @@ constexpr int kEltBytes = 2;
 // 256-byte K/V row into L2, where the other column's load finds it.
 #ifndef KVC_TMA_L2_PROMOTION
 #define KVC_TMA_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
+// Query rows per KV head from which the tcgen05 kernel (128-row blocks) takes over.
+#ifndef KVC_TC_MIN_ROWS
+#define KVC_TC_MIN_ROWS 64
 #endif
 
 // Split-K sizing: aim for this many waves of resident CTAs, so that the last
@@ -193,6 +199,31 @@ int streamk_occ(int D, int NT, bool paged) {
                           : streamk_occupancy<128, 2, T, false>());
 }
 
+template <int D, typename T, bool PAGED>
+int tc_occupancy() {
+  static int occ = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const size_t smem = kvc::TcCfg<D>::smem_bytes();
+    cudaFuncSetAttribute(kvc::attend_tc_kernel<D, T, PAGED>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kvc::attend_tc_kernel<D, T, PAGED>, kvc::TcCfg<D>::kThreads, smem) !=
+        cudaSuccess)
+      n = 1;
+    // every resident CTA holds TMEM columns: never more than the 512 an SM has
+    occ = std::max(1, std::min(n, 512 / kvc::TcCfg<D>::kTmemCols));
+  });
+  return occ;
+}
+
+template <typename T>
+int tc_occ(int D, bool paged) {
+  if (D == 64) return paged ? tc_occupancy<64, T, true>() : tc_occupancy<64, T, false>();
+  return paged ? tc_occupancy<128, T, true>() : tc_occupancy<128, T, false>();
+}
+
 int mma_scratch_floats(int D, int NT) {
   if (D == 64)
     return NT == 1 ? kvc::MmaCfg<64>::scratch_floats<1>()
@@ -205,7 +236,8 @@ int mma_scratch_floats(int D, int NT) {
 
 // ------------------------------------------------------------ attend plan
 struct Plan {
-  bool mma;          // tensor-core kernel (else the CUDA-core kernel)
+  bool tc;           // tcgen05 kernel, 128 query rows per CTA
+  bool mma;          // mma.sync tensor-core kernel (else the CUDA-core kernel)
   bool streamk;      // mma: persistent stream-K kernel (grid = resident CTAs)
   int grid;          // streamk: persistent CTAs
   size_t slots;      // streamk: partial-result slots (R rows x D each) in the workspace
@@ -270,9 +302,18 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
   const int rows = (H_q / c->H_kv) * T_new;
   // Three or more query rows per K/V row make q.k and p.v a dense contraction
   // worth the tensor cores; one or two rows stay on CUDA cores.
-  pl.mma = c->tma && rows >= 3;
+  // From KVC_TC_MIN_ROWS rows a 128-row block fills the tcgen05 MMA's M.
+  pl.tc = c->tma && rows >= KVC_TC_MIN_ROWS;
+  pl.mma = c->tma && rows >= 3 && !pl.tc;
   int tile, occ, scratch = 1 << 30;
-  if (pl.mma) {
+  if (pl.tc) {
+    pl.NT = 0;
+    pl.R = kvc::TcCfg<64>::kRows;
+    tile = kvc::TcCfg<64>::kTile;
+    occ = c->dtype == KVC_BF16 ? tc_occ<__nv_bfloat16>(c->D, c->paged)
+                               : tc_occ<__half>(c->D, c->paged);
+    scratch = c->D == 64 ? kvc::TcCfg<64>::kScratchFloats : kvc::TcCfg<128>::kScratchFloats;
+  } else if (pl.mma) {
     pl.NT = rows <= 8 ? 1 : (rows <= 16 ? 2 : 4);
     pl.R = pl.NT * 8;
     tile = 64;
@@ -452,6 +493,46 @@ kvc_status dispatch_d(const kvc::AttendParams& p, int D, int R, bool paged, cuda
     case 64: return dispatch_paged<64, T>(p, R, paged, s);
     default: return dispatch_paged<128, T>(p, R, paged, s);
   }
+}
+
+template <int D, typename T, bool PAGED>
+kvc_status launch_attend_tc(const kvc::AttendParams& p, const CUtensorMap& tk,
+                            const CUtensorMap& tv, cudaStream_t stream) {
+  using C = kvc::TcCfg<D>;
+  tc_occupancy<D, T, PAGED>();  // sets the shared-memory attribute once
+  dim3 grid(p.num_splits * p.row_blocks, p.H_kv, p.B);
+  kvc::attend_tc_kernel<D, T, PAGED><<<grid, C::kThreads, C::smem_bytes(), stream>>>(p, tk, tv);
+  return cuda_status(cudaGetLastError());
+}
+
+template <typename T>
+kvc_status dispatch_tc(const kvc::AttendParams& p, int D, bool paged, const CUtensorMap& tk,
+                       const CUtensorMap& tv, cudaStream_t s) {
+  if (D == 64)
+    return paged ? launch_attend_tc<64, T, true>(p, tk, tv, s)
+                 : launch_attend_tc<64, T, false>(p, tk, tv, s);
+  return paged ? launch_attend_tc<128, T, true>(p, tk, tv, s)
+               : launch_attend_tc<128, T, false>(p, tk, tv, s);
+}
+
+// Launch the attend kernel a plan chose for layer `layer`.
+kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::AttendParams& p,
+                    cudaStream_t s) {
+  const bool bf = c->dtype == KVC_BF16;
+  if (pl.tc)
+    return bf ? dispatch_tc<__nv_bfloat16>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s)
+              : dispatch_tc<__half>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s);
+  if (pl.streamk)
+    return bf ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
+                                                c->tmk[layer], c->tmv[layer], s)
+              : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
+                                         c->tmv[layer], s);
+  if (pl.mma)
+    return bf ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
+                                            c->tmv[layer], s)
+              : dispatch_mma<__half>(p, c->D, pl.NT, c->paged, c->tmk[layer], c->tmv[layer], s);
+  return bf ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
+            : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
 }
 
 }  // namespace
@@ -675,19 +756,7 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   p.counters = c->tickets;
   p.err = c->d_err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (pl.streamk)
-    return c->dtype == KVC_BF16
-               ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
-                                                 c->tmk[layer], c->tmv[layer], s)
-               : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
-                                          c->tmv[layer], s);
-  if (pl.mma)
-    return c->dtype == KVC_BF16
-               ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
-                                             c->tmv[layer], s)
-               : dispatch_mma<__half>(p, c->D, pl.NT, c->paged, c->tmk[layer], c->tmv[layer], s);
-  return c->dtype == KVC_BF16 ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
-                              : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
+  return run_plan(c, layer, pl, p, s);
 }
 
 kvc_status kvc_get_error(kvc_cache* c) {
@@ -800,19 +869,7 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
                         : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
   p.counters = static_cast<int*>(base);
   p.err = c->d_err;
-  if (pl.streamk)
-    return c->dtype == KVC_BF16
-               ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
-                                                 c->tmk[layer], c->tmv[layer], s)
-               : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
-                                          c->tmv[layer], s);
-  if (pl.mma)
-    return c->dtype == KVC_BF16
-               ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
-                                             c->tmv[layer], s)
-               : dispatch_mma<__half>(p, c->D, pl.NT, c->paged, c->tmk[layer], c->tmv[layer], s);
-  return c->dtype == KVC_BF16 ? dispatch_d<__nv_bfloat16>(p, c->D, pl.R, c->paged, s)
-                              : dispatch_d<__half>(p, c->D, pl.R, c->paged, s);
+  return run_plan(c, layer, pl, p, s);
 }
 
 // ---------------------------------------------------------------------------

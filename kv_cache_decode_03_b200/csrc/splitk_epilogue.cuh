@@ -27,10 +27,11 @@ __device__ __forceinline__ void store_elt(T* ptr, float v) {
   else *ptr = __float2half_rn(v);
 }
 
-// red_acc: [W][R][D] fp32, red_m / red_l: [W][R].  scratch: >= R * num_splits floats
-// of shared memory that nothing else uses.  flags: one shared int.  All NT
-// threads of the CTA call this together after red_* are written and synced.
-template <typename T, int D, int R, int W, int NT>
+// red_acc: [W][R] rows of D fp32, LD floats apart; red_m / red_l: [W][R].
+// scratch: >= R * num_splits floats of shared memory that nothing else uses.
+// flags: one shared int.  All NT threads of the CTA call this together after
+// red_* are written and synced.
+template <typename T, int D, int R, int W, int NT, int LD = D>
 __device__ __forceinline__ void finish_slice(const AttendParams& p, const float* red_acc,
                                              const float* red_m, const float* red_l,
                                              float* scratch, int* flag, int b, int g, int rb,
@@ -52,7 +53,7 @@ __device__ __forceinline__ void finish_slice(const AttendParams& p, const float*
     for (int w = 0; w < W; ++w) {
       const float f = exp2f(red_m[w * R + rr] - M);
       lsum = fmaf(red_l[w * R + rr], f, lsum);
-      o = fmaf(red_acc[(w * R + rr) * D + d], f, o);
+      o = fmaf(red_acc[(w * R + rr) * LD + d], f, o);
     }
     const int i = (r0 + rr) % p.T_new;
     const size_t orow = row_base + rr;

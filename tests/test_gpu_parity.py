@@ -90,6 +90,54 @@ def test_page_sizes(P):
 
 
 # ---------------------------------------------------------------------------
+# 64 or more query rows per KV head (the 128-row tcgen05 blocks): MQA decode,
+# verify chunks, prefill chunks; row counts that leave a ragged last block and
+# blocks that cut one head's chunk in two
+# ---------------------------------------------------------------------------
+
+TC_HEADS = [(64, 1, 1), (16, 2, 8), (8, 1, 25), (32, 1, 9), (12, 12, 128)]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("heads", TC_HEADS, ids=lambda h: f"hq{h[0]}_hkv{h[1]}_t{h[2]}")
+def test_many_rows_grid(D, dtype, paged, heads):
+    H_q, H_kv, T_new = heads
+    seed = 3000 + D + 7 * H_q + 13 * T_new + (1 if dtype == "bf16" else 0)
+    if paged:
+        case = W.paged_case("rows", 3, H_q, H_kv, D, dtype, T_new, 0, 700, 16, seed=seed,
+                            pool_seed=seed + 1)
+    else:
+        L = W.rng(seed, "L").integers(0, 700, size=3, endpoint=True)
+        L[0] = 0
+        case = W.contig_case("rows", 3, H_q, H_kv, D, dtype, T_new, L, seed=seed,
+                             max_T=int(L.max()) + T_new + 5)
+    run_case(case)
+
+
+@pytest.mark.parametrize("P", [8, 64, 256])
+def test_many_rows_page_sizes(P):
+    case = W.paged_case(f"rows_pages{P}", 3, 32, 1, 128, "bf16", 4, 0, 900, P, seed=70 + P,
+                        pool_seed=80 + P, share_frac=0.5, share_tokens=4 * P)
+    run_case(case)
+
+
+def test_many_rows_long_context_split_cap():
+    """One request, one KV head, 30K positions: the split count hits the merge's
+    shared-memory cap."""
+    case = W.contig_case("rows_long", 1, 64, 1, 128, "bf16", 2, [30000], seed=90,
+                         max_T=30002)
+    run_case(case)
+
+
+def test_many_rows_deterministic():
+    case = W.paged_case("rows_det", 2, 32, 1, 128, "bf16", 8, 500, 5000, 16, seed=91,
+                        pool_seed=92)
+    run_case(case, twice=True)
+
+
+# ---------------------------------------------------------------------------
 # edge cases
 # ---------------------------------------------------------------------------
 
