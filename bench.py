@@ -41,10 +41,19 @@ import workloads as W  # noqa: E402
 METRIC = ("decode-attention KV HBM GB/s (% of B200 peak) and tokens/s per layer-step")
 
 
-def kernel_source_sha256() -> str:
+# The sources each profiled kernel is compiled from: a committed ncu summary stays
+# valid while these files are unchanged.
+KERNEL_SOURCES = {
+    "attend_streamk_kernel": ("attend_streamk.cuh", "splitk_epilogue.cuh", "device_common.cuh",
+                              "params.cuh"),
+}
+
+
+def kernel_source_sha256(kernel: str = "attend_streamk_kernel") -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in sorted((ROOT / "kv_cache_decode_03_b200" / "csrc").glob("*")):
+    for name in KERNEL_SOURCES[kernel]:
+        f = ROOT / "kv_cache_decode_03_b200" / "csrc" / name
         h.update(f.name.encode())
         h.update(f.read_bytes())
     return h.hexdigest()
@@ -52,7 +61,7 @@ def kernel_source_sha256() -> str:
 
 def profiled_traffic(kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if its sources still match."""
-    sha = kernel_source_sha256()
+    sha = kernel_source_sha256(kernel.split("<")[0])
     for f in sorted((ROOT / "profiles").glob("*.md")):
         kv = {}
         for line in f.read_text().splitlines():

@@ -8,10 +8,18 @@
 // block of 128 query rows as the MMA M dimension:
 //     S[128 x 64]  = Q[128 x D] . K_tile^T        tcgen05.mma, fp32 in TMEM
 //     O[128 x D]  += P[128 x 64] . V_tile          tcgen05.mma, fp32 in TMEM
-// Thread 0 issues the TMA loads and the MMAs; thread t owns TMEM lane t, i.e.
-// query row t, for the softmax: it reads its 64 scores with tcgen05.ld, keeps
-// the running max and sum in registers and writes its row of P back over the
-// scores in TMEM, where the second MMA takes it as its A operand.
+// Roles (warp-specialised, 224 threads):
+//   warps 5, 6  TMA producers of K and of V tiles (64 tokens) into two rings;
+//            a K stage is free again as soon as its S MMA is done, so K runs
+//            several tiles ahead of V; the page lookups of a tile are spread
+//            over the warp's lanes;
+//   warp 4   MMA issuer (one lane): S(j+1) = Q.K(j+1)^T is issued while the
+//            softmax of tile j runs (S double-buffered in TMEM), then
+//            O += P(j).V(j) once P(j) is written;
+//   warps 0-3 softmax: thread t owns TMEM lane t, i.e. query row t: it reads
+//            its 64 scores with tcgen05.ld, keeps the running max and sum in
+//            registers and writes its row of P back over the scores in TMEM,
+//            where the P.V MMA takes it as its A operand.
 //
 // Precision of P: a bf16 P (8-bit significand) moves short-context outputs by
 // up to ~2^-9 max|v|, several times the 2e-3 bound on the output.  For bf16
@@ -27,12 +35,14 @@
 // Shared-memory operands use the canonical 128-byte-swizzled layouts the TMA
 // tiles already have: Q and K are K-major (8-row groups of 1024 bytes,
 // 16-element k-steps of 32 bytes inside a row), V is MN-major (64-element boxes
-// along D, 8-token groups of 1024 bytes).  TMEM: S in columns [0, 64), then P
-// over it (two 16-bit values per column: P_hi in [0, 32), P_lo in [32, 64)),
-// O in [64, 64 + D).
+// along D, 8-token groups of 1024 bytes).  TMEM: two S buffers in columns
+// [0, 64) and [64, 128), each overwritten by its P (two 16-bit values per
+// column: P_hi in the first 32 columns, P_lo in the next 32), O in
+// [128, 128 + D).
 //
-// Every wait is bounded; a timeout raises KVC_ERR_TIMEOUT, all threads leave
-// the loop together (barrier with a vote), thread 0 waits (bounded) for its
+// Every wait is bounded; a timeout raises KVC_ERR_TIMEOUT and sets the CTA's
+// abort word, which ends every role's loop; the CTA then agrees on the abort
+// with a barrier vote, the producer and the MMA lane wait (bounded) for their
 // copies and MMAs in flight, and the TMEM is released before the CTA exits.
 #pragma once
 
@@ -43,37 +53,43 @@
 #include "params.cuh"
 #include "splitk_epilogue.cuh"
 
-#ifndef KVC_TC_STAGES
-#define KVC_TC_STAGES 2
-#endif
 
 namespace kvc {
 
 template <int D>
 struct TcCfg {
   static_assert(D == 64 || D == 128, "tcgen05 attend: D must be 64 or 128");
-  static constexpr int kThreads = 128;           // one thread per query row (TMEM lane)
+  static constexpr int kSoftmaxThreads = 128;    // one thread per query row (TMEM lane)
+  static constexpr int kMmaWarp = 4;
+  static constexpr int kKWarp = 5;               // K producer
+  static constexpr int kVWarp = 6;               // V producer
+  static constexpr int kThreads = 224;
   static constexpr int kRows = 128;              // MMA M
   static constexpr int kTile = 64;               // tokens per K/V tile (MMA N of S)
   static constexpr int kHalves = D / 64;         // 64-element boxes across a row
   static constexpr int kBoxBytes = kTile * 128;  // one box of a K/V tile
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStages = KVC_TC_STAGES;
-  static constexpr int kRing = 2 * kStages * kTileBytes;  // K stages, then V stages
-  static constexpr int kQBox = kRows * 128;               // one 64-element box of Q
+  // stages sized so that two CTAs share an SM (<= 113 KB of shared memory each)
+  static constexpr int kKStages = D == 128 ? 3 : 4;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
+  static constexpr int kKRing = kKStages * kTileBytes;
+  static constexpr int kVRing = kVStages * kTileBytes;
+  static constexpr int kQBox = kRows * 128;      // one 64-element box of Q
   static constexpr int kQBytes = kRows * D * 2;
-  static constexpr int kTmemCols = D == 64 ? 128 : 256;   // S/P + O, a power of two
-  static constexpr int kData = kRing + kQBytes;           // 1024-aligned operand area
+  static constexpr int kTmemCols = 256;          // S/P x 2, O
+  static constexpr int kOCol = 128;
+  static constexpr int kData = kKRing + kVRing + kQBytes;  // 1024-aligned operand area
   // after the loop the operand area holds the per-row results:
   static constexpr int kAccLd = D + 4;  // padded rows: conflict-free float4 stores
   static constexpr int kAccBytes = kRows * kAccLd * 4;
   static constexpr int kScratchOff = kAccBytes + 2 * kRows * 4;
   static constexpr int kScratchFloats = (kData - kScratchOff) / 4;
   static_assert(kScratchOff + kRows * 4 <= kData, "result area too small");
+  // K full/empty, V full/empty, s_full x2, p_full x2, o_done, drain
+  static constexpr int kBarriers = 2 * kKStages + 2 * kVStages + 6;
 
-  static constexpr size_t smem_bytes() {
-    return 1024 /* alignment slack */ + kData + (kStages + 3) * sizeof(uint64_t) + 16;
-  }
+  // The dynamic shared memory starts 1024-byte aligned (checked at run time).
+  static constexpr size_t smem_bytes() { return kData + kBarriers * sizeof(uint64_t) + 16; }
 };
 
 // UMMA shared-memory descriptor for a 128-byte-swizzled operand whose atoms
@@ -171,6 +187,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {  // MUFU 2^x; 2^-inf = 0
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -179,24 +201,28 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 template <int D, typename T, bool PAGED>
-__global__ void __launch_bounds__(TcCfg<D>::kThreads)
+__global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     attend_tc_kernel(const AttendParams p, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv) {
   using C = TcCfg<D>;
   constexpr int R = C::kRows;
-  constexpr int NTH = C::kThreads;
-  constexpr int S = C::kStages;
+  constexpr int NSM = C::kSoftmaxThreads;
+  constexpr int SK = C::kKStages;
+  constexpr int SV = C::kVStages;
   constexpr bool kSplitP = Elt<T>::kCode == KVC_BF16;
-  extern __shared__ __align__(1024) unsigned char tc_smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sk = smem;                      // K stages
-  unsigned char* sv = smem + S * C::kTileBytes;  // V stages
-  unsigned char* sq = smem + C::kRing;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kData);
-  uint64_t* sbar = full + S;  // S = Q.K^T done
-  uint64_t* obar = sbar + 1;  // O += P.V done
-  uint64_t* dbar = obar + 1;  // drain after an abort
+  extern __shared__ __align__(1024) unsigned char tc_smem[];
+  unsigned char* const smem = tc_smem;
+  unsigned char* sk = smem;                // K stages
+  unsigned char* sv = smem + C::kKRing;    // V stages
+  unsigned char* sq = sv + C::kVRing;      // Q
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(smem + C::kData);
+  uint64_t* k_empty = k_full + SK;   // K stage consumed by its S MMA
+  uint64_t* v_full = k_empty + SK;
+  uint64_t* v_empty = v_full + SV;   // V stage consumed by its P.V MMA
+  uint64_t* s_full = v_empty + SV;   // [2] S buffer holds Q.K^T
+  uint64_t* p_full = s_full + 2;     // [2] S buffer holds P (128 arrivals)
+  uint64_t* o_done = p_full + 2;     // O += P.V of the last issued tile done
+  uint64_t* dbar = o_done + 1;       // drain after an abort
   uint32_t* tslot = reinterpret_cast<uint32_t*>(dbar + 1);
   int* flags = reinterpret_cast<int*>(tslot + 1);  // [0] abort [1] last
   float* red_acc = reinterpret_cast<float*>(smem);  // operand area, after the loop
@@ -206,6 +232,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane_id = tid & 31;
   const int s = blockIdx.x / p.row_blocks;  // row blocks vary fastest (shared K/V in L2)
   const int rb = blockIdx.x - s * p.row_blocks;
   const int g = blockIdx.y;
@@ -223,6 +250,10 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
   const int n_blk = L + i_max + 1;
   const int t_begin = s * p.split_tokens;
   if (t_begin >= n_blk) return;
+  if (smem_addr(smem) & 1023u) {  // swizzle atoms need 1024-byte alignment
+    if (tid == 0) flag_error(p.err, KVC_ERR_UNSUPPORTED);
+    return;
+  }
   if (L < 0 || L + p.T_new > p.max_T ||
       (PAGED && ((L + p.T_new - 1) >> p.page_shift) >= p.max_pages)) {
     if (tid == 0) flag_error(p.err, KVC_ERR_BOUNDS);
@@ -241,16 +272,25 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-#pragma unroll
-    for (int st = 0; st < S; ++st) mbar_init(&full[st], 1);
-    mbar_init(sbar, 1);
-    mbar_init(obar, 1);
+    for (int st = 0; st < SK; ++st) {
+      mbar_init(&k_full[st], 1);
+      mbar_init(&k_empty[st], 1);
+    }
+    for (int st = 0; st < SV; ++st) {
+      mbar_init(&v_full[st], 1);
+      mbar_init(&v_empty[st], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&s_full[k], 1);
+      mbar_init(&p_full[k], NSM);
+    }
+    mbar_init(o_done, 1);
     mbar_init(dbar, 1);
     flags[0] = 0;
     flags[1] = 0;
     fence_barrier_init();
   }
-  {
+  if (tid < NSM) {
     const char* qrow =
         static_cast<const char*>(p.q) +
         ((((size_t)b * p.H_q + (size_t)g * p.group) * p.T_new) + r0 + tid) * D * 2;
@@ -259,15 +299,13 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
       const uint4 v = tid < nr ? ld_global_nc_v4(qrow + ch * 16) : make_uint4(0, 0, 0, 0);
       st_shared_v4(sq + (ch >> 3) * C::kQBox + tid * 128 + (((ch & 7) ^ (tid & 7)) << 4), v);
     }
+    fence_async_smem();
   }
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tS = tmem;                           // columns [0, 64)
-  const uint32_t tO = tmem + 64;                      // columns [64, 64 + D)
-  const uint32_t lane = (uint32_t)(warp * 32) << 16;  // this warp's 32 TMEM lanes
+  const uint32_t tO = tmem + C::kOCol;
 
   volatile int* abort_word = flags;
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -288,69 +326,75 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
     }
   };
 
-  // ---- producer (thread 0): K and V tiles of 64 tokens by TMA, no multicast
-  const uint64_t pol = p.row_blocks > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
-  int issued = 0, consumed = 0;
-  bool mma_issued = false;
-  auto issue = [&](int j) {
-    const int st = j % S;
-    const int t0 = t_begin + j * C::kTile;
-    unsigned char* dk = sk + st * C::kTileBytes;
-    unsigned char* dv = sv + st * C::kTileBytes;
-    mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes);  // every box is full (zero fill)
-    if (!PAGED) {
-      const int y = (b * p.H_kv + g) * p.max_T + t0;
-#pragma unroll
-      for (int h = 0; h < C::kHalves; ++h) {
-        tma_load_2d(dk + h * C::kBoxBytes, &tmk, h * 64, y, &full[st], pol);
-        tma_load_2d(dv + h * C::kBoxBytes, &tmv, h * 64, y, &full[st], pol);
-      }
-    } else {
-      const int Pg = 1 << p.page_shift;
-      const int box_rows = Pg < C::kTile ? Pg : C::kTile;
-      const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
-      const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
+  bool ok = true;
+  int issued = 0;            // producer: tiles whose loads were issued
+  bool mma_issued = false;   // MMA lane
+  float m_ref = -INFINITY;   // softmax: the row's reference max (base 2) and
+  float l = 0.f;             // sum of 2^(s - m_ref)
+
+  if (warp == C::kKWarp || warp == C::kVWarp) {
+    // ---- TMA producers (no multicast): warp 5 loads K, warp 6 loads V; lane k
+    // loads box k of a paged tile
+    const bool is_k = warp == C::kKWarp;
+    const int NS = is_k ? SK : SV;
+    unsigned char* ring = is_k ? sk : sv;
+    uint64_t* full = is_k ? k_full : v_full;
+    uint64_t* empty = is_k ? k_empty : v_empty;
+    const CUtensorMap* tm = is_k ? &tmk : &tmv;
+    const uint64_t pol = p.row_blocks > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
+    if (lane_id == 0) prefetch_tmap(tm);
 #pragma unroll 1
-      for (int t = t0; t < t0 + C::kTile; t += box_rows) {
-        int y = beyond;
-        if (t < t_stop) {
-          const int page = bt[t >> p.page_shift];
-          if (page >= 0 && page < p.num_pages)
-            y = (page * p.H_kv + g) * Pg + (t & (Pg - 1));
-          else
-            flag_error(p.err, KVC_ERR_BOUNDS);
-        }
-        const int off = (t - t0) * 128;
-#pragma unroll
-        for (int h = 0; h < C::kHalves; ++h) {
-          tma_load_2d(dk + h * C::kBoxBytes + off, &tmk, h * 64, y, &full[st], pol);
-          tma_load_2d(dv + h * C::kBoxBytes + off, &tmv, h * 64, y, &full[st], pol);
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % NS;
+      if (j >= NS) {
+        bool w = true;
+        if (lane_id == 0) w = wait(&empty[st], ((j / NS) - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
         }
       }
+      const int t0 = t_begin + j * C::kTile;
+      unsigned char* dst = ring + st * C::kTileBytes;
+      if (lane_id == 0) mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+      __syncwarp();
+      if (!PAGED) {
+        if (lane_id < C::kHalves)
+          tma_load_2d(dst + lane_id * C::kBoxBytes, tm, lane_id * 64,
+                      (b * p.H_kv + g) * p.max_T + t0, &full[st], pol);
+      } else {
+        const int Pg = 1 << p.page_shift;
+        const int box_rows = Pg < C::kTile ? Pg : C::kTile;
+        const int nbox = C::kTile / box_rows;  // <= 8 (pages of 8 or more tokens)
+        if (lane_id < nbox) {
+          const int t = t0 + lane_id * box_rows;
+          int y = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
+          if (t < t_stop) {
+            const int page = p.block_table[(size_t)b * p.max_pages + (t >> p.page_shift)];
+            if (page >= 0 && page < p.num_pages)
+              y = (page * p.H_kv + g) * Pg + (t & (Pg - 1));
+            else
+              flag_error(p.err, KVC_ERR_BOUNDS);
+          }
+          const int off = lane_id * box_rows * 128;
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h)
+            tma_load_2d(dst + h * C::kBoxBytes + off, tm, h * 64, y, &full[st], pol);
+        }
+      }
+      ++issued;
     }
-    ++issued;
-  };
-  if (tid == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-    for (int j = 0; j < min(S, ntiles); ++j) issue(j);
-  }
-
-  const uint32_t idesc_s = umma_idesc<T>(R, C::kTile, false);
-  const uint32_t idesc_o = umma_idesc<T>(R, D, true);
-  const uint32_t sq_a = smem_addr(sq), sk_a = smem_addr(sk), sv_a = smem_addr(sv);
-
-  // this thread's query row sees positions [0, vis)
-  const int vis = tid < nr ? L + (r0 + tid) % p.T_new + 1 : 0;
-  float m_ref = -INFINITY, l = 0.f;
-
-#pragma unroll 1
-  for (int j = 0; j < ntiles; ++j) {
-    const int st = j % S;
-    if (tid == 0 && !*abort_word) {
-      if (wait(&full[st], (j / S) & 1)) {
-        ++consumed;
+  } else if (warp == C::kMmaWarp) {
+    // ---- MMA issuer: S(j+1) ahead of P(j).V(j); S buffer j&1 holds S(j), then P(j)
+    if (lane_id == 0) {
+      const uint32_t idesc_s = umma_idesc<T>(R, C::kTile, false);
+      const uint32_t idesc_o = umma_idesc<T>(R, D, true);
+      const uint32_t sq_a = smem_addr(sq), sk_a = smem_addr(sk), sv_a = smem_addr(sv);
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % SK;
+        if (!wait(&k_full[st], (j / SK) & 1)) return false;
         tc_fence_after();
+        const uint32_t tS = tmem + (j & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qoff = (kk >> 2) * C::kQBox + (kk & 3) * 32;
@@ -358,31 +402,83 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
           umma_f16(tS, umma_desc_sw128(sq_a + qoff, 16, 1024),
                    umma_desc_sw128(sk_a + koff, 16, 1024), idesc_s, kk > 0);
         }
-        umma_commit(sbar);
+        umma_commit(&s_full[j & 1]);
+        umma_commit(&k_empty[st]);
         mma_issued = true;
+        return true;
+      };
+      ok = issue_s(0);
+#pragma unroll 1
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles) {
+          // buffer (j+1)&1 still holds P(j-1) until its P.V MMA is done
+          if (j >= 1 && !wait(o_done, (j - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          if (!issue_s(j + 1)) {
+            ok = false;
+            break;
+          }
+        }
+        const int st = j % SV;
+        if (!wait(&p_full[j & 1], (j >> 1) & 1) || !wait(&v_full[st], (j / SV) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tP = tmem + (j & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < C::kTile / 16; ++kk) {
+          const uint64_t bv =
+              umma_desc_sw128(sv_a + st * C::kTileBytes + kk * 2048, C::kBoxBytes, 1024);
+          umma_f16_tmem_a(tO, tP + kk * 8, bv, idesc_o, j > 0 || kk > 0);
+          if constexpr (kSplitP) umma_f16_tmem_a(tO, tP + 32 + kk * 8, bv, idesc_o, true);
+        }
+        umma_commit(&v_empty[st]);
+        umma_commit(o_done);
       }
     }
-    // tcgen05.ld / st below are warp-collective: a warp goes on only as a whole
-    const bool ok = __all_sync(0xffffffffu, wait(sbar, j & 1));
-    if (ok) {
+    __syncwarp();
+  } else {
+    // ---- softmax: thread tid owns query row tid (TMEM lane tid)
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;  // this warp's 32 TMEM lanes
+    const int vis = tid < nr ? L + (r0 + tid) % p.T_new + 1 : 0;  // positions [0, vis)
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+#pragma unroll 1
+    for (int j = 0; j < ntiles; ++j) {
+      const int buf = j & 1;
+      const uint32_t tS = tmem + buf * 64 + lane;
+      // tcgen05.ld / st are warp-collective: a warp goes on only as a whole
+      ok = __all_sync(0xffffffffu, wait(&s_full[buf], (j >> 1) & 1));
+      if (!ok) break;
       tc_fence_after();
-      // ---- softmax of this thread's row over the tile's 64 tokens
-      float sc[64];
+      float2 sc[32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld16(tS + lane + c4 * 16, sc + c4 * 16);
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld16(tS + c4 * 16, reinterpret_cast<float*>(sc) + c4 * 16);
       tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) sc[c] = __fmul2_rn(sc[c], sc2);
       const int t0 = t_begin + j * C::kTile;
+      if (__any_sync(0xffffffffu, t0 + C::kTile > vis)) {  // tile reaches past some row's end
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (t0 + 2 * c >= vis) sc[c].x = -INFINITY;
+          if (t0 + 2 * c + 1 >= vis) sc[c].y = -INFINITY;
+        }
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        sc[c] = (t0 + c < vis) ? sc[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sc[c]);
-      }
+      for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(sc[c].x, sc[c].y));
       // Move the reference max when the tile's max passes it by 2^8 and rescale
       // this row of O (before any visible token the row is all zero: alpha 1).
       const bool move = mx > m_ref + 8.f;
-      const float alpha = (move && m_ref != -INFINITY) ? exp2f(m_ref - mx) : 1.f;
+      const float alpha = (move && m_ref != -INFINITY) ? ex2_approx(m_ref - mx) : 1.f;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {  // the warp's 32 rows together
+        // O must hold P(j-1).V(j-1) first
+        ok = __all_sync(0xffffffffu, wait(o_done, (j - 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int c16 = 0; c16 < D / 16; ++c16) {
           float ov[16];
@@ -399,58 +495,48 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
         m_ref = mx;
       }
       const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const float2 mu2 = make_float2(-mu, -mu);
       uint32_t ph[32];
-      float lsum = 0.f;
+      float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = exp2f(sc[2 * c] - mu);
-        const float p1 = exp2f(sc[2 * c + 1] - mu);
-        lsum += p0 + p1;
-        ph[c] = Elt<T>::pack2(p0, p1);
-        if constexpr (kSplitP) {  // keep the rounding remainder in sc[] for P_lo
-          sc[2 * c] = p0 - __uint_as_float(ph[c] << 16);
-          sc[2 * c + 1] = p1 - __uint_as_float(ph[c] & 0xFFFF0000u);
-        }
+        const float2 e = __fadd2_rn(sc[c], mu2);
+        const float2 pp = make_float2(ex2_approx(e.x), ex2_approx(e.y));
+        lsum = __fadd2_rn(lsum, pp);
+        ph[c] = Elt<T>::pack2(pp.x, pp.y);
+        if constexpr (kSplitP)  // keep the rounding remainder in sc[] for P_lo
+          sc[c] = __fadd2_rn(pp, make_float2(-__uint_as_float(ph[c] << 16),
+                                             -__uint_as_float(ph[c] & 0xFFFF0000u)));
       }
-      l += lsum;
+      l += lsum.x + lsum.y;
       // P over this row's scores: 64 tokens in 32 columns (even token low half)
-      tmem_st16(tS + lane, ph);
-      tmem_st16(tS + lane + 16, ph + 16);
+      tmem_st16(tS, ph);
+      tmem_st16(tS + 16, ph + 16);
       if constexpr (kSplitP) {
         uint32_t pl[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pl[c] = Elt<T>::pack2(sc[2 * c], sc[2 * c + 1]);
-        tmem_st16(tS + lane + 32, pl);
-        tmem_st16(tS + lane + 48, pl + 16);
+        for (int c = 0; c < 32; ++c) pl[c] = Elt<T>::pack2(sc[c].x, sc[c].y);
+        tmem_st16(tS + 32, pl);
+        tmem_st16(tS + 48, pl + 16);
       }
       tmem_wait_st();
       tc_fence_before();
+      mbar_arrive(&p_full[buf]);
     }
-    if (__syncthreads_or(!ok)) break;  // everyone leaves together
-
-    if (tid == 0) {  // O += P . V, then refill the stage once it is free
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < C::kTile / 16; ++kk) {
-        const uint64_t bv =
-            umma_desc_sw128(sv_a + st * C::kTileBytes + kk * 2048, C::kBoxBytes, 1024);
-        umma_f16_tmem_a(tO, tS + kk * 8, bv, idesc_o, j > 0 || kk > 0);
-        if constexpr (kSplitP) umma_f16_tmem_a(tO, tS + 32 + kk * 8, bv, idesc_o, true);
-      }
-      umma_commit(obar);
-      if (wait(obar, j & 1) && j + S < ntiles) issue(j + S);
-    }
+    if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, wait(o_done, (ntiles - 1) & 1));
   }
 
   const bool bad = __syncthreads_or(*abort_word != 0);
   if (bad) {
-    if (tid == 0) {  // nothing may still write this CTA's shared memory or TMEM
-      if (mma_issued) {
-        umma_commit(dbar);
-        mbar_wait(dbar, 0, p.err);
-      }
-      for (int j = consumed; j < issued; ++j)
-        if (!mbar_wait(&full[j % S], (j / S) & 1, p.err)) break;
+    if ((warp == C::kKWarp || warp == C::kVWarp) && lane_id == 0) {  // loads in flight
+      const int NS = warp == C::kKWarp ? SK : SV;
+      uint64_t* full = warp == C::kKWarp ? k_full : v_full;
+      for (int j = max(0, issued - NS); j < issued; ++j)
+        if (!mbar_wait(&full[j % NS], (j / NS) & 1, p.err)) break;
+    }
+    if (warp == C::kMmaWarp && lane_id == 0 && mma_issued) {  // MMAs still in flight
+      umma_commit(dbar);
+      mbar_wait(dbar, 0, p.err);
     }
     tc_fence_before();
     __syncthreads();
@@ -460,29 +546,34 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads)
                    : "memory");
     return;
   }
+  if (warp >= C::kMmaWarp) return;  // producers and MMA issuer are done
 
-  // ---- this row's unnormalised O, reference max and sum to shared memory
+  // ---- this row's unnormalised O, reference max and sum to shared memory (every
+  // MMA and load has completed: the ring and Q are idle)
   tc_fence_after();
-#pragma unroll 1
-  for (int c16 = 0; c16 < D / 16; ++c16) {
-    float ov[16];
-    tmem_ld16(tO + lane + c16 * 16, ov);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 16; i += 4)
-      *reinterpret_cast<float4*>(red_acc + tid * C::kAccLd + c16 * 16 + i) =
-          make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
-  }
   red_m[tid] = m_ref;
   red_l[tid] = l;
+  {
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+#pragma unroll 1
+    for (int c16 = 0; c16 < D / 16; ++c16) {
+      float ov[16];
+      tmem_ld16(tO + lane + c16 * 16, ov);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<float4*>(red_acc + tid * C::kAccLd + c16 * 16 + i) =
+            make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  named_barrier_sync(1, NSM);
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(C::kTmemCols)
                  : "memory");
-  finish_slice<T, D, R, 1, NTH, C::kAccLd>(p, red_acc, red_m, red_l, scratch, &flags[1], b, g, rb,
-                                           s, r0, nr, L, ns_blk);
+  finish_slice<T, D, R, 1, NSM, C::kAccLd>(p, red_acc, red_m, red_l, scratch, &flags[1], b, g,
+                                           rb, s, r0, nr, L, ns_blk);
 }
 
 }  // namespace kvc
