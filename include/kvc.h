@@ -28,9 +28,10 @@
  *     16-byte aligned.  `stream` is a cudaStream_t (NULL = legacy default stream);
  *     every call is asynchronous on it.
  *   - seq_lens: device int32[B]; seq_lens[b] is the committed length L_b of request
- *     b BEFORE the new tokens.  The library never modifies it: committing T_new
- *     tokens (append/commit) means the caller adds T_new to seq_lens after the step;
- *     rolling back after a rejected speculative draft means lowering it.
+ *     b BEFORE the new tokens.  Append and attend never modify it: committing tokens
+ *     (append/commit) means raising it after the step, rolling back after a rejected
+ *     speculative draft means lowering it -- by the caller, or on the device with
+ *     kvc_commit / kvc_rollback.
  *   - GQA: query head h reads KV head h / (H_q / H_kv).  MHA: H_q == H_kv.  MQA: H_kv == 1.
  *   - Causality: new row i (0 <= i < T_new) of request b sees positions 0 .. L_b + i.
  *   - Paged cache: pool[page][H_kv][page_size][D] for K and for V of each layer;
@@ -188,6 +189,48 @@ void* kvc_v_pool(kvc_cache* cache, int layer);
 
 /* kvc_layer_pool_bytes -- bytes of one layer's K (equally V) pool. */
 size_t kvc_layer_pool_bytes(const kvc_cache* cache);
+
+/*
+ * kvc_commit -- advance every request's committed length by its accepted count
+ * ("llm-perf-lab" README: the preallocated cache commits in two phases, append then
+ * commit, and speculative decoding keeps only the accepted prefix of the gamma verified
+ * tokens).  After an append of T_new tokens at positions L_b .. L_b+T_new-1, the
+ * caller accepts accepted[b] of them and this call sets seq_lens[b] = L_b + accepted[b],
+ * on the device and in stream order (accepted[] is typically written by the verify
+ * step's own kernels, so the host never waits).  Positions past the new length keep the
+ * rejected K/V until the next append overwrites them; no attend reads them.
+ *   seq_lens   device int32[B], updated in place.
+ *   accepted   device int32[B].
+ *   T_new      the number of appended tokens the counts refer to.
+ * A count outside [0, T_new] or a new length above max_T leaves that request unchanged
+ * and sets KVC_ERR_BOUNDS in the sticky error word.
+ */
+kvc_status kvc_commit(kvc_cache* cache, int32_t* seq_lens, const int32_t* accepted, int T_new,
+                      void* stream);
+
+/*
+ * kvc_rollback -- lower every request's committed length: seq_lens[b] -= drop[b]
+ * ("llm-perf-lab" README: rolling the cache back).  The dropped positions' K/V stay in
+ * the pools until an append overwrites them.  A drop outside [0, seq_lens[b]] leaves
+ * that request unchanged and sets KVC_ERR_BOUNDS.  seq_lens, drop: device int32[B].
+ */
+kvc_status kvc_rollback(kvc_cache* cache, int32_t* seq_lens, const int32_t* drop, void* stream);
+
+/*
+ * kvc_copy_pages -- make page dst[i] a bit-exact copy of page src[i] (i < n) in every
+ * layer, K and V, of a paged cache ("9. 推理" 9.6: a cache managed in fixed-size pages).
+ * This is the copy of copy-on-write: before an append would land in a page that other
+ * requests also list (a shared prefix whose last page is partly filled), the caller,
+ * which owns page reference counts and block tables, takes a free page, copies the
+ * shared page into it with this call and points the request's block-table entry at the
+ * copy, then appends.
+ *   src, dst   device int32[n] page ids in [0, num_pages).  The dst pages must be
+ *              distinct and none may also be a src page of the same call.
+ * Contiguous caches return KVC_ERR_UNSUPPORTED.  A page id outside the pool skips that
+ * pair and sets KVC_ERR_BOUNDS.
+ */
+kvc_status kvc_copy_pages(kvc_cache* cache, const int32_t* src, const int32_t* dst, int n,
+                          void* stream);
 
 /*
  * kvc_plan_splits -- how kvc_attend would divide the work for these arguments (for

@@ -68,6 +68,9 @@ def library() -> ctypes.CDLL:
         "kvc_v_pool": ([P, I], P),
         "kvc_layer_pool_bytes": ([P], SZ),
         "kvc_plan_splits": ([P, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I)], I),
+        "kvc_commit": ([P, P, P, I, P], I),
+        "kvc_rollback": ([P, P, P, P], I),
+        "kvc_copy_pages": ([P, P, P, I, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -169,6 +172,19 @@ def kvc_plan_splits(cache: int, H_q: int, T_new: int, max_pages: int = 0) -> tup
     _check(library().kvc_plan_splits(cache, H_q, T_new, max_pages, ctypes.byref(ns),
                                      ctypes.byref(st)), "kvc_plan_splits")
     return ns.value, st.value
+
+
+def kvc_commit(cache: int, seq_lens: int, accepted: int, T_new: int, stream: int) -> None:
+    _check(library().kvc_commit(cache, seq_lens, accepted, T_new, stream or None), "kvc_commit")
+
+
+def kvc_rollback(cache: int, seq_lens: int, drop: int, stream: int) -> None:
+    _check(library().kvc_rollback(cache, seq_lens, drop, stream or None), "kvc_rollback")
+
+
+def kvc_copy_pages(cache: int, src: int, dst: int, n: int, stream: int) -> None:
+    _check(library().kvc_copy_pages(cache, src or None, dst or None, n, stream or None),
+           "kvc_copy_pages")
 
 
 # ---------------------------------------------------------------------------
@@ -291,3 +307,24 @@ class KVCache:
 
     def plan(self, H_q: int, T_new: int, max_pages: int = 0) -> tuple[int, int]:
         return kvc_plan_splits(self.handle, H_q, T_new, max_pages)
+
+    def commit(self, seq_lens, accepted, T_new: int, stream=None) -> None:
+        """seq_lens[b] += accepted[b] on the device (0 <= accepted[b] <= T_new)."""
+        import torch
+        kvc_commit(self.handle, self._dev(seq_lens, "seq_lens", torch.int32),
+                   self._dev(accepted, "accepted", torch.int32), int(T_new), self._stream(stream))
+
+    def rollback(self, seq_lens, drop, stream=None) -> None:
+        """seq_lens[b] -= drop[b] on the device (0 <= drop[b] <= seq_lens[b])."""
+        import torch
+        kvc_rollback(self.handle, self._dev(seq_lens, "seq_lens", torch.int32),
+                     self._dev(drop, "drop", torch.int32), self._stream(stream))
+
+    def copy_pages(self, src, dst, stream=None) -> None:
+        """Page dst[i] := page src[i] in every layer, K and V (paged caches)."""
+        import torch
+        n = int(src.numel())
+        if int(dst.numel()) != n:
+            raise ValueError("src and dst must hold the same number of pages")
+        kvc_copy_pages(self.handle, self._dev(src, "src", torch.int32) if n else 0,
+                       self._dev(dst, "dst", torch.int32) if n else 0, n, self._stream(stream))

@@ -15,6 +15,7 @@
 #include "attend_mma.cuh"
 #include "attend_streamk.cuh"
 #include "attend_tc.cuh"
+#include "cache_ops.cuh"
 #include "kvc.h"
 
 struct kvc_cache {
@@ -693,6 +694,40 @@ kvc_status kvc_append(kvc_cache* c, int layer, const void* k_new, const void* v_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (c->paged) kvc::append_kernel<true><<<blocks, 256, 0, s>>>(p);
   else kvc::append_kernel<false><<<blocks, 256, 0, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+kvc_status kvc_commit(kvc_cache* c, int32_t* seq_lens, const int32_t* accepted, int T_new,
+                      void* stream) {
+  if (!c || !seq_lens || !accepted || T_new <= 0 || !aligned4(seq_lens) || !aligned4(accepted))
+    return KVC_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kvc::commit_kernel<<<(c->B + 127) / 128, 128, 0, s>>>(seq_lens, accepted, c->B, T_new,
+                                                          c->max_T, c->d_err);
+  return cuda_status(cudaGetLastError());
+}
+
+kvc_status kvc_rollback(kvc_cache* c, int32_t* seq_lens, const int32_t* drop, void* stream) {
+  if (!c || !seq_lens || !drop || !aligned4(seq_lens) || !aligned4(drop))
+    return KVC_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kvc::rollback_kernel<<<(c->B + 127) / 128, 128, 0, s>>>(seq_lens, drop, c->B, c->d_err);
+  return cuda_status(cudaGetLastError());
+}
+
+kvc_status kvc_copy_pages(kvc_cache* c, const int32_t* src, const int32_t* dst, int n,
+                          void* stream) {
+  if (!c || n < 0 || (n > 0 && (!src || !dst || !aligned4(src) || !aligned4(dst))))
+    return KVC_ERR_INVALID_ARG;
+  if (!c->paged) return KVC_ERR_UNSUPPORTED;
+  if (n == 0) return KVC_OK;
+  if (2LL * c->num_layers > 65535) return KVC_ERR_UNSUPPORTED;
+  const size_t page_bytes = (size_t)c->H_kv * c->page_size * c->D * kEltBytes;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid((unsigned)n, (unsigned)(2 * c->num_layers));
+  kvc::copy_pages_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<uint4*>(c->pool),
+                                               c->layer_bytes / 16, src, dst, n, c->num_layers,
+                                               c->num_pages, (int)(page_bytes / 16), c->d_err);
   return cuda_status(cudaGetLastError());
 }
 

@@ -74,6 +74,12 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_attend.restype = None
     lib.oracle_attend_chunked.argtypes = [I, I, I, I, I, I, P, P, P, I, P, D, I, P, I]
     lib.oracle_attend_chunked.restype = None
+    lib.oracle_commit.argtypes = [I, P, P, I, I]
+    lib.oracle_commit.restype = I
+    lib.oracle_rollback.argtypes = [I, P, P]
+    lib.oracle_rollback.restype = I
+    lib.oracle_copy_pages.argtypes = [I, I64, P, P, I, P]
+    lib.oracle_copy_pages.restype = I
     return lib
 
 
@@ -165,6 +171,35 @@ class Oracle:
             assert np.all((pages >= 0) & (pages < num_pages))
         self.lib.oracle_append_paged(B, H_kv, T_new, D, P, max_pages, _ptr(new_kv),
                                      _ptr(sl), _ptr(bt), _ptr(pool))
+
+    # -- commit / rollback / page copy -----------------------------------
+    def commit(self, seq_lens, accepted, T_new: int, max_T: int) -> tuple[np.ndarray, int]:
+        """New lengths after accepting accepted[b] of T_new appended tokens, and the
+        number of requests left unchanged because their count was out of range."""
+        sl = _i32(seq_lens).copy()
+        acc = _i32(accepted)
+        assert acc.shape == sl.shape
+        bad = self.lib.oracle_commit(sl.size, _ptr(sl), _ptr(acc), int(T_new), int(max_T))
+        return sl, int(bad)
+
+    def rollback(self, seq_lens, drop) -> tuple[np.ndarray, int]:
+        """New lengths after dropping drop[b] committed tokens, and the number of
+        requests left unchanged because their count was out of range."""
+        sl = _i32(seq_lens).copy()
+        dr = _i32(drop)
+        assert dr.shape == sl.shape
+        bad = self.lib.oracle_rollback(sl.size, _ptr(sl), _ptr(dr))
+        return sl, int(bad)
+
+    def copy_pages(self, pool, src, dst) -> int:
+        """pool (num_pages, ...) uint16, updated in place: page dst[i] := page src[i].
+        Returns the number of pairs skipped for an id outside the pool."""
+        assert pool.dtype == np.uint16 and pool.flags["C_CONTIGUOUS"]
+        s, d = _i32(src), _i32(dst)
+        assert s.shape == d.shape
+        page_elems = int(np.prod(pool.shape[1:]))
+        return int(self.lib.oracle_copy_pages(pool.shape[0], page_elems, _ptr(s), _ptr(d),
+                                              s.size, _ptr(pool)))
 
     def gather_paged(self, pool, block_table, n_visible, T_cap: int) -> np.ndarray:
         """Logical (B,H_kv,T_cap,D) view of the first n_visible[b] positions (rest zero)."""

@@ -184,6 +184,63 @@ void oracle_append_paged(int B, int H_kv, int T_new, int D, int P, int max_pages
             }
 }
 
+/* ------------------------------------------------------------------ */
+/* Commit, rollback and page copy ([P1]: a two-phase append/commit      */
+/* cache; speculative decoding keeps the accepted prefix of the         */
+/* verified tokens and rolls the rest back; [P3] 9.6: fixed-size pages).*/
+/* A request (or page pair) whose values are out of range is left as it */
+/* is; the number of those is returned.                                 */
+/* ------------------------------------------------------------------ */
+
+/* seq_lens[b] becomes seq_lens[b] + accepted[b] when 0 <= accepted[b] <= T_new
+ * and the result stays within the capacity max_T. */
+int oracle_commit(int B, int32_t* seq_lens, const int32_t* accepted, int T_new, int max_T)
+{
+    int rejected = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t grown = (int64_t)seq_lens[b] + accepted[b];
+        if (accepted[b] < 0 || accepted[b] > T_new || seq_lens[b] < 0 || grown > max_T) {
+            ++rejected;
+            continue;
+        }
+        seq_lens[b] = (int32_t)grown;
+    }
+    return rejected;
+}
+
+/* seq_lens[b] becomes seq_lens[b] - drop[b] when 0 <= drop[b] <= seq_lens[b]. */
+int oracle_rollback(int B, int32_t* seq_lens, const int32_t* drop)
+{
+    int rejected = 0;
+    for (int b = 0; b < B; ++b) {
+        if (drop[b] < 0 || drop[b] > seq_lens[b]) {
+            ++rejected;
+            continue;
+        }
+        seq_lens[b] -= drop[b];
+    }
+    return rejected;
+}
+
+/* One pool of num_pages pages of page_elems elements: page dst[i] receives a
+ * copy of page src[i] for every i < n whose two ids lie in [0, num_pages). */
+int oracle_copy_pages(int num_pages, int64_t page_elems, const int32_t* src,
+                      const int32_t* dst, int n, uint16_t* pool)
+{
+    int rejected = 0;
+    for (int i = 0; i < n; ++i) {
+        if (src[i] < 0 || src[i] >= num_pages || dst[i] < 0 || dst[i] >= num_pages) {
+            ++rejected;
+            continue;
+        }
+        const uint16_t* from = pool + (int64_t)src[i] * page_elems;
+        uint16_t* to = pool + (int64_t)dst[i] * page_elems;
+        for (int64_t e = 0; e < page_elems; ++e)
+            to[e] = from[e];
+    }
+    return rejected;
+}
+
 /* Logical view of request b's first n_b positions from the paged pool:
  * out (B, H_kv, T_cap, D), rows >= n_b left untouched. */
 void oracle_gather_paged(int B, int H_kv, int D, int P, int max_pages, int T_cap,

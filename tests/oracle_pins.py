@@ -25,7 +25,14 @@ What pins what:
   project 12), a request's result does not depend on its batch mates
   (inference chapter 9.10: test batch 1 and batch 2);
 * the paged layout -- a shuffled pool read through its block table gives the
-  same logical rows as the contiguous cache ("9. 推理" section 9.6).
+  same logical rows as the contiguous cache ("9. 推理" section 9.6);
+* commit / rollback / page copy ("llm-perf-lab" README: two-phase
+  append/commit, speculative decoding keeps the accepted prefix) -- a
+  speculative round (append gamma drafts, commit the accepted ones, append the
+  next token) attends exactly like plain cached decoding of the accepted
+  prefix; commit then rollback of the same counts is the identity; out-of-range
+  counts change nothing; copy-on-write of a shared, partly filled page leaves
+  every request's logical cache equal to an unshared contiguous cache.
 """
 from __future__ import annotations
 
@@ -389,6 +396,87 @@ def check_paged_equals_contig(o):
         assert np.array_equal(logical[b, :, :n], contig[b, :, :n])
 
 
+def check_speculative_round_equals_plain_decode(o):
+    """Verify gamma drafts, keep the first a_b, append the next token: the next step's
+    output equals cached decoding that only ever appended the accepted tokens."""
+    B, H_q, H_kv, D, gamma = 3, 4, 2, 32, 4
+    L0 = np.array([5, 0, 11], np.int32)
+    acc = np.array([2, 0, 4], np.int32)
+    T_cap = int(L0.max()) + gamma + 3   # slack rows: a planted off-by-one stays in bounds
+    scale = 0.25
+    for dtype in (FP16, BF16):
+        dt = DT[dtype]
+        hist_k = normal_bits((B, H_kv, T_cap, D), dt, 21, "spec_hk")
+        hist_v = normal_bits((B, H_kv, T_cap, D), dt, 21, "spec_hv")
+        draft_k = normal_bits((B, H_kv, gamma, D), dt, 21, "spec_dk")
+        draft_v = normal_bits((B, H_kv, gamma, D), dt, 21, "spec_dv")
+        nxt_k = normal_bits((B, H_kv, 1, D), dt, 21, "spec_nk")
+        nxt_v = normal_bits((B, H_kv, 1, D), dt, 21, "spec_nv")
+        q = normal_bits((B, H_q, 1, D), dt, 21, "spec_q")
+        # speculative: append gamma drafts, commit acc, append the next token
+        Ks, Vs = hist_k.copy(), hist_v.copy()
+        o.append_contig(Ks, draft_k, L0)
+        o.append_contig(Vs, draft_v, L0)
+        L1, bad = o.commit(L0, acc, gamma, T_cap)
+        assert bad == 0
+        o.append_contig(Ks, nxt_k, L1)
+        o.append_contig(Vs, nxt_v, L1)
+        spec = o.attend(q, Ks, Vs, L1, scale, dtype, nthreads=2)
+        # plain: per request, the history, then only the accepted drafts, then the token
+        Kp, Vp = hist_k.copy(), hist_v.copy()
+        for b in range(B):
+            a, l0 = int(acc[b]), int(L0[b])
+            Kp[b, :, l0:l0 + a] = draft_k[b, :, :a]
+            Vp[b, :, l0:l0 + a] = draft_v[b, :, :a]
+            Kp[b, :, l0 + a] = nxt_k[b, :, 0]
+            Vp[b, :, l0 + a] = nxt_v[b, :, 0]
+        plain = o.attend(q, Kp, Vp, L0 + acc, scale, dtype, nthreads=2)
+        assert np.array_equal(spec, plain)
+
+
+def check_commit_rollback(o):
+    L = np.array([0, 7, 100, 3], np.int32)
+    a = np.array([3, 0, 2, 1], np.int32)
+    L1, bad = o.commit(L, a, 3, 1000)
+    assert bad == 0 and np.array_equal(L1 - L, a)
+    L2, bad = o.rollback(L1, a)
+    assert bad == 0 and np.array_equal(L2, L)
+    # out-of-range counts and capacity overflow leave a request as it is
+    L3, bad = o.commit(L, np.array([4, -1, 2, 0], np.int32), 3, 101)
+    assert bad == 3 and np.array_equal(L3, np.array([0, 7, 100, 3]))
+    L4, bad = o.rollback(L, np.array([1, 8, 100, -2], np.int32))
+    assert bad == 3 and np.array_equal(L4, np.array([0, 7, 0, 3]))
+
+
+def check_copy_on_write(o):
+    """Two requests share prefix pages, the last one partly filled; request 1 copies
+    that page, re-points its table and both append: every request's logical cache
+    equals its own unshared contiguous cache, and the skipped pairs change nothing."""
+    H_kv, D, P = 2, 8, 4
+    prefix = 6                       # pages 0 (full) and 1 (half) shared
+    T_cap = prefix + 1
+    shared = normal_bits((1, H_kv, prefix, D), "fp16", 31, "cow_prefix")[0]
+    new = normal_bits((2, H_kv, 1, D), "fp16", 31, "cow_new")
+    num_pages = 5
+    pool = np.full((num_pages, H_kv, P, D), np.uint16(0x3C00), np.uint16)
+    for pos in range(prefix):
+        pool[pos // P, :, pos % P] = shared[:, pos]
+    bt = np.array([[0, 1, 4, 4], [0, 1, 4, 4]], np.int32)   # spare columns: a valid page
+    before = pool.copy()
+    assert o.copy_pages(pool, [1, 9, -1], [3, 2, 4]) == 2      # one valid pair
+    assert np.array_equal(pool[3], before[1])
+    assert np.array_equal(np.delete(pool, 3, axis=0), np.delete(before, 3, axis=0))
+    bt[1, 1] = 3                                               # request 1 owns its copy
+    L = np.array([prefix, prefix], np.int32)
+    o.append_paged(pool, new, L, bt)
+    logical = o.gather_paged(pool, bt, L + 1, T_cap)
+    for b in range(2):
+        contig = np.zeros((1, H_kv, T_cap, D), np.uint16)
+        contig[0, :, :prefix] = shared
+        o.append_contig(contig, np.ascontiguousarray(new[b:b + 1]), L[b:b + 1])
+        assert np.array_equal(logical[b], contig[0]), f"request {b}"
+
+
 ALL_CHECKS = [
     check_decode_fp16_exhaustive,
     check_decode_bf16_exhaustive,
@@ -403,4 +491,7 @@ ALL_CHECKS = [
     check_gqa_equals_expanded_mha,
     check_batch_invariance,
     check_paged_equals_contig,
+    check_speculative_round_equals_plain_decode,
+    check_commit_rollback,
+    check_copy_on_write,
 ]

@@ -49,6 +49,14 @@ MUTANTS = [
     ("kv_bytes_without_k_and_v", "return (uint64_t)2 *", "return (uint64_t)1 *", 0),
     ("chunked_no_rescale_of_sum", "l *= alpha;", "l *= 1.0;", 0),
     ("chunked_no_rescale_of_acc", "acc[d] *= alpha;", "acc[d] *= 1.0;", 0),
+    ("commit_one_too_far", "seq_lens[b] = (int32_t)grown;", "seq_lens[b] = (int32_t)grown + 1;", 0),
+    ("commit_accepts_past_chunk", "accepted[b] > T_new ||", "accepted[b] > T_new + 1 ||", 0),
+    ("rollback_adds", "seq_lens[b] -= drop[b];", "seq_lens[b] += drop[b];", 0),
+    ("copy_pages_reversed",
+     "const uint16_t* from = pool + (int64_t)src[i] * page_elems;\n        uint16_t* to = pool + (int64_t)dst[i] * page_elems;",
+     "const uint16_t* from = pool + (int64_t)dst[i] * page_elems;\n        uint16_t* to = pool + (int64_t)src[i] * page_elems;", 0),
+    ("copy_pages_half_page", "for (int64_t e = 0; e < page_elems; ++e)",
+     "for (int64_t e = 0; e < page_elems / 2; ++e)", 0),
 ]
 
 
