@@ -132,6 +132,21 @@ kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T
                       float scale, void* out, void* stream);
 
 /*
+ * kvc_attend_window -- kvc_attend restricted to a sliding window with attention sinks
+ * ("项目 9-16" roadmap: sliding-window attention over the last W positions, with the
+ * first positions kept as attention sinks).  New row i of request b (n = L_b + i + 1
+ * positions, causal within the chunk) attends position j iff
+ *     j < n  and  (j >= n - window  or  j < sink);
+ * window = 0 means no window (exactly kvc_attend; sink is then irrelevant).  Only the
+ * positions some row of a block can see are read, so the cost follows W + sink, not n.
+ * Other arguments, layouts and errors as kvc_attend; window or sink < 0 is
+ * KVC_ERR_INVALID_ARG.
+ */
+kvc_status kvc_attend_window(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
+                             const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                             float scale, int window, int sink, void* out, void* stream);
+
+/*
  * kvc_append_attend -- kvc_append followed by kvc_attend for the same new tokens, in
  * one launch where the kernel allows it ("9. 推理" 9.3: the new token's K/V join the
  * cache and are attended in the same step).  Arguments are those of the two calls.

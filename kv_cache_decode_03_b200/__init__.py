@@ -60,6 +60,7 @@ def library() -> ctypes.CDLL:
         "kvc_append": ([P, I, P, P, I, P, I, P, P], I),
         "kvc_attend": ([P, I, P, I, I, P, I, P, F, P, P], I),
         "kvc_attend_noalloc": ([P, I, P, I, I, P, I, P, F, P, P], I),
+        "kvc_attend_window": ([P, I, P, I, I, P, I, P, F, I, I, P, P], I),
         "kvc_append_attend": ([P, I, P, P, P, I, I, P, I, P, F, P, P], I),
         "kvc_reserve": ([P, I, I, I], I),
         "kvc_get_error": ([P], I),
@@ -126,6 +127,14 @@ def kvc_attend(cache: int, layer: int, q: int, H_q: int, T_new: int, block_table
                max_pages: int, seq_lens: int, scale: float, out: int, stream: int) -> None:
     _check(library().kvc_attend(cache, layer, q, H_q, T_new, block_table or None, max_pages,
                                 seq_lens, scale, out, stream or None), "kvc_attend")
+
+
+def kvc_attend_window(cache: int, layer: int, q: int, H_q: int, T_new: int, block_table: int,
+                      max_pages: int, seq_lens: int, scale: float, window: int, sink: int,
+                      out: int, stream: int) -> None:
+    _check(library().kvc_attend_window(cache, layer, q, H_q, T_new, block_table or None,
+                                       max_pages, seq_lens, scale, window, sink, out,
+                                       stream or None), "kvc_attend_window")
 
 
 def kvc_append_attend(cache: int, layer: int, k_new: int, v_new: int, q: int, H_q: int,
@@ -278,6 +287,24 @@ class KVCache:
         kvc_attend(self.handle, layer, self._dev(q, "q", self.torch_dtype), H_q, T_new, bt, mp,
                    self._dev(seq_lens, "seq_lens", torch.int32), float(scale),
                    self._dev(out, "out", self.torch_dtype), self._stream(stream))
+        return out
+
+    def attend_window(self, layer: int, q, seq_lens, window: int, sink: int = 0,
+                      block_table=None, scale: float | None = None, out=None, stream=None):
+        """Attention over the last `window` positions plus the first `sink` of each row."""
+        import torch
+        B, H_q, T_new, D = (int(x) for x in q.shape)
+        assert B == self.B and D == self.D
+        if out is None:
+            out = torch.empty_like(q)
+        if scale is None:
+            scale = 1.0 / D ** 0.5
+        bt = 0 if block_table is None else self._dev(block_table, "block_table", torch.int32)
+        mp = 0 if block_table is None else int(block_table.shape[1])
+        kvc_attend_window(self.handle, layer, self._dev(q, "q", self.torch_dtype), H_q, T_new,
+                          bt, mp, self._dev(seq_lens, "seq_lens", torch.int32), float(scale),
+                          int(window), int(sink), self._dev(out, "out", self.torch_dtype),
+                          self._stream(stream))
         return out
 
     def append_attend(self, layer: int, k_new, v_new, q, seq_lens, block_table=None,

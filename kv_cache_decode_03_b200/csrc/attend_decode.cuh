@@ -141,16 +141,17 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 2)
     }
   const int n_blk = L + i_max + 1;  // positions the block must read
   const int vis_min = L + i_min + 1;
-  const int t_begin = s * p.split_tokens;
-  if (t_begin >= n_blk) return;  // the slice is past every row's horizon
+  const Span sp = block_span(vis_min, n_blk, p.window, p.sink, C::kTile);
+  const int t_begin = s * p.split_tokens;  // virtual positions (window.cuh)
+  if (t_begin >= sp.n_virt) return;  // the slice is past every row's horizon
   if (L < 0 || L + p.T_new > p.max_T ||
       (PAGED && ((L + p.T_new - 1) >> p.page_shift) >= p.max_pages)) {
     if (threadIdx.x == 0) flag_error(p.err, KVC_ERR_BOUNDS);
     return;
   }
-  const int t_stop = min(t_begin + p.split_tokens, n_blk);
+  const int t_stop = min(t_begin + p.split_tokens, sp.n_virt);
   const int ntiles = ceil_div(t_stop - t_begin, C::kTile);
-  const int ns_blk = ceil_div(n_blk, p.split_tokens);
+  const int ns_blk = ceil_div(sp.n_virt, p.split_tokens);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -173,8 +174,9 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 2)
   const uint64_t pol = l2_policy_evict_first();
   auto issue = [&](int j) {
     const int st = j % C::kStages;
-    const int t0 = t_begin + j * C::kTile;
-    const int t1 = min(t0 + C::kTile, t_stop);
+    const int t0v = t_begin + j * C::kTile;
+    const int t0 = sp.real(t0v);
+    const int t1 = t0 + min(C::kTile, t_stop - t0v);
     unsigned char* dk = sk + st * C::kTileBytes;
     unsigned char* dv = sv + st * C::kTileBytes;
     const char* kp = static_cast<const char*>(p.k_pool);
@@ -285,9 +287,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 2)
     consumed = j + 1;
     const unsigned char* tk = sk + st * C::kTileBytes;
     const unsigned char* tv = sv + st * C::kTileBytes;
-    const int t0 = t_begin + j * C::kTile;
-    const int valid = min(C::kTile, t_stop - t0);
-    const bool unmasked = (t0 + C::kTile <= vis_min);  // every row sees the whole tile
+    const int t0v = t_begin + j * C::kTile;
+    const int t0 = sp.real(t0v);
+    const int valid = min(C::kTile, t_stop - t0v);
+    const bool unmasked =  // every row sees the whole tile
+        tile_fully_visible(t0, C::kTile, vis_min, n_blk, p.window, p.sink);
 
     float sc[C::kPasses][R];
 #pragma unroll
@@ -315,7 +319,8 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 2)
       } else {
         const int pos = t0 + tok;
 #pragma unroll
-        for (int rr = 0; rr < R; ++rr) sc[pp][rr] = (pos < vis[rr]) ? part[rr] : -INFINITY;
+        for (int rr = 0; rr < R; ++rr)
+          sc[pp][rr] = visible(pos, vis[rr], p.window, p.sink) ? part[rr] : -INFINITY;
       }
     }
 
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 2)
   named_barrier_sync(1, NT);
 
   finish_slice<T, D, R, W, NT>(p, red_acc, red_m, red_l, red_acc + W * R * D, &flags[1], b, g,
-                               rb, s, r0, nr, L, ns_blk);
+                               rb, s, r0, nr, L, ns_blk, sp);
 }
 
 }  // namespace kvc

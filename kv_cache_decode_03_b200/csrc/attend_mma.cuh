@@ -114,16 +114,17 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
   }
   const int n_blk = L + i_max + 1;
   const int vis_min = L + i_min + 1;
-  const int t_begin = s * p.split_tokens;
-  if (t_begin >= n_blk) return;
+  const Span sp = block_span(vis_min, n_blk, p.window, p.sink, C::kTile);
+  const int t_begin = s * p.split_tokens;  // virtual positions (window.cuh)
+  if (t_begin >= sp.n_virt) return;
   if (L < 0 || L + p.T_new > p.max_T ||
       (PAGED && ((L + p.T_new - 1) >> p.page_shift) >= p.max_pages)) {
     if (threadIdx.x == 0) flag_error(p.err, KVC_ERR_BOUNDS);
     return;
   }
-  const int t_stop = min(t_begin + p.split_tokens, n_blk);
+  const int t_stop = min(t_begin + p.split_tokens, sp.n_virt);
   const int ntiles = ceil_div(t_stop - t_begin, C::kTile);
-  const int ns_blk = ceil_div(n_blk, p.split_tokens);
+  const int ns_blk = ceil_div(sp.n_virt, p.split_tokens);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -147,7 +148,9 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
   const uint64_t pol = p.row_blocks > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
   auto issue = [&](int j) {
     const int st = j % C::kStages;
-    const int t0 = t_begin + j * C::kTile;
+    const int t0v = t_begin + j * C::kTile;
+    const int t0 = sp.real(t0v);
+    const int t_end = t0 + (t_stop - t0v);  // real end of the slice within this tile's run
     unsigned char* dk = sk + st * C::kTileBytes;
     unsigned char* dv = sv + st * C::kTileBytes;
     mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes);  // every box is full (zero fill)
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
 #pragma unroll 1
       for (int t = t0; t < t0 + C::kTile; t += box_rows) {
         int y = beyond;
-        if (t < t_stop) {
+        if (t < t_end) {
           const int page = bt[t >> p.page_shift];
           if (page >= 0 && page < p.num_pages)
             y = (page * p.H_kv + g) * P + (t & (P - 1));
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
     consumed = j + 1;
     const uint32_t kb = sk_addr + st * C::kTileBytes;
     const uint32_t vb = sv_addr + st * C::kTileBytes;
-    const int t0 = t_begin + j * C::kTile;
+    const int t0 = sp.real(t_begin + j * C::kTile);
 
     // S^T = K . Q^T for this warp's 16 tokens
     float sacc[NT][4];
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
 
     // scale to base-2 units, mask, online softmax per score column (query row)
     const int tok0 = t0 + wrow + (lane >> 2);
-    const bool unmasked = (t0 + C::kTile <= vis_min);
+    const bool unmasked = tile_fully_visible(t0, C::kTile, vis_min, n_blk, p.window, p.sink);
     bool grew = false;
     float alpha[NT][2];
 #pragma unroll
@@ -289,8 +292,8 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
         float s0 = sacc[nt][c] * p.scale_log2;
         float s1 = sacc[nt][2 + c] * p.scale_log2;
         if (!unmasked) {
-          s0 = (tok0 < vis[nt][c]) ? s0 : -INFINITY;
-          s1 = (tok0 + 8 < vis[nt][c]) ? s1 : -INFINITY;
+          s0 = visible(tok0, vis[nt][c], p.window, p.sink) ? s0 : -INFINITY;
+          s1 = visible(tok0 + 8, vis[nt][c], p.window, p.sink) ? s1 : -INFINITY;
         }
         float mx = fmaxf(s0, s1);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
@@ -320,11 +323,17 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
         }
     }
     // P^T fragments: transpose each 8x8 (token x row) block into (row x token)
-    uint32_t pb[NT][2];
+    uint32_t pb[NT][2], pl[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      pb[nt][0] = movmatrix_trans(Elt<T>::pack2(sacc[nt][0], sacc[nt][1]));
-      pb[nt][1] = movmatrix_trans(Elt<T>::pack2(sacc[nt][2], sacc[nt][3]));
+      const uint32_t h0 = Elt<T>::pack2(sacc[nt][0], sacc[nt][1]);
+      const uint32_t h1 = Elt<T>::pack2(sacc[nt][2], sacc[nt][3]);
+      pb[nt][0] = movmatrix_trans(h0);
+      pb[nt][1] = movmatrix_trans(h1);
+      if constexpr (SplitP<T>::kOn) {  // bf16: the weights' rounding remainders
+        pl[nt][0] = movmatrix_trans(bf16_remainder2(sacc[nt][0], sacc[nt][1], h0));
+        pl[nt][1] = movmatrix_trans(bf16_remainder2(sacc[nt][2], sacc[nt][3], h1));
+      }
     }
     // O^T += V^T . P^T
 #pragma unroll
@@ -332,7 +341,10 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
       uint32_t a[4];
       ldmatrix_x4_trans(a, vb + swz<D>(v_row, 2 * mt + v_cs));
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+        if constexpr (SplitP<T>::kOn) mma_16816<T>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
@@ -378,7 +390,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads)
   }
   named_barrier_sync(1, NTH);
   finish_slice<T, D, R, W, NTH>(p, red_acc, red_m, red_l, red_acc + W * R * D, &flags[1], b, g,
-                                rb, s, r0, nr, L, ns_blk);
+                                rb, s, r0, nr, L, ns_blk, sp);
 }
 
 }  // namespace kvc

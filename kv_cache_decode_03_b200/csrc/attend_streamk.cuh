@@ -467,18 +467,27 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
           o[mt][nt][3] *= alpha[nt][1];
         }
     }
-    uint32_t pb[NT][2];
+    uint32_t pb[NT][2], pl[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      pb[nt][0] = movmatrix_trans(Elt<T>::pack2(sacc[nt][0], sacc[nt][1]));
-      pb[nt][1] = movmatrix_trans(Elt<T>::pack2(sacc[nt][2], sacc[nt][3]));
+      const uint32_t h0 = Elt<T>::pack2(sacc[nt][0], sacc[nt][1]);
+      const uint32_t h1 = Elt<T>::pack2(sacc[nt][2], sacc[nt][3]);
+      pb[nt][0] = movmatrix_trans(h0);
+      pb[nt][1] = movmatrix_trans(h1);
+      if constexpr (SplitP<T>::kOn) {  // bf16: the weights' rounding remainders
+        pl[nt][0] = movmatrix_trans(bf16_remainder2(sacc[nt][0], sacc[nt][1], h0));
+        pl[nt][1] = movmatrix_trans(bf16_remainder2(sacc[nt][2], sacc[nt][3], h1));
+      }
     }
 #pragma unroll
     for (int mt = 0; mt < C::kMTiles; ++mt) {
       uint32_t a[4];
       ldmatrix_x4_trans(a, vb + swz<D>(v_row, 2 * mt + v_cs));
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+        if constexpr (SplitP<T>::kOn) mma_16816<T>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+      }
     }
 
     const bool piece_end = (j == ntiles - 1) || (cur.k == cur.seg_tiles - 1);

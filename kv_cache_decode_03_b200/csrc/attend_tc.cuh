@@ -248,8 +248,15 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     if (i1 >= i0) i_max = i1;
   }
   const int n_blk = L + i_max + 1;
-  const int t_begin = s * p.split_tokens;
-  if (t_begin >= n_blk) return;
+  int i_min = 0;  // first new row of the block
+  if (nr < p.T_new) {
+    const int i0 = r0 % p.T_new, i1 = (r0 + nr - 1) % p.T_new;
+    if (i1 >= i0) i_min = i0;
+  }
+  const int vis_min = L + i_min + 1;
+  const Span sp = block_span(vis_min, n_blk, p.window, p.sink, C::kTile);
+  const int t_begin = s * p.split_tokens;  // virtual positions (window.cuh)
+  if (t_begin >= sp.n_virt) return;
   if (smem_addr(smem) & 1023u) {  // swizzle atoms need 1024-byte alignment
     if (tid == 0) flag_error(p.err, KVC_ERR_UNSUPPORTED);
     return;
@@ -259,9 +266,9 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     if (tid == 0) flag_error(p.err, KVC_ERR_BOUNDS);
     return;
   }
-  const int t_stop = min(t_begin + p.split_tokens, n_blk);
+  const int t_stop = min(t_begin + p.split_tokens, sp.n_virt);
   const int ntiles = ceil_div(t_stop - t_begin, C::kTile);
-  const int ns_blk = ceil_div(n_blk, p.split_tokens);
+  const int ns_blk = ceil_div(sp.n_virt, p.split_tokens);
 
   // ---- TMEM, barriers, and Q: row tid in 64-element boxes, 128-byte swizzled
   if (warp == 0) {
@@ -354,7 +361,9 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
           break;
         }
       }
-      const int t0 = t_begin + j * C::kTile;
+      const int t0v = t_begin + j * C::kTile;
+      const int t0 = sp.real(t0v);
+      const int t_end = t0 + (t_stop - t0v);  // real end of the slice within this tile's run
       unsigned char* dst = ring + st * C::kTileBytes;
       if (lane_id == 0) mbar_arrive_expect_tx(&full[st], C::kTileBytes);
       __syncwarp();
@@ -369,7 +378,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
         if (lane_id < nbox) {
           const int t = t0 + lane_id * box_rows;
           int y = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
-          if (t < t_stop) {
+          if (t < t_end) {
             const int page = p.block_table[(size_t)b * p.max_pages + (t >> p.page_shift)];
             if (page >= 0 && page < p.num_pages)
               y = (page * p.H_kv + g) * Pg + (t & (Pg - 1));
@@ -459,12 +468,12 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 32; ++c) sc[c] = __fmul2_rn(sc[c], sc2);
-      const int t0 = t_begin + j * C::kTile;
-      if (__any_sync(0xffffffffu, t0 + C::kTile > vis)) {  // tile reaches past some row's end
+      const int t0 = sp.real(t_begin + j * C::kTile);
+      if (!tile_fully_visible(t0, C::kTile, vis_min, n_blk, p.window, p.sink)) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          if (t0 + 2 * c >= vis) sc[c].x = -INFINITY;
-          if (t0 + 2 * c + 1 >= vis) sc[c].y = -INFINITY;
+          if (!visible(t0 + 2 * c, vis, p.window, p.sink)) sc[c].x = -INFINITY;
+          if (!visible(t0 + 2 * c + 1, vis, p.window, p.sink)) sc[c].y = -INFINITY;
         }
       }
       float mx = -INFINITY;
@@ -573,7 +582,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
                  "r"(C::kTmemCols)
                  : "memory");
   finish_slice<T, D, R, 1, NSM, C::kAccLd>(p, red_acc, red_m, red_l, scratch, &flags[1], b, g,
-                                           rb, s, r0, nr, L, ns_blk);
+                                           rb, s, r0, nr, L, ns_blk, sp);
 }
 
 }  // namespace kvc

@@ -160,6 +160,21 @@ struct Elt<__nv_bfloat16> {
   }
 };
 
+// Softmax weights enter the p.V product in the cache's 16-bit type.  A bf16 weight
+// (8-bit significand) moves short-context outputs past the 2e-3 bound, so bf16
+// weights are split as hi + lo (both bf16, lo the rounding remainder) and both
+// products accumulate; fp16 weights (11-bit significand) stay whole.
+template <typename T>
+struct SplitP {
+  static constexpr bool kOn = Elt<T>::kCode == KVC_BF16;
+};
+
+// The bf16 pair of remainders a - hi.x, b - hi.y of a packed bf16 pair hi.
+__device__ __forceinline__ uint32_t bf16_remainder2(float a, float b, uint32_t hi) {
+  return Elt<__nv_bfloat16>::pack2(a - __uint_as_float(hi << 16),
+                                   b - __uint_as_float(hi & 0xFFFF0000u));
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(const void* p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"

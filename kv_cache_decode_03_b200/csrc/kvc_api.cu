@@ -298,7 +298,9 @@ int occupancy(const kvc_cache* c, int R) {
                               : occupancy_for<__half>(c->D, R, c->paged);
 }
 
-Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
+// window / sink: sliding-window attention (window.cuh); 0 = full attention.
+Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window = 0,
+               int sink = 0) {
   Plan pl{};
   const int rows = (H_q / c->H_kv) * T_new;
   // Three or more query rows per K/V row make q.k and p.v a dense contraction
@@ -332,7 +334,7 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
   // slots need no split size and every CTA streams the same bytes.
   const int max_batch = c->D == 64 ? kvc::StreamKCfg<64>::kMaxBatch
                                    : kvc::StreamKCfg<128>::kMaxBatch;
-  if (pl.mma && pl.NT <= 2 && c->B <= max_batch) {
+  if (pl.mma && pl.NT <= 2 && c->B <= max_batch && window == 0) {
     pl.streamk = true;
     const int socc = c->dtype == KVC_BF16 ? streamk_occ<__nv_bfloat16>(c->D, pl.NT, c->paged)
                                           : streamk_occ<__half>(c->D, pl.NT, c->paged);
@@ -347,6 +349,9 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages) {
   }
   long long cap = c->max_T;
   if (c->paged) cap = std::min<long long>(cap, (long long)max_pages * c->page_size);
+  if (window > 0)  // a block reads at most its sink tiles and W + T_new positions (+ a tile)
+    cap = std::min<long long>(cap, (long long)(sink + tile - 1) / tile * tile + window + T_new +
+                                       tile);
   cap = std::max<long long>(cap, 1);
   const long long units = (long long)c->B * c->H_kv * pl.row_blocks;
   const long long target = (long long)KVC_SPLIT_WAVES * c->num_sms * occ;
@@ -748,9 +753,9 @@ kvc_status kvc_reserve(kvc_cache* c, int H_q, int T_new, int max_pages) {
   return ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
 }
 
-kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new,
-                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
-                      float scale, void* out, void* stream) {
+kvc_status kvc_attend_window(kvc_cache* c, int layer, const void* q, int H_q, int T_new,
+                             const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                             float scale, int window, int sink, void* out, void* stream) {
   if (!c || layer < 0 || layer >= c->num_layers || T_new <= 0 || H_q <= 0 ||
       H_q % c->H_kv != 0)
     return KVC_ERR_INVALID_ARG;
@@ -759,8 +764,9 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   if (c->paged && (!block_table || !aligned4(block_table) || max_pages <= 0))
     return KVC_ERR_INVALID_ARG;
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
-  if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
-  const Plan pl = make_plan(c, H_q, T_new, max_pages);
+  if (!(scale == scale) || window < 0 || sink < 0) return KVC_ERR_INVALID_ARG;
+  if (window == 0) sink = 0;  // no window: every position is visible anyway
+  const Plan pl = make_plan(c, H_q, T_new, max_pages, window, sink);
   kvc_status st = ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
   if (st != KVC_OK) return st;
   kvc::AttendParams p{};
@@ -781,6 +787,8 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   p.page_shift = c->page_shift;
   p.num_pages = c->num_pages;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.window = window;
+  p.sink = sink;
   p.split_tokens = pl.split_tokens;
   p.num_splits = pl.num_splits;
   p.row_blocks = pl.row_blocks;
@@ -792,6 +800,13 @@ kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new
   p.err = c->d_err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return run_plan(c, layer, pl, p, s);
+}
+
+kvc_status kvc_attend(kvc_cache* c, int layer, const void* q, int H_q, int T_new,
+                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                      float scale, void* out, void* stream) {
+  return kvc_attend_window(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, 0,
+                           0, out, stream);
 }
 
 kvc_status kvc_get_error(kvc_cache* c) {

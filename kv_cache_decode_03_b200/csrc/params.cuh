@@ -33,7 +33,10 @@ struct AttendParams {
   int page_shift;                        // log2(page_size) (paged)
   int num_pages;
   float scale_log2;   // scale * log2(e): scores are kept in base-2 units
-  int split_tokens;   // tokens per split-K slice (a multiple of the tile)
+  int window;         // sliding window W (0 = none): row with n positions sees [n - W, n)
+  int sink;           // ... and the first `sink` positions (window.cuh)
+  int split_tokens;   // tokens per split-K slice (a multiple of the tile; virtual
+                      // positions when a window is set, window.cuh)
   int num_splits;     // slices in the grid
   int row_blocks;     // CTAs per KV head along the query rows
   float* ws_o;        // (B, H_q, T_new, num_splits, D) normalised partial outputs

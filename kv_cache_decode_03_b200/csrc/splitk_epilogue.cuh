@@ -18,6 +18,7 @@
 
 #include "device_common.cuh"
 #include "params.cuh"
+#include "window.cuh"
 
 namespace kvc {
 
@@ -29,25 +30,37 @@ __device__ __forceinline__ void store_elt(T* ptr, float v) {
 
 // red_acc: [W][R] rows of D fp32, LD floats apart; red_m / red_l: [W][R].
 // scratch: >= R * num_splits floats of shared memory that nothing else uses.
-// flags: one shared int.  All NT threads of the CTA call this together after
+// flags: one shared int.  sp: the block's virtual tile span (window.cuh); slices
+// count virtual positions.  All NT threads of the CTA call this together after
 // red_* are written and synced.
 template <typename T, int D, int R, int W, int NT, int LD = D>
 __device__ __forceinline__ void finish_slice(const AttendParams& p, const float* red_acc,
                                              const float* red_m, const float* red_l,
                                              float* scratch, int* flag, int b, int g, int rb,
-                                             int s, int r0, int nr, int L, int ns_blk) {
+                                             int s, int r0, int nr, int L, int ns_blk,
+                                             const Span& sp) {
   const int tid = threadIdx.x;
   T* out = static_cast<T*>(p.out);
   const size_t row_base = ((size_t)b * p.H_q + (size_t)g * p.group) * p.T_new + r0;
+  // slices holding a row's positions: its last visible position, L + i, decides
+  auto row_slices = [&](int i) { return ceil_div(sp.virt(L + i) + 1, p.split_tokens); };
 #pragma unroll 1
   for (int idx = tid; idx < R * D; idx += NT) {
     const int rr = idx / D;
     const int d = idx - rr * D;
     if (rr >= nr) break;  // rows are the outer index
+    const int i = (r0 + rr) % p.T_new;
+    const int ns_row = row_slices(i);
+    if (s >= ns_row) continue;  // the slice is past this row's last position
+    const size_t orow = row_base + rr;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < W; ++w) M = fmaxf(M, red_m[w * R + rr]);
-    if (M == -INFINITY) continue;  // no visible position of this row in the slice
+    if (M == -INFINITY) {  // the row sees nothing here (left of its window): empty partial
+      p.ws_o[(orow * p.num_splits + s) * D + d] = 0.f;
+      if (d == 0) p.ws_lse[orow * p.num_splits + s] = -INFINITY;
+      continue;
+    }
     float lsum = 0.f, o = 0.f;
 #pragma unroll
     for (int w = 0; w < W; ++w) {
@@ -55,9 +68,7 @@ __device__ __forceinline__ void finish_slice(const AttendParams& p, const float*
       lsum = fmaf(red_l[w * R + rr], f, lsum);
       o = fmaf(red_acc[(w * R + rr) * LD + d], f, o);
     }
-    const int i = (r0 + rr) % p.T_new;
-    const size_t orow = row_base + rr;
-    if (ceil_div(L + i + 1, p.split_tokens) == 1) {
+    if (ns_row == 1) {
       store_elt<T>(out + orow * D + d, o / lsum);
     } else {
       p.ws_o[(orow * p.num_splits + s) * D + d] = o / lsum;
@@ -84,8 +95,7 @@ __device__ __forceinline__ void finish_slice(const AttendParams& p, const float*
     float v = -INFINITY;
     if (rr < nr) {
       const int i = (r0 + rr) % p.T_new;
-      if (k < ceil_div(L + i + 1, p.split_tokens))
-        v = __ldcg(p.ws_lse + (row_base + rr) * p.num_splits + k);
+      if (k < row_slices(i)) v = __ldcg(p.ws_lse + (row_base + rr) * p.num_splits + k);
     }
     scratch[idx] = v;
   }
@@ -110,7 +120,7 @@ __device__ __forceinline__ void finish_slice(const AttendParams& p, const float*
     const int d = idx - rr * D;
     if (rr >= nr) break;
     const int i = (r0 + rr) % p.T_new;
-    const int ns_row = ceil_div(L + i + 1, p.split_tokens);
+    const int ns_row = row_slices(i);
     if (ns_row <= 1) continue;
     const float* po = p.ws_o + (row_base + rr) * p.num_splits * D + d;
     const float* w = scratch + rr * nsl;

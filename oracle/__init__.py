@@ -74,6 +74,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_attend.restype = None
     lib.oracle_attend_chunked.argtypes = [I, I, I, I, I, I, P, P, P, I, P, D, I, P, I]
     lib.oracle_attend_chunked.restype = None
+    lib.oracle_attend_window.argtypes = [I, I, I, I, I, I, P, P, P, I, P, D, I, I, P, I]
+    lib.oracle_attend_window.restype = None
     lib.oracle_commit.argtypes = [I, P, P, I, I]
     lib.oracle_commit.restype = I
     lib.oracle_rollback.argtypes = [I, P, P]
@@ -232,6 +234,18 @@ class Oracle:
         out = np.empty((B, H_q, T_new, D), dtype=np.float64)
         self.lib.oracle_attend(B, H_q, H_kv, T_new, D, T_cap, _ptr(q), _ptr(K), _ptr(V),
                                dtype, _ptr(sl), float(scale), _ptr(out), int(nthreads))
+        return out
+
+    def attend_window(self, q, K, V, seq_lens, scale: float, dtype: int, window: int,
+                      sink: int = 0, nthreads: int = 0):
+        """fp64 output of attention over each row's last `window` positions and the
+        first `sink` positions (window 0: all positions)."""
+        q, K, V, sl, B, H_q, H_kv, T_new, D, T_cap = self._check_attend(q, K, V, seq_lens)
+        assert window >= 0 and sink >= 0
+        out = np.empty((B, H_q, T_new, D), dtype=np.float64)
+        self.lib.oracle_attend_window(B, H_q, H_kv, T_new, D, T_cap, _ptr(q), _ptr(K), _ptr(V),
+                                      dtype, _ptr(sl), float(scale), int(window), int(sink),
+                                      _ptr(out), int(nthreads))
         return out
 
     def attend_chunked(self, q, K, V, seq_lens, scale: float, dtype: int, chunk: int,

@@ -330,6 +330,78 @@ void oracle_attend(int B, int H_q, int H_kv, int T_new, int D, int T_cap,
 }
 
 /*
+ * Sliding-window attention with attention sinks ([P2] roadmap: sliding-window
+ * attention keeps each query's last W positions; attention sinks keep the first
+ * S positions as well).  The row with n positions attends position j iff
+ *   j < n  and  (W == 0  or  j >= n - W  or  j < S);
+ * W == 0 is full attention.  Otherwise the naive definition: every score is
+ * materialised, invisible ones are excluded from the max, the sum and the
+ * weighted V sum.
+ */
+static void attend_row_window(int D, int n, int W, int S, const uint16_t* qrow,
+                              const uint16_t* Kbase, const uint16_t* Vbase, int dtype,
+                              double scale, double* orow)
+{
+    double* s = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    char* seen = (char*)malloc((size_t)(n > 0 ? n : 1));
+    double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int d = 0; d < D; ++d)
+        qd[d] = decode(qrow[d], dtype);
+    for (int j = 0; j < n; ++j) {
+        seen[j] = (W == 0 || j >= n - W || j < S);
+        double dot = 0.0;
+        const uint16_t* krow = Kbase + (int64_t)j * D;
+        for (int d = 0; d < D; ++d)
+            dot += qd[d] * decode(krow[d], dtype);
+        s[j] = scale * dot;
+    }
+    double mx = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (seen[j] && s[j] > mx)
+            mx = s[j];
+    double denom = 0.0;
+    for (int j = 0; j < n; ++j) {
+        s[j] = seen[j] ? exp(s[j] - mx) : 0.0;
+        denom += s[j];
+    }
+    for (int d = 0; d < D; ++d)
+        orow[d] = 0.0;
+    for (int j = 0; j < n; ++j) {
+        if (!seen[j])
+            continue;
+        double pj = s[j] / denom;
+        const uint16_t* vrow = Vbase + (int64_t)j * D;
+        for (int d = 0; d < D; ++d)
+            orow[d] += pj * decode(vrow[d], dtype);
+    }
+    free(qd);
+    free(seen);
+    free(s);
+}
+
+void oracle_attend_window(int B, int H_q, int H_kv, int T_new, int D, int T_cap,
+                          const uint16_t* q, const uint16_t* K, const uint16_t* V, int dtype,
+                          const int32_t* seq_lens, double scale, int window, int sink,
+                          double* out, int nthreads)
+{
+    int group = H_q / H_kv;
+    int64_t nrows = (int64_t)B * H_q * T_new;
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int i = (int)(r % T_new);
+        int h = (int)((r / T_new) % H_q);
+        int b = (int)(r / ((int64_t)T_new * H_q));
+        int g = h / group;
+        int n = seq_lens[b] + i + 1;
+        const uint16_t* Kb = K + ((int64_t)b * H_kv + g) * T_cap * D;
+        const uint16_t* Vb = V + ((int64_t)b * H_kv + g) * T_cap * D;
+        attend_row_window(D, n, window, sink, q + r * D, Kb, Vb, dtype, scale, out + r * D);
+    }
+}
+
+/*
  * Chunked attention ([P1]: blocking the computation over the keys only
  * reorders it; the result equals naive attention for any chunk size).
  * Keys are taken `chunk` at a time; a running maximum m, running sum l

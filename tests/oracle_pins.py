@@ -32,7 +32,11 @@ What pins what:
   next token) attends exactly like plain cached decoding of the accepted
   prefix; commit then rollback of the same counts is the identity; out-of-range
   counts change nothing; copy-on-write of a shared, partly filled page leaves
-  every request's logical cache equal to an unshared contiguous cache.
+  every request's logical cache equal to an unshared contiguous cache;
+* sliding window with attention sinks ("项目 9-16" roadmap) -- a window longer
+  than the context is full attention, a window of one gives the row's own value
+  (a sink covering everything gives full attention again), and every row equals
+  plain attention over a contiguous cache holding only its visible positions.
 """
 from __future__ import annotations
 
@@ -454,7 +458,7 @@ def check_copy_on_write(o):
     equals its own unshared contiguous cache, and the skipped pairs change nothing."""
     H_kv, D, P = 2, 8, 4
     prefix = 6                       # pages 0 (full) and 1 (half) shared
-    T_cap = prefix + 1
+    T_cap = prefix + 3               # slack rows: a planted off-by-one stays in bounds
     shared = normal_bits((1, H_kv, prefix, D), "fp16", 31, "cow_prefix")[0]
     new = normal_bits((2, H_kv, 1, D), "fp16", 31, "cow_new")
     num_pages = 5
@@ -474,7 +478,48 @@ def check_copy_on_write(o):
         contig = np.zeros((1, H_kv, T_cap, D), np.uint16)
         contig[0, :, :prefix] = shared
         o.append_contig(contig, np.ascontiguousarray(new[b:b + 1]), L[b:b + 1])
-        assert np.array_equal(logical[b], contig[0]), f"request {b}"
+        assert np.array_equal(logical[b, :, :prefix + 1], contig[0, :, :prefix + 1]), \
+            f"request {b}"
+
+
+def check_window_special_cases(o):
+    B, H_q, H_kv, T_new, D = 2, 4, 2, 3, 32
+    for dtype in (FP16, BF16):
+        q, K, V, L = random_case(B, H_q, H_kv, T_new, D, [37, 5], dtype, seed=131 + dtype)
+        full = o.attend(q, K, V, L, 0.3, dtype, nthreads=2)
+        assert np.array_equal(o.attend_window(q, K, V, L, 0.3, dtype, 10 ** 6, 0), full)
+        assert np.array_equal(o.attend_window(q, K, V, L, 0.3, dtype, 1, 10 ** 6), full)
+        own = o.attend_window(q, K, V, L, 0.3, dtype, 1, 0)
+        Vd = o.decode(V, dtype)
+        for b in range(B):
+            for h in range(H_q):
+                for i in range(T_new):
+                    n = int(L[b]) + i + 1
+                    assert np.array_equal(own[b, h, i], Vd[b, h // (H_q // H_kv), n - 1])
+
+
+def check_window_equals_gathered(o):
+    """Each row's windowed output equals plain attention over a contiguous cache that
+    holds exactly its visible positions (sinks first, then the window), in order."""
+    B, H_q, H_kv, T_new, D = 2, 6, 3, 4, 16
+    cases = [(8, 0), (8, 3), (3, 5), (20, 2), (1, 1)]
+    for dtype in (FP16, BF16):
+        q, K, V, L = random_case(B, H_q, H_kv, T_new, D, [30, 9], dtype, seed=141 + dtype)
+        g = H_q // H_kv
+        for W, S in cases:
+            win = o.attend_window(q, K, V, L, 0.25, dtype, W, S, nthreads=2)
+            for b in range(B):
+                for h in range(H_q):
+                    for i in range(T_new):
+                        n = int(L[b]) + i + 1
+                        keep = [j for j in range(n) if j >= n - W or j < S]
+                        Kg = np.ascontiguousarray(K[b:b + 1, h // g:h // g + 1, keep])
+                        Vg = np.ascontiguousarray(V[b:b + 1, h // g:h // g + 1, keep])
+                        qr = np.ascontiguousarray(q[b:b + 1, h:h + 1, i:i + 1])
+                        ref = o.attend(qr, Kg, Vg, np.array([len(keep) - 1], np.int32), 0.25,
+                                       dtype, nthreads=1)
+                        assert_close(win[b, h, i], ref[0, 0, 0], 1e-15, 1e-13,
+                                     what=f"W={W} S={S} b={b} h={h} i={i}")
 
 
 ALL_CHECKS = [
@@ -494,4 +539,6 @@ ALL_CHECKS = [
     check_speculative_round_equals_plain_decode,
     check_commit_rollback,
     check_copy_on_write,
+    check_window_special_cases,
+    check_window_equals_gathered,
 ]

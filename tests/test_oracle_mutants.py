@@ -57,6 +57,12 @@ MUTANTS = [
      "const uint16_t* from = pool + (int64_t)dst[i] * page_elems;\n        uint16_t* to = pool + (int64_t)src[i] * page_elems;", 0),
     ("copy_pages_half_page", "for (int64_t e = 0; e < page_elems; ++e)",
      "for (int64_t e = 0; e < page_elems / 2; ++e)", 0),
+    ("window_one_short", "seen[j] = (W == 0 || j >= n - W || j < S);",
+     "seen[j] = (W == 0 || j > n - W || j < S);", 0),
+    ("window_drops_sinks", "seen[j] = (W == 0 || j >= n - W || j < S);",
+     "seen[j] = (W == 0 || j >= n - W);", 0),
+    ("window_one_sink_too_many", "seen[j] = (W == 0 || j >= n - W || j < S);",
+     "seen[j] = (W == 0 || j >= n - W || j <= S);", 0),
 ]
 
 
