@@ -69,6 +69,12 @@ typedef enum {
 
 typedef enum { KVC_FP16 = 0, KVC_BF16 = 1 } kvc_dtype;
 
+/* How K and V are stored (kvc_create_quantized). */
+typedef enum {
+    KVC_KV_NATIVE = 0,   /* in the cache's dtype (kvc_create) */
+    KVC_KV_FP8_E4M3 = 1  /* FP8 E4M3 codes plus one fp32 scale per (token, KV head) */
+} kvc_kv_format;
+
 typedef struct kvc_cache kvc_cache;
 
 /*
@@ -84,6 +90,27 @@ typedef struct kvc_cache kvc_cache;
  */
 kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int page_size,
                       int num_layers, int num_pages, kvc_cache** out);
+
+/*
+ * kvc_create_quantized -- kvc_create with K and V stored in `kv_format`.  The pages
+ * leave KV quantisation uncovered ("llm-perf-lab" README; "9. 推理" 9.3 counts the
+ * bytes a decode step reads, which FP8 halves); the format is this library's own:
+ *   KVC_KV_FP8_E4M3: every appended K (and V) row x of D values becomes
+ *       scale = amax / 448       (amax = max_d |x_d|; an all-zero row takes scale 1)
+ *       code_d = E4M3(x_d / scale)   (nearest, ties to even, saturated to +-448)
+ *     with both divisions in fp32, so codes and scales are a function of the row alone.
+ *     Attention then uses code * scale exactly (up to fp32 rounding).  Code pools have
+ *     the layouts of kvc_create with 1-byte elements; scale pools hold one fp32 per row:
+ *     contiguous (B, H_kv, T_pad) with T_pad = max_T rounded up to a multiple of 64,
+ *     paged (num_pages, H_kv, page_size).
+ *     Requires dtype KVC_BF16 (q, k_new, v_new and out stay bf16), D 64 or 128, and
+ *     page_size 0 or at least 8; otherwise KVC_ERR_UNSUPPORTED.
+ * All other calls take the same arguments as for a native cache.  kvc_bytes counts the
+ * codes and the scales.
+ */
+kvc_status kvc_create_quantized(int B, int H_kv, int D, int max_T, kvc_dtype dtype,
+                                kvc_kv_format kv_format, int page_size, int num_layers,
+                                int num_pages, kvc_cache** out);
 
 /* kvc_destroy -- free the pools, workspace and handle (synchronises the device). NULL is ok. */
 kvc_status kvc_destroy(kvc_cache* cache);
@@ -204,6 +231,13 @@ void* kvc_v_pool(kvc_cache* cache, int layer);
 
 /* kvc_layer_pool_bytes -- bytes of one layer's K (equally V) pool. */
 size_t kvc_layer_pool_bytes(const kvc_cache* cache);
+
+/* kvc_k_scales / kvc_v_scales -- device address of a layer's fp32 K / V scale pool of a
+ * quantised cache (NULL for a native cache or a layer out of range); kvc_layer_scale_floats
+ * -- the number of scales in one of them (0 for a native cache). */
+float* kvc_k_scales(kvc_cache* cache, int layer);
+float* kvc_v_scales(kvc_cache* cache, int layer);
+size_t kvc_layer_scale_floats(const kvc_cache* cache);
 
 /*
  * kvc_commit -- advance every request's committed length by its accepted count

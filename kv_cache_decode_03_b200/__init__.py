@@ -69,6 +69,10 @@ def library() -> ctypes.CDLL:
         "kvc_v_pool": ([P, I], P),
         "kvc_layer_pool_bytes": ([P], SZ),
         "kvc_plan_splits": ([P, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I)], I),
+        "kvc_create_quantized": ([I, I, I, I, I, I, I, I, I, ctypes.POINTER(P)], I),
+        "kvc_k_scales": ([P, I], P),
+        "kvc_v_scales": ([P, I], P),
+        "kvc_layer_scale_floats": ([P], SZ),
         "kvc_commit": ([P, P, P, I, P], I),
         "kvc_rollback": ([P, P, P, P], I),
         "kvc_copy_pages": ([P, P, P, I, P], I),
@@ -100,6 +104,19 @@ def kvc_create(B: int, H_kv: int, D: int, max_T: int, dtype, page_size: int = 0,
     h = ctypes.c_void_p()
     _check(library().kvc_create(B, H_kv, D, max_T, code, page_size, num_layers, num_pages,
                                 ctypes.byref(h)), "kvc_create")
+    return int(h.value)
+
+
+KV_FORMATS = {"native": 0, "fp8": 1}
+
+
+def kvc_create_quantized(B: int, H_kv: int, D: int, max_T: int, dtype, kv_format,
+                         page_size: int = 0, num_layers: int = 1, num_pages: int = 0) -> int:
+    code = _DTYPE_CODES[dtype] if isinstance(dtype, str) else int(dtype)
+    fmt = KV_FORMATS[kv_format] if isinstance(kv_format, str) else int(kv_format)
+    h = ctypes.c_void_p()
+    _check(library().kvc_create_quantized(B, H_kv, D, max_T, code, fmt, page_size, num_layers,
+                                          num_pages, ctypes.byref(h)), "kvc_create_quantized")
     return int(h.value)
 
 
@@ -176,6 +193,18 @@ def kvc_layer_pool_bytes(cache: int) -> int:
     return int(library().kvc_layer_pool_bytes(cache))
 
 
+def kvc_k_scales(cache: int, layer: int) -> int:
+    return int(library().kvc_k_scales(cache, layer) or 0)
+
+
+def kvc_v_scales(cache: int, layer: int) -> int:
+    return int(library().kvc_v_scales(cache, layer) or 0)
+
+
+def kvc_layer_scale_floats(cache: int) -> int:
+    return int(library().kvc_layer_scale_floats(cache))
+
+
 def kvc_plan_splits(cache: int, H_q: int, T_new: int, max_pages: int = 0) -> tuple[int, int]:
     ns, st = ctypes.c_int(), ctypes.c_int()
     _check(library().kvc_plan_splits(cache, H_q, T_new, max_pages, ctypes.byref(ns),
@@ -203,11 +232,12 @@ def kvc_copy_pages(cache: int, src: int, dst: int, n: int, stream: int) -> None:
 class _DeviceView:
     """__cuda_array_interface__ over memory the cache owns (keeps the cache alive)."""
 
-    def __init__(self, owner, ptr: int, nbytes: int):
+    def __init__(self, owner, ptr: int, nbytes: int, typestr: str = "<i2"):
         self._owner = owner
+        size = int(typestr[-1])
         self.__cuda_array_interface__ = {
-            "shape": (nbytes // 2,), "typestr": "<i2", "data": (ptr, False), "version": 3,
-            "strides": None,
+            "shape": (nbytes // size,), "typestr": typestr, "data": (ptr, False),
+            "version": 3, "strides": None,
         }
 
 
@@ -215,13 +245,19 @@ class KVCache:
     """A cache handle plus torch-tensor marshalling for append / attend."""
 
     def __init__(self, B: int, H_kv: int, D: int, max_T: int, dtype: str = "bf16",
-                 page_size: int = 0, num_layers: int = 1, num_pages: int = 0):
+                 page_size: int = 0, num_layers: int = 1, num_pages: int = 0,
+                 kv_format: str = "native"):
         import torch
         self.torch_dtype = {"fp16": torch.float16, "bf16": torch.bfloat16}[dtype]
         self.B, self.H_kv, self.D, self.max_T = B, H_kv, D, max_T
         self.dtype, self.page_size, self.num_layers, self.num_pages = (dtype, page_size,
                                                                       num_layers, num_pages)
-        self.handle = kvc_create(B, H_kv, D, max_T, dtype, page_size, num_layers, num_pages)
+        self.kv_format = kv_format
+        if kv_format == "native":
+            self.handle = kvc_create(B, H_kv, D, max_T, dtype, page_size, num_layers, num_pages)
+        else:
+            self.handle = kvc_create_quantized(B, H_kv, D, max_T, dtype, kv_format, page_size,
+                                               num_layers, num_pages)
 
     def close(self) -> None:
         if self.handle:
@@ -239,17 +275,35 @@ class KVCache:
         return kvc_bytes(self.handle)
 
     def pool(self, layer: int, which: str):
-        """A torch view (dtype of the cache) of one layer's K or V pool, in its layout:
-        contiguous (B, H_kv, max_T, D) or paged (num_pages, H_kv, page_size, D)."""
+        """A torch view of one layer's K or V pool, in its layout: contiguous
+        (B, H_kv, max_T, D) or paged (num_pages, H_kv, page_size, D); the cache's dtype,
+        or uint8 E4M3 codes for an FP8 cache."""
         import torch
         ptr = kvc_k_pool(self.handle, layer) if which == "k" else kvc_v_pool(self.handle, layer)
         if not ptr:
             raise IndexError(layer)
         nbytes = kvc_layer_pool_bytes(self.handle)
-        t = torch.as_tensor(_DeviceView(self, ptr, nbytes), device="cuda")
         shape = ((self.num_pages, self.H_kv, self.page_size, self.D) if self.page_size
                  else (self.B, self.H_kv, self.max_T, self.D))
+        if self.kv_format == "fp8":
+            t = torch.as_tensor(_DeviceView(self, ptr, nbytes, "|u1"), device="cuda")
+            return t.view(shape)
+        t = torch.as_tensor(_DeviceView(self, ptr, nbytes), device="cuda")
         return t.view(self.torch_dtype).view(shape)
+
+    def scales(self, layer: int, which: str):
+        """fp32 scales of an FP8 cache: contiguous (B, H_kv, T_pad), paged
+        (num_pages, H_kv, page_size)."""
+        import torch
+        ptr = (kvc_k_scales(self.handle, layer) if which == "k"
+               else kvc_v_scales(self.handle, layer))
+        if not ptr:
+            raise IndexError(layer)
+        n = kvc_layer_scale_floats(self.handle)
+        t = torch.as_tensor(_DeviceView(self, ptr, 4 * n, "<f4"), device="cuda")
+        if self.page_size:
+            return t.view(self.num_pages, self.H_kv, self.page_size)
+        return t.view(self.B, self.H_kv, n // (self.B * self.H_kv))
 
     def _stream(self, stream) -> int:
         import torch

@@ -27,14 +27,22 @@ def nvcc() -> str:
 
 
 def build(verbose: bool = False, out: Path = LIB, extra: list[str] | None = None) -> Path:
+    # compile beside the target and rename over it, so that a process that has the old
+    # library loaded keeps an intact file
+    tmp = out.with_name(f".{out.name}.{os.getpid()}.tmp")
     cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "--expt-relaxed-constexpr",
            "-Xcompiler", "-fPIC", "-shared", f"-I{INCLUDE}", f"-I{CSRC}",
            *(["-Xptxas", "-v"] if verbose else []), *(extra or []),
-           *[str(s) for s in SOURCES], "-o", str(out)]
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libkvc.so")
+           *[str(s) for s in SOURCES], "-o", str(tmp)]
+    try:
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+            raise RuntimeError("nvcc failed building libkvc.so")
+        os.replace(tmp, out)
+    finally:
+        if tmp.exists():
+            tmp.unlink()
     if verbose:
         sys.stderr.write(res.stderr)
     return out

@@ -12,10 +12,12 @@
 
 #include "append.cuh"
 #include "attend_decode.cuh"
+#include "attend_fp8.cuh"
 #include "attend_mma.cuh"
 #include "attend_streamk.cuh"
 #include "attend_tc.cuh"
 #include "cache_ops.cuh"
+#include "fp8.cuh"
 #include "kvc.h"
 
 struct kvc_cache {
@@ -29,6 +31,10 @@ struct kvc_cache {
   size_t ws_bytes;
   int* tickets;        // slice tickets, zero between launches (own allocation, so that
   size_t n_tickets;    // partial layouts of different plans can never overwrite them)
+  bool fp8;                        // FP8 (E4M3) codes + per-(token, head) scales (fp8.cuh)
+  float* scales;                   // fp8: layers x {K, V} x scale_floats
+  size_t scale_floats;             // fp8: scales of one layer's K (equally V)
+  int T_pad;                       // fp8, contiguous: scale row length (whole 64-token tiles)
   bool tma;                        // tensor maps built: the tensor-core path is available
   std::vector<CUtensorMap> tmk;    // per layer: K pool as a 2-D (rows, D) tensor
   std::vector<CUtensorMap> tmv;
@@ -116,8 +122,38 @@ bool make_tmap(CUtensorMap* m, void* base, kvc_dtype dtype, int D, long long row
   return r == CUDA_SUCCESS;
 }
 
+// FP8 code pools: 2-D (rows, D) bytes, one D-byte row per box row, no swizzle.
+bool make_tmap_fp8(CUtensorMap* m, void* base, int D, long long rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D};
+  const cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        KVC_TMA_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 void build_tmaps(kvc_cache* c) {
   c->tma = false;
+  if (c->fp8) {
+    const long long rows = c->paged ? (long long)c->num_pages * c->H_kv * c->page_size
+                                    : (long long)c->B * c->H_kv * c->max_T;
+    if (rows + 64 >= (1LL << 31)) return;
+    const int box_rows = c->paged ? std::min(c->page_size, 64) : 64;
+    c->tmk.resize(c->num_layers);
+    c->tmv.resize(c->num_layers);
+    for (int l = 0; l < c->num_layers; ++l)
+      if (!make_tmap_fp8(&c->tmk[l], c->pool + (size_t)(2 * l) * c->layer_bytes, c->D, rows,
+                         box_rows) ||
+          !make_tmap_fp8(&c->tmv[l], c->pool + (size_t)(2 * l + 1) * c->layer_bytes, c->D, rows,
+                         box_rows))
+        return;
+    c->tma = true;
+    return;
+  }
   if (c->D != 64 && c->D != 128) return;
   if (c->paged && c->page_size < 8) return;  // boxes must start on 1024-byte swizzle atoms
   const long long rows = c->paged ? (long long)c->num_pages * c->H_kv * c->page_size
@@ -225,6 +261,48 @@ int tc_occ(int D, bool paged) {
   return paged ? tc_occupancy<128, T, true>() : tc_occupancy<128, T, false>();
 }
 
+template <int D, int NT, bool PAGED>
+int fp8_occupancy() {
+  static int occ = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const size_t smem = kvc::Fp8Cfg<D>::template smem_bytes<NT>();
+    cudaFuncSetAttribute(kvc::attend_fp8_kernel<D, NT, PAGED>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kvc::attend_fp8_kernel<D, NT, PAGED>, kvc::Fp8Cfg<D>::kThreads, smem) !=
+        cudaSuccess)
+      n = 1;
+    occ = std::max(1, n);
+  });
+  return occ;
+}
+
+template <int D, bool PAGED>
+int fp8_occ_nt(int NT) {
+  switch (NT) {
+    case 1: return fp8_occupancy<D, 1, PAGED>();
+    case 2: return fp8_occupancy<D, 2, PAGED>();
+    default: return fp8_occupancy<D, 4, PAGED>();
+  }
+}
+
+int fp8_occ(int D, int NT, bool paged) {
+  if (D == 64) return paged ? fp8_occ_nt<64, true>(NT) : fp8_occ_nt<64, false>(NT);
+  return paged ? fp8_occ_nt<128, true>(NT) : fp8_occ_nt<128, false>(NT);
+}
+
+int fp8_scratch_floats(int D, int NT) {
+  if (D == 64)
+    return NT == 1 ? kvc::Fp8Cfg<64>::scratch_floats<1>()
+                   : NT == 2 ? kvc::Fp8Cfg<64>::scratch_floats<2>()
+                             : kvc::Fp8Cfg<64>::scratch_floats<4>();
+  return NT == 1 ? kvc::Fp8Cfg<128>::scratch_floats<1>()
+                 : NT == 2 ? kvc::Fp8Cfg<128>::scratch_floats<2>()
+                           : kvc::Fp8Cfg<128>::scratch_floats<4>();
+}
+
 int mma_scratch_floats(int D, int NT) {
   if (D == 64)
     return NT == 1 ? kvc::MmaCfg<64>::scratch_floats<1>()
@@ -237,6 +315,7 @@ int mma_scratch_floats(int D, int NT) {
 
 // ------------------------------------------------------------ attend plan
 struct Plan {
+  bool fp8;          // FP8 cache: attend_fp8_kernel (fixed split, NT 8-row n-tiles)
   bool tc;           // tcgen05 kernel, 128 query rows per CTA
   bool mma;          // mma.sync tensor-core kernel (else the CUDA-core kernel)
   bool streamk;      // mma: persistent stream-K kernel (grid = resident CTAs)
@@ -306,10 +385,17 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
   // Three or more query rows per K/V row make q.k and p.v a dense contraction
   // worth the tensor cores; one or two rows stay on CUDA cores.
   // From KVC_TC_MIN_ROWS rows a 128-row block fills the tcgen05 MMA's M.
-  pl.tc = c->tma && rows >= KVC_TC_MIN_ROWS;
-  pl.mma = c->tma && rows >= 3 && !pl.tc;
+  pl.fp8 = c->fp8;
+  pl.tc = !c->fp8 && c->tma && rows >= KVC_TC_MIN_ROWS;
+  pl.mma = !c->fp8 && c->tma && rows >= 3 && !pl.tc;
   int tile, occ, scratch = 1 << 30;
-  if (pl.tc) {
+  if (pl.fp8) {
+    pl.NT = rows <= 8 ? 1 : (rows <= 16 ? 2 : 4);
+    pl.R = pl.NT * 8;
+    tile = kvc::Fp8Cfg<64>::kTile;
+    occ = fp8_occ(c->D, pl.NT, c->paged);
+    scratch = fp8_scratch_floats(c->D, pl.NT);
+  } else if (pl.tc) {
     pl.NT = 0;
     pl.R = kvc::TcCfg<64>::kRows;
     tile = kvc::TcCfg<64>::kTile;
@@ -521,9 +607,42 @@ kvc_status dispatch_tc(const kvc::AttendParams& p, int D, bool paged, const CUte
                : launch_attend_tc<128, T, false>(p, tk, tv, s);
 }
 
+template <int D, int NT, bool PAGED>
+kvc_status launch_attend_fp8(const kvc::AttendParams& p, const kvc::Fp8Scales& sc,
+                             const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+  using C = kvc::Fp8Cfg<D>;
+  fp8_occupancy<D, NT, PAGED>();  // sets the shared-memory attribute once
+  dim3 grid(p.num_splits * p.row_blocks, p.H_kv, p.B);
+  kvc::attend_fp8_kernel<D, NT, PAGED>
+      <<<grid, C::kThreads, C::template smem_bytes<NT>(), stream>>>(p, sc, tk, tv);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D, bool PAGED>
+kvc_status dispatch_fp8_nt(const kvc::AttendParams& p, const kvc::Fp8Scales& sc, int NT,
+                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  switch (NT) {
+    case 1: return launch_attend_fp8<D, 1, PAGED>(p, sc, tk, tv, s);
+    case 2: return launch_attend_fp8<D, 2, PAGED>(p, sc, tk, tv, s);
+    default: return launch_attend_fp8<D, 4, PAGED>(p, sc, tk, tv, s);
+  }
+}
+
+float* scale_pool(const kvc_cache* c, int layer, int which) {
+  return c->scales + (size_t)(2 * layer + which) * c->scale_floats;
+}
+
 // Launch the attend kernel a plan chose for layer `layer`.
 kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::AttendParams& p,
                     cudaStream_t s) {
+  if (pl.fp8) {
+    const kvc::Fp8Scales sc{scale_pool(c, layer, 0), scale_pool(c, layer, 1), c->T_pad};
+    if (c->D == 64)
+      return c->paged ? dispatch_fp8_nt<64, true>(p, sc, pl.NT, c->tmk[layer], c->tmv[layer], s)
+                      : dispatch_fp8_nt<64, false>(p, sc, pl.NT, c->tmk[layer], c->tmv[layer], s);
+    return c->paged ? dispatch_fp8_nt<128, true>(p, sc, pl.NT, c->tmk[layer], c->tmv[layer], s)
+                    : dispatch_fp8_nt<128, false>(p, sc, pl.NT, c->tmk[layer], c->tmv[layer], s);
+  }
   const bool bf = c->dtype == KVC_BF16;
   if (pl.tc)
     return bf ? dispatch_tc<__nv_bfloat16>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s)
@@ -565,14 +684,20 @@ size_t kvc_bytes_formula(int layers, int kv_heads, int head_dim, long long seq_l
          (size_t)bytes_per_elem * (size_t)batch;
 }
 
-kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int page_size,
-                      int num_layers, int num_pages, kvc_cache** out) {
+static kvc_status create_cache(int B, int H_kv, int D, int max_T, kvc_dtype dtype,
+                               kvc_kv_format kv_format, int page_size, int num_layers,
+                               int num_pages, kvc_cache** out) {
   if (!out) return KVC_ERR_INVALID_ARG;
   *out = nullptr;
   if (B <= 0 || H_kv <= 0 || max_T <= 0 || num_layers <= 0 || page_size < 0 || num_pages < 0)
     return KVC_ERR_INVALID_ARG;
   if (dtype != KVC_FP16 && dtype != KVC_BF16) return KVC_ERR_INVALID_ARG;
+  if (kv_format != KVC_KV_NATIVE && kv_format != KVC_KV_FP8_E4M3) return KVC_ERR_INVALID_ARG;
   if (D != 32 && D != 64 && D != 128) return KVC_ERR_UNSUPPORTED;
+  const bool fp8 = kv_format == KVC_KV_FP8_E4M3;
+  // the FP8 path: bf16 queries, D 64 or 128, pages of 8 or more tokens
+  if (fp8 && (dtype != KVC_BF16 || D == 32 || (page_size > 0 && page_size < 8)))
+    return KVC_ERR_UNSUPPORTED;
   const bool paged = page_size > 0;
   int shift = 0;
   if (paged) {
@@ -591,9 +716,9 @@ kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int pa
     cudaGetLastError();
     return KVC_ERR_CUDA;
   }
-  const size_t layer_bytes =
-      paged ? (size_t)num_pages * H_kv * page_size * D * kEltBytes
-            : (size_t)B * H_kv * max_T * D * kEltBytes;
+  const int elt = fp8 ? 1 : kEltBytes;
+  const size_t layer_bytes = paged ? (size_t)num_pages * H_kv * page_size * D * elt
+                                   : (size_t)B * H_kv * max_T * D * elt;
   kvc_cache* c = new kvc_cache();
   c->B = B;
   c->H_kv = H_kv;
@@ -606,6 +731,11 @@ kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int pa
   c->dtype = dtype;
   c->paged = paged;
   c->layer_bytes = layer_bytes;
+  c->fp8 = fp8;
+  c->T_pad = (max_T + 63) / 64 * 64;
+  c->scale_floats = fp8 ? (paged ? (size_t)num_pages * H_kv * page_size
+                                 : (size_t)B * H_kv * c->T_pad)
+                        : 0;
   c->device = dev;
   c->num_sms = sms;
   void* pool = nullptr;
@@ -623,18 +753,56 @@ kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int pa
     return KVC_ERR_OOM;
   }
   c->d_err = static_cast<int*>(err);
+  if (fp8) {
+    void* sc = nullptr;
+    const size_t sbytes = 2 * c->scale_floats * (size_t)num_layers * sizeof(float);
+    if (cudaMalloc(&sc, sbytes) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(c->pool);
+      cudaFree(c->d_err);
+      delete c;
+      return KVC_ERR_OOM;
+    }
+    c->scales = static_cast<float*>(sc);
+    if (cudaMemset(sc, 0, sbytes) != cudaSuccess) {  // finite scales everywhere
+      cudaGetLastError();
+      cudaFree(c->pool);
+      cudaFree(c->d_err);
+      cudaFree(sc);
+      delete c;
+      return KVC_ERR_CUDA;
+    }
+  }
   if (cudaMemset(c->pool, 0, 2 * layer_bytes * (size_t)num_layers) != cudaSuccess ||
       cudaMemset(c->d_err, 0, sizeof(int)) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     cudaFree(c->pool);
     cudaFree(c->d_err);
+    if (c->scales) cudaFree(c->scales);
     delete c;
     return KVC_ERR_CUDA;
   }
   build_tmaps(c);
+  if (fp8 && !c->tma) {  // the FP8 attend needs its tensor maps
+    kvc_destroy(c);
+    return KVC_ERR_UNSUPPORTED;
+  }
   *out = c;
   return KVC_OK;
+}
+
+kvc_status kvc_create(int B, int H_kv, int D, int max_T, kvc_dtype dtype, int page_size,
+                      int num_layers, int num_pages, kvc_cache** out) {
+  return create_cache(B, H_kv, D, max_T, dtype, KVC_KV_NATIVE, page_size, num_layers, num_pages,
+                      out);
+}
+
+kvc_status kvc_create_quantized(int B, int H_kv, int D, int max_T, kvc_dtype dtype,
+                                kvc_kv_format kv_format, int page_size, int num_layers,
+                                int num_pages, kvc_cache** out) {
+  return create_cache(B, H_kv, D, max_T, dtype, kv_format, page_size, num_layers, num_pages,
+                      out);
 }
 
 kvc_status kvc_destroy(kvc_cache* c) {
@@ -642,6 +810,7 @@ kvc_status kvc_destroy(kvc_cache* c) {
   cudaError_t e = cudaDeviceSynchronize();
   cudaFree(c->pool);
   cudaFree(c->d_err);
+  if (c->scales) cudaFree(c->scales);
   if (c->ws) cudaFree(c->ws);
   if (c->tickets) cudaFree(c->tickets);
   delete c;
@@ -650,6 +819,12 @@ kvc_status kvc_destroy(kvc_cache* c) {
 
 size_t kvc_bytes(const kvc_cache* c) {
   if (!c) return 0;
+  if (c->fp8) {  // one byte a code, plus one fp32 scale a (token, head) for K and for V
+    const long long T = c->paged ? (long long)c->num_pages * c->page_size : c->max_T;
+    const int batch = c->paged ? 1 : c->B;
+    return kvc_bytes_formula(c->num_layers, c->H_kv, c->D, T, 1, batch) +
+           kvc_bytes_formula(c->num_layers, c->H_kv, 1, T, (int)sizeof(float), batch);
+  }
   if (c->paged)
     return kvc_bytes_formula(c->num_layers, c->H_kv, c->D,
                              (long long)c->num_pages * c->page_size, kEltBytes, 1);
@@ -668,6 +843,18 @@ void* kvc_v_pool(kvc_cache* c, int layer) {
   return c->pool + (size_t)(2 * layer + 1) * c->layer_bytes;
 }
 
+float* kvc_k_scales(kvc_cache* c, int layer) {
+  if (!c || !c->fp8 || layer < 0 || layer >= c->num_layers) return nullptr;
+  return scale_pool(c, layer, 0);
+}
+
+float* kvc_v_scales(kvc_cache* c, int layer) {
+  if (!c || !c->fp8 || layer < 0 || layer >= c->num_layers) return nullptr;
+  return scale_pool(c, layer, 1);
+}
+
+size_t kvc_layer_scale_floats(const kvc_cache* c) { return c ? c->scale_floats : 0; }
+
 kvc_status kvc_append(kvc_cache* c, int layer, const void* k_new, const void* v_new, int T_new,
                       const int32_t* block_table, int max_pages, const int32_t* seq_lens,
                       void* stream) {
@@ -678,6 +865,33 @@ kvc_status kvc_append(kvc_cache* c, int layer, const void* k_new, const void* v_
   if (c->paged && (!block_table || !aligned4(block_table) || max_pages <= 0))
     return KVC_ERR_INVALID_ARG;
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c->fp8) {
+    kvc::AppendFp8Params q{};
+    q.k_new = k_new;
+    q.v_new = v_new;
+    q.k_codes = static_cast<uint8_t*>(kvc_k_pool(c, layer));
+    q.v_codes = static_cast<uint8_t*>(kvc_v_pool(c, layer));
+    q.k_scales = scale_pool(c, layer, 0);
+    q.v_scales = scale_pool(c, layer, 1);
+    q.seq_lens = seq_lens;
+    q.block_table = block_table;
+    q.B = c->B;
+    q.H_kv = c->H_kv;
+    q.T_new = T_new;
+    q.D = c->D;
+    q.max_T = c->max_T;
+    q.T_pad = c->T_pad;
+    q.max_pages = max_pages;
+    q.page_shift = c->page_shift;
+    q.num_pages = c->num_pages;
+    q.err = c->d_err;
+    const long long warps = 2LL * c->B * c->H_kv * T_new;
+    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
+    if (c->paged) kvc::append_fp8_kernel<true><<<blocks, 256, 0, st>>>(q);
+    else kvc::append_fp8_kernel<false><<<blocks, 256, 0, st>>>(q);
+    return cuda_status(cudaGetLastError());
+  }
   kvc::AppendParams p{};
   p.k_new = k_new;
   p.v_new = v_new;
@@ -727,12 +941,18 @@ kvc_status kvc_copy_pages(kvc_cache* c, const int32_t* src, const int32_t* dst, 
   if (!c->paged) return KVC_ERR_UNSUPPORTED;
   if (n == 0) return KVC_OK;
   if (2LL * c->num_layers > 65535) return KVC_ERR_UNSUPPORTED;
-  const size_t page_bytes = (size_t)c->H_kv * c->page_size * c->D * kEltBytes;
+  const size_t page_bytes = (size_t)c->H_kv * c->page_size * c->D * (c->fp8 ? 1 : kEltBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid((unsigned)n, (unsigned)(2 * c->num_layers));
   kvc::copy_pages_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<uint4*>(c->pool),
                                                c->layer_bytes / 16, src, dst, n, c->num_layers,
                                                c->num_pages, (int)(page_bytes / 16), c->d_err);
+  if (c->fp8) {  // the pages' scales too: H_kv * page_size floats a page
+    const size_t scale_page_bytes = (size_t)c->H_kv * c->page_size * sizeof(float);
+    kvc::copy_pages_kernel<<<grid, 256, 0, s>>>(
+        reinterpret_cast<uint4*>(c->scales), c->scale_floats * sizeof(float) / 16, src, dst, n,
+        c->num_layers, c->num_pages, (int)(scale_page_bytes / 16), c->d_err);
+  }
   return cuda_status(cudaGetLastError());
 }
 

@@ -27,6 +27,7 @@ Pins (closed forms, library routines, exhaustive checks, page values) live in
 from __future__ import annotations
 
 import ctypes
+import os
 import subprocess
 from pathlib import Path
 
@@ -45,9 +46,17 @@ _lib_path = None
 
 def build(src: Path = SRC, out: Path = LIB, defines: tuple[str, ...] = ()) -> Path:
     """Compile the oracle with gcc (-O2, OpenMP).  Returns the .so path."""
+    # compile beside the target and rename over it: a process that still has the old
+    # library mapped keeps its (unlinked) file intact
+    tmp = Path(out).with_name(f".{Path(out).name}.{os.getpid()}.tmp")
     cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-           "-D_GNU_SOURCE", *[f"-D{d}" for d in defines], str(src), "-o", str(out), "-lm"]
-    subprocess.run(cmd, check=True)
+           "-D_GNU_SOURCE", *[f"-D{d}" for d in defines], str(src), "-o", str(tmp), "-lm"]
+    try:
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    finally:
+        if tmp.exists():
+            tmp.unlink()
     return out
 
 
@@ -76,6 +85,16 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_attend_chunked.restype = None
     lib.oracle_attend_window.argtypes = [I, I, I, I, I, I, P, P, P, I, P, D, I, I, P, I]
     lib.oracle_attend_window.restype = None
+    lib.oracle_decode_e4m3.argtypes = [P, P, I64]
+    lib.oracle_decode_e4m3.restype = None
+    lib.oracle_encode_e4m3.argtypes = [P, P, I64]
+    lib.oracle_encode_e4m3.restype = None
+    lib.oracle_quantize_fp8.argtypes = [P, I64, I, P, P]
+    lib.oracle_quantize_fp8.restype = None
+    lib.oracle_gather_rows.argtypes = [I, I, I, I, I, I, P, P, P, P]
+    lib.oracle_gather_rows.restype = None
+    lib.oracle_attend_fp8.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, D, I, I, P, I]
+    lib.oracle_attend_fp8.restype = None
     lib.oracle_commit.argtypes = [I, P, P, I, I]
     lib.oracle_commit.restype = I
     lib.oracle_rollback.argtypes = [I, P, P]
@@ -173,6 +192,85 @@ class Oracle:
             assert np.all((pages >= 0) & (pages < num_pages))
         self.lib.oracle_append_paged(B, H_kv, T_new, D, P, max_pages, _ptr(new_kv),
                                      _ptr(sl), _ptr(bt), _ptr(pool))
+
+    # -- FP8 (E4M3) cache ------------------------------------------------
+    def decode_e4m3(self, codes) -> np.ndarray:
+        c = np.ascontiguousarray(codes, dtype=np.uint8)
+        out = np.empty(c.shape, dtype=np.float64)
+        self.lib.oracle_decode_e4m3(_ptr(c), _ptr(out), c.size)
+        return out
+
+    def encode_e4m3(self, values) -> np.ndarray:
+        v = np.ascontiguousarray(values, dtype=np.float32)
+        out = np.empty(v.shape, dtype=np.uint8)
+        self.lib.oracle_encode_e4m3(_ptr(v), _ptr(out), v.size)
+        return out
+
+    def quantize_fp8(self, rows) -> tuple[np.ndarray, np.ndarray]:
+        """bf16 words (..., D) -> E4M3 codes (..., D) and fp32 scales (...)."""
+        r = _u16(rows)
+        D = r.shape[-1]
+        n = r.size // D
+        codes = np.empty(r.shape, dtype=np.uint8)
+        scales = np.empty(r.shape[:-1], dtype=np.float32)
+        self.lib.oracle_quantize_fp8(_ptr(r), n, D, _ptr(codes), _ptr(scales))
+        return codes, scales
+
+    def append_fp8(self, codes, scales, new_kv, seq_lens, block_table=None) -> None:
+        """Quantise the new rows (B, H_kv, T_new, D) and write codes and scales into the
+        pool images in place: contiguous codes (B, H_kv, T_cap, D) with scales
+        (B, H_kv, T_pad); paged codes (num_pages, H_kv, P, D) with scales
+        (num_pages, H_kv, P); row L_b + i of (b, g) as for the 16-bit append."""
+        qc, qs = self.quantize_fp8(new_kv)
+        B, H_kv, T_new, _ = qc.shape
+        sl = _i32(seq_lens)
+        for b in range(B):
+            for i in range(T_new):
+                pos = int(sl[b]) + i
+                if block_table is None:
+                    codes[b, :, pos] = qc[b, :, i]
+                    scales[b, :, pos] = qs[b, :, i]
+                else:
+                    P = codes.shape[2]
+                    page = int(block_table[b, pos // P])
+                    codes[page, :, pos % P] = qc[b, :, i]
+                    scales[page, :, pos % P] = qs[b, :, i]
+
+    def gather_rows(self, pool, block_table, n_visible, T_cap: int) -> np.ndarray:
+        """Logical (B, H_kv, T_cap, ...) view of a paged pool (num_pages, H_kv, P, ...) of
+        any element type: the first n_visible[b] positions, the rest zero."""
+        pool = np.ascontiguousarray(pool)
+        num_pages, H_kv, P = pool.shape[:3]
+        row_bytes = int(np.prod(pool.shape[3:], dtype=np.int64)) * pool.itemsize
+        bt = _i32(block_table)
+        nv = _i32(n_visible)
+        B, max_pages = bt.shape
+        assert np.all(nv <= T_cap)
+        out = np.zeros((B, H_kv, T_cap) + pool.shape[3:], dtype=pool.dtype)
+        self.lib.oracle_gather_rows(B, H_kv, row_bytes, P, max_pages, T_cap, _ptr(pool),
+                                    _ptr(bt), _ptr(nv), _ptr(out))
+        return out
+
+    def attend_fp8(self, q, Kc, Ks, Vc, Vs, seq_lens, scale: float, window: int = 0,
+                   sink: int = 0, nthreads: int = 0) -> np.ndarray:
+        """fp64 attention of bf16 queries (B,H_q,T_new,D) over K = Kc * Ks, V = Vc * Vs
+        (codes (B,H_kv,T_cap,D), scales (B,H_kv,T_cap))."""
+        q = _u16(q)
+        Kc = np.ascontiguousarray(Kc, dtype=np.uint8)
+        Vc = np.ascontiguousarray(Vc, dtype=np.uint8)
+        B, H_kv, T_cap, D = Kc.shape
+        Ks = np.ascontiguousarray(Ks[..., :T_cap], dtype=np.float32)
+        Vs = np.ascontiguousarray(Vs[..., :T_cap], dtype=np.float32)
+        _, H_q, T_new, _ = q.shape
+        sl = _i32(seq_lens)
+        assert q.shape == (B, H_q, T_new, D) and Vc.shape == Kc.shape
+        assert Ks.shape == (B, H_kv, T_cap) and Vs.shape == Ks.shape
+        assert np.all(sl + T_new <= T_cap)
+        out = np.empty((B, H_q, T_new, D), dtype=np.float64)
+        self.lib.oracle_attend_fp8(B, H_q, H_kv, T_new, D, T_cap, _ptr(q), _ptr(Kc), _ptr(Ks),
+                                   _ptr(Vc), _ptr(Vs), _ptr(sl), float(scale), int(window),
+                                   int(sink), _ptr(out), int(nthreads))
+        return out
 
     # -- commit / rollback / page copy -----------------------------------
     def commit(self, seq_lens, accepted, T_new: int, max_T: int) -> tuple[np.ndarray, int]:

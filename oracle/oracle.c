@@ -185,6 +185,178 @@ void oracle_append_paged(int B, int H_kv, int T_new, int D, int P, int max_pages
 }
 
 /* ------------------------------------------------------------------ */
+/* FP8 (E4M3) cache.  The pages leave KV quantisation uncovered ([P1];   */
+/* [P3] 9.3 counts the bytes a decode step reads); the format is stated  */
+/* in full here.  E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa */
+/* bits, no infinities, S.1111.111 is NaN, largest finite value 448.     */
+/* A row x of D values is stored as                                      */
+/*   scale = amax / 448 (fp32; amax = max |x_d|; scale 1 if amax == 0)   */
+/*   code_d = E4M3(x_d / scale) (fp32 division; nearest value, ties to   */
+/*            the even code, magnitudes at or above 448 give 448).       */
+/* ------------------------------------------------------------------ */
+
+static double decode_e4m3(uint8_t c)
+{
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 15;
+    int m = c & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9)            /* subnormal: m * 2^-9 */
+                        : ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Nearest finite E4M3 value by search over the 127 non-negative finite codes;
+ * a tie takes the code whose last mantissa bit is 0. */
+static uint8_t encode_e4m3(float xf)
+{
+    double x = (double)xf;
+    if (x != x)
+        return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00; /* -0 keeps its sign */
+    double a = fabs(x);
+    if (a >= 448.0)
+        return (uint8_t)(sign | 0x7E);
+    static double value[0x7F]; /* the non-negative finite codes, decoded once */
+    static int ready = 0;
+    if (!ready) {
+        for (int c = 0; c <= 0x7E; ++c)
+            value[c] = decode_e4m3((uint8_t)c);
+        ready = 1;
+    }
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(value[c] - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    if (best == 0)
+        return 0x00 | sign; /* +0 / -0 */
+    return (uint8_t)(sign | best);
+}
+
+void oracle_decode_e4m3(const uint8_t* src, double* dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = decode_e4m3(src[i]);
+}
+
+void oracle_encode_e4m3(const float* src, uint8_t* dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = encode_e4m3(src[i]);
+}
+
+/* rows (n_rows, D) of bf16 words -> codes (n_rows, D) and scales (n_rows) */
+void oracle_quantize_fp8(const uint16_t* rows, int64_t n_rows, int D, uint8_t* codes,
+                         float* scales)
+{
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint16_t* x = rows + r * D;
+        float amax = 0.0f;
+        for (int d = 0; d < D; ++d) {
+            float v = (float)decode_bf16(x[d]);
+            float av = v < 0 ? -v : v;
+            if (av > amax)
+                amax = av;
+        }
+        float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scales[r] = scale;
+        for (int d = 0; d < D; ++d) {
+            float v = (float)decode_bf16(x[d]);
+            codes[r * D + d] = encode_e4m3(v / scale);
+        }
+    }
+}
+
+/* Logical rows of a paged pool of fixed-size rows (any element type): row pos of
+ * (b, g) is row slot = pos % P of page block_table[b][pos / P]. */
+void oracle_gather_rows(int B, int H_kv, int row_bytes, int P, int max_pages, int T_cap,
+                        const uint8_t* pool, const int32_t* block_table,
+                        const int32_t* n_visible, uint8_t* out)
+{
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < H_kv; ++g)
+            for (int64_t pos = 0; pos < n_visible[b]; ++pos) {
+                int64_t page = block_table[(int64_t)b * max_pages + pos / P];
+                int64_t slot = pos % P;
+                const uint8_t* src = pool + ((page * H_kv + g) * P + slot) * row_bytes;
+                uint8_t* dst = out + (((int64_t)b * H_kv + g) * T_cap + pos) * row_bytes;
+                for (int k = 0; k < row_bytes; ++k)
+                    dst[k] = src[k];
+            }
+}
+
+/* Attention of bf16 queries over FP8 K/V: K[j] = code * scale exactly, in fp64;
+ * the visibility rule of oracle_attend_window (window 0: all positions). */
+static void attend_row_fp8(int D, int n, int W, int S, const uint16_t* qrow,
+                           const uint8_t* Kc, const float* Ks, const uint8_t* Vc,
+                           const float* Vs, double scale, double* orow)
+{
+    double* s = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    char* seen = (char*)malloc((size_t)(n > 0 ? n : 1));
+    double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int d = 0; d < D; ++d)
+        qd[d] = decode_bf16(qrow[d]);
+    for (int j = 0; j < n; ++j) {
+        seen[j] = (W == 0 || j >= n - W || j < S);
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += qd[d] * (decode_e4m3(Kc[(int64_t)j * D + d]) * (double)Ks[j]);
+        s[j] = scale * dot;
+    }
+    double mx = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (seen[j] && s[j] > mx)
+            mx = s[j];
+    double denom = 0.0;
+    for (int j = 0; j < n; ++j) {
+        s[j] = seen[j] ? exp(s[j] - mx) : 0.0;
+        denom += s[j];
+    }
+    for (int d = 0; d < D; ++d)
+        orow[d] = 0.0;
+    for (int j = 0; j < n; ++j) {
+        if (!seen[j])
+            continue;
+        double pj = s[j] / denom;
+        for (int d = 0; d < D; ++d)
+            orow[d] += pj * (decode_e4m3(Vc[(int64_t)j * D + d]) * (double)Vs[j]);
+    }
+    free(qd);
+    free(seen);
+    free(s);
+}
+
+/* q: (B, H_q, T_new, D) bf16 words; Kc, Vc: (B, H_kv, T_cap, D) codes;
+ * Ks, Vs: (B, H_kv, T_cap) scales. */
+void oracle_attend_fp8(int B, int H_q, int H_kv, int T_new, int D, int T_cap,
+                       const uint16_t* q, const uint8_t* Kc, const float* Ks,
+                       const uint8_t* Vc, const float* Vs, const int32_t* seq_lens,
+                       double scale, int window, int sink, double* out, int nthreads)
+{
+    int group = H_q / H_kv;
+    int64_t nrows = (int64_t)B * H_q * T_new;
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int i = (int)(r % T_new);
+        int h = (int)((r / T_new) % H_q);
+        int b = (int)(r / ((int64_t)T_new * H_q));
+        int g = h / group;
+        int n = seq_lens[b] + i + 1;
+        int64_t base = ((int64_t)b * H_kv + g) * T_cap;
+        attend_row_fp8(D, n, window, sink, q + r * D, Kc + base * D, Ks + base, Vc + base * D,
+                       Vs + base, scale, out + r * D);
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Commit, rollback and page copy ([P1]: a two-phase append/commit      */
 /* cache; speculative decoding keeps the accepted prefix of the         */
 /* verified tokens and rolls the rest back; [P3] 9.6: fixed-size pages).*/

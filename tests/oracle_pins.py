@@ -36,7 +36,12 @@ What pins what:
 * sliding window with attention sinks ("项目 9-16" roadmap) -- a window longer
   than the context is full attention, a window of one gives the row's own value
   (a sink covering everything gives full attention again), and every row equals
-  plain attention over a contiguous cache holding only its visible positions.
+  plain attention over a contiguous cache holding only its visible positions;
+* the FP8 (E4M3) cache -- decoding against torch's float8_e4m3fn over all 256
+  codes, encoding against torch's round-to-nearest-even below 448 (plus exact
+  ties between neighbours and saturation above), row quantisation against the
+  format's half-step error bound and its amax -> 448 property, and attention
+  over the dequantised values against torch's fp64 SDPA (causal and windowed).
 """
 from __future__ import annotations
 
@@ -522,6 +527,91 @@ def check_window_equals_gathered(o):
                                      what=f"W={W} S={S} b={b} h={h} i={i}")
 
 
+def bf16_words(x) -> np.ndarray:
+    """float64 values rounded to bf16 (torch, nearest even), as storage words."""
+    t = torch.from_numpy(np.asarray(x, np.float64)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def check_e4m3_decode_exhaustive(o):
+    codes = np.arange(256, dtype=np.uint8)
+    got = o.decode_e4m3(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), np.nonzero(~same)
+
+
+def check_e4m3_encode(o):
+    finite = o.decode_e4m3(np.arange(0x7F, dtype=np.uint8))          # 0 .. 448
+    mids = ((finite[:-1] + finite[1:]) / 2).astype(np.float32)      # exact ties
+    r = np.random.default_rng(7)
+    probe = np.concatenate([mids, -mids, r.standard_normal(20000).astype(np.float32) * 30,
+                            np.float32([0.0, -0.0, 1e-9, 2.0 ** -10, 2.0 ** -9, 447.9,
+                                        -447.9])])
+    got = o.encode_e4m3(probe)
+    ref = torch.from_numpy(probe).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    small = np.abs(probe) < 448
+    assert np.array_equal(got[small], ref[small])
+    # ties go to the even code
+    tie = o.encode_e4m3(mids)
+    assert np.all((tie & 1) == 0)
+    # saturation and NaN
+    big = np.float32([448.0, 460.0, 1e6, -500.0, np.inf])
+    assert np.array_equal(o.encode_e4m3(big), np.uint8([0x7E, 0x7E, 0x7E, 0xFE, 0x7E]))
+    assert o.encode_e4m3(np.float32([np.nan]))[0] & 0x7F == 0x7F
+
+
+def check_quantize_fp8(o):
+    r = np.random.default_rng(11)
+    x = r.standard_normal((64, 128)) * np.exp(r.uniform(-8, 8, size=(64, 1)))
+    x[3] = 0.0                                            # an all-zero row
+    x[5, :] = 1e-30                                       # below bf16's normal range
+    bits = bf16_words(x)
+    codes, scales = o.quantize_fp8(bits)
+    xd = np_decode(bits, BF16)
+    assert scales[3] == 1.0 and not codes[3].any()
+    deq = o.decode_e4m3(codes) * scales[:, None].astype(np.float64)
+    y = np.abs(xd) / scales[:, None]                     # the row in code units
+    half_step = np.where(y >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(y, 1e-300))) - 4),
+                         2.0 ** -10)
+    assert np.all(np.abs(deq - xd) <= half_step * scales[:, None] * (1 + 1e-6) + 1e-300)
+    for i in range(64):
+        if scales[i] != 1.0 or codes[i].any():
+            j = int(np.argmax(np.abs(xd[i])))
+            assert codes[i, j] & 0x7F == 0x7E, i          # amax lands on +-448 ...
+            assert abs(deq[i, j] - xd[i, j]) <= 2.0 ** -22 * abs(xd[i, j]), i  # ... exactly
+
+
+def check_attend_fp8_vs_sdpa(o):
+    B, H_q, H_kv, T_new, D = 2, 4, 2, 3, 32
+    L = np.array([40, 9], np.int32)
+    T_cap = int(L.max()) + T_new
+    r = np.random.default_rng(13)
+    q = bf16_words(r.standard_normal((B, H_q, T_new, D)))
+    Kc = r.integers(0, 256, size=(B, H_kv, T_cap, D)).astype(np.uint8)
+    Vc = r.integers(0, 256, size=(B, H_kv, T_cap, D)).astype(np.uint8)
+    Kc[(Kc & 0x7F) == 0x7F] = 0x01                       # no NaN codes
+    Vc[(Vc & 0x7F) == 0x7F] = 0x02
+    Ks = np.float32(r.uniform(1e-3, 2e-2, size=(B, H_kv, T_cap)))
+    Vs = np.float32(r.uniform(1e-2, 1.0, size=(B, H_kv, T_cap)))
+    to64 = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64)
+    K = (to64(Kc) * torch.from_numpy(Ks.astype(np.float64))[..., None])
+    V = (to64(Vc) * torch.from_numpy(Vs.astype(np.float64))[..., None])
+    qd = torch.from_numpy(np_decode(q, BF16))
+    g = H_q // H_kv
+    for W, S in ((0, 0), (5, 2), (1, 0)):
+        got = o.attend_fp8(q, Kc, Ks, Vc, Vs, L, 0.3, W, S, nthreads=2)
+        for b in range(B):
+            n = np.arange(T_new)[:, None] + int(L[b]) + 1          # visible counts per row
+            j = np.arange(T_cap)[None, :]
+            keep = (j < n) & ((W == 0) | (j >= n - W) | (j < S))
+            mask = torch.from_numpy(np.where(keep, 0.0, -np.inf))
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qd[b:b + 1], K[b:b + 1].repeat_interleave(g, 1), V[b:b + 1].repeat_interleave(g, 1),
+                attn_mask=mask, scale=0.3)
+            assert_close(got[b], ref[0].numpy(), 1e-13, 1e-11, what=f"W={W} S={S} b={b}")
+
+
 ALL_CHECKS = [
     check_decode_fp16_exhaustive,
     check_decode_bf16_exhaustive,
@@ -541,4 +631,8 @@ ALL_CHECKS = [
     check_copy_on_write,
     check_window_special_cases,
     check_window_equals_gathered,
+    check_e4m3_decode_exhaustive,
+    check_e4m3_encode,
+    check_quantize_fp8,
+    check_attend_fp8_vs_sdpa,
 ]

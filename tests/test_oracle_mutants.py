@@ -63,6 +63,12 @@ MUTANTS = [
      "seen[j] = (W == 0 || j >= n - W);", 0),
     ("window_one_sink_too_many", "seen[j] = (W == 0 || j >= n - W || j < S);",
      "seen[j] = (W == 0 || j >= n - W || j <= S);", 0),
+    ("e4m3_exponent_bias", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 11)", 0),
+    ("e4m3_subnormal_scale", "ldexp((double)m, -9)", "ldexp((double)m, -10)", 0),
+    ("e4m3_ties_to_odd", "(c & 1) == 0 && (best & 1) == 1", "(c & 1) == 1 && (best & 1) == 0", 0),
+    ("fp8_scale_447", "amax / 448.0f", "amax / 447.0f", 0),
+    ("fp8_attend_drops_v_scale", "* (double)Vs[j])", "* 1.0)", 0),
+    ("fp8_attend_k_scale_from_v", "(double)Ks[j])", "(double)Vs[j])", 0),
 ]
 
 
