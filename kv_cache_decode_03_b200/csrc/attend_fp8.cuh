@@ -1,24 +1,32 @@
 // attend_fp8.cuh -- N2 for the FP8 cache (fp8.cuh): split-K attention whose K/V tiles
 // arrive as E4M3 codes with one fp32 scale per (token, KV head).
 //
-// Same contract and structure as attend_mma.cuh (tensor cores, mma.m16n8k16 with the
-// K/V tokens as M and the query rows as N, fixed split-K, the shared slice epilogue,
-// windows through window.cuh); what differs is the data path:
-//   - thread 0 loads each 64-token tile's codes with 2-D TMA (one D-byte row per token,
-//     no swizzle, no multicast) and the tile's K and V scales with 1-D bulk copies;
-//   - each warp converts its own 16 tokens of codes to bf16 (exact: E4M3 has 3
-//     mantissa bits) into a 128-byte-swizzled buffer, releases the stage at once, and
-//     runs the bf16 MMAs from the buffer;
-//   - the K scale multiplies the token's score, the V scale the token's softmax
-//     weight in the p.V product (never the running sum l), so the result is attention
-//     over code * scale exactly, up to fp32 rounding.
-// bf16 q/out only; weights are split hi + lo like every bf16 tensor-core path.
+// Same contract and structure as attend_mma.cuh (mma.m16n8k16 with the K/V tokens as M
+// and the query rows as N, fixed split-K, the shared slice epilogue, windows through
+// window.cuh).  The codes never pass through shared memory as wider values:
+//   - thread 0 loads each 64-token tile's codes with 2-D TMA (one D-byte row a token,
+//     128-byte swizzle for D = 128, 64-byte for D = 64, no multicast) and the tile's K
+//     and V scales with 1-D bulk copies;
+//   - K: ldmatrix reads 16-byte code chunks; each 32-bit fragment register holds codes
+//     4c..4c+3 of a row, which two cvt.f16x2.e4m3x2 turn into the f16 A-fragment
+//     halves for k = 2c, 2c+1 and k = 8+2c, 9+2c -- a fixed permutation of the k index
+//     that the Q fragments (built once) follow, so q.k is unchanged;
+//   - V: the same loads and conversions, then movmatrix.trans of each 8x8 f16 block
+//     gives V^T fragments whose 16 D-rows come in a fixed permuted order (codes
+//     0,1,4,5,8,9,12,13 then 2,3,6,7,10,11,14,15 of each chunk), undone when the
+//     accumulators are written out;
+//   - the MMAs run in f16 (E4M3 converts to f16 exactly).  Each query row is scaled by a
+//     power of two into f16 range (exact; folded back into the score).  The K scale
+//     multiplies the token's score; the V scale enters the p.V weight through a second
+//     running maximum over s + log2(v_scale), so the f16 weights stay <= 1, while the
+//     sum l keeps its own maximum; out = O * 2^(mo - m) / l is attention over
+//     code * scale exactly, up to fp32 rounding and the 11-bit f16 weights.
+// bf16 q/out only.
 #pragma once
 
 #include <cuda.h>
 #include <math.h>
 
-#include "attend_mma.cuh"
 #include "device_common.cuh"
 #include "fp8.cuh"
 #include "params.cuh"
@@ -29,22 +37,21 @@ namespace kvc {
 
 template <int D>
 struct Fp8Cfg {
+  static_assert(D == 64 || D == 128, "FP8 attend: D must be 64 or 128");
   static constexpr int kWarps = 4;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kTile = 64;                 // tokens per stage, 16 per warp
   static constexpr int kCodeBytes = kTile * D;     // K (or V) codes per stage
+  static constexpr int kChunks = D / 16;           // 16-code chunks in a row
   static constexpr int kStages = 4;
   static constexpr int kRing = 2 * kStages * kCodeBytes;
-  static constexpr int kScaleBytes = 2 * kTile * 4;                   // K and V scales
-  static constexpr int kConvBytes = MmaCfg<D>::kTileBytes;             // one bf16 tile
-  static constexpr int kData = kRing + kStages * kScaleBytes + 2 * kConvBytes;
-  static constexpr int kKSteps = D / 16;
-  static constexpr int kMTiles = D / 16;
+  static constexpr int kScaleBytes = 2 * kTile * 4;  // K and V scales of a tile
+  static constexpr int kData = kRing + kStages * kScaleBytes;
 
   template <int NT>
   static constexpr size_t smem_bytes() {
-    return 1024 + kData + kWarps * NT * 8 * 2 * sizeof(float) + 2 * kStages * sizeof(uint64_t) +
-           16;
+    return 1024 + kData + kWarps * NT * 8 * 2 * sizeof(float) + NT * 8 * sizeof(int) +
+           2 * kStages * sizeof(uint64_t) + 16;
   }
   template <int NT>
   static constexpr int scratch_floats() {
@@ -52,6 +59,32 @@ struct Fp8Cfg {
   }
   static_assert(kRing >= kWarps * 32 * D * 4, "the result buffer must fit the rings");
 };
+
+// Byte offset of 16-byte chunk `chunk` of code row `row` in a swizzled tile: TMA's
+// 128-byte swizzle (D = 128: one row is one 128-byte line) or 64-byte swizzle (D = 64).
+template <int D>
+__device__ __forceinline__ uint32_t swz8(int row, int chunk) {
+  if constexpr (D == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
+  else return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two_codes));
+  return h2;
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Row of chunk `chunk`'s 16 d-values that V^T row rho (0..15) of an m-tile holds.
+__device__ __forceinline__ int vt_row_to_d(int rho) {
+  const int j = rho & 7;
+  return 4 * (j >> 1) + (j & 1) + (rho >= 8 ? 2 : 0);
+}
 
 struct Fp8Scales {
   const float* k;  // contiguous (B, H_kv, T_pad); paged (num_pages, H_kv, P)
@@ -70,17 +103,17 @@ __global__ void __launch_bounds__(Fp8Cfg<D>::kThreads)
   constexpr int NTH = C::kThreads;
   constexpr int R = NT * 8;  // query rows per CTA (padded)
   constexpr int S = C::kStages;
+  constexpr int KC = C::kChunks;
   extern __shared__ unsigned char fp8_smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(fp8_smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* ck = smem;                          // K code stages
-  unsigned char* cv = smem + S * C::kCodeBytes;      // V code stages
+  unsigned char* ck = smem;                               // K code stages
+  unsigned char* cv = smem + S * C::kCodeBytes;           // V code stages
   float* scl = reinterpret_cast<float*>(smem + C::kRing);  // [S][K 64 | V 64]
-  unsigned char* bk = smem + C::kRing + S * C::kScaleBytes;  // bf16 K tile (swizzled)
-  unsigned char* bv = bk + C::kConvBytes;                    // bf16 V tile
   float* red_m = reinterpret_cast<float*>(smem + C::kData);
   float* red_l = red_m + W * R;
-  uint64_t* full = reinterpret_cast<uint64_t*>(red_l + W * R);
+  int* qexp = reinterpret_cast<int*>(red_l + W * R);      // [R] query-row exponents
+  uint64_t* full = reinterpret_cast<uint64_t*>(qexp + R);
   uint64_t* empty = full + S;
   int* flags = reinterpret_cast<int*>(empty + S);  // [0] abort, [1] last
   float* red_acc = reinterpret_cast<float*>(smem);  // code rings, after the loop
@@ -127,7 +160,50 @@ __global__ void __launch_bounds__(Fp8Cfg<D>::kThreads)
     flags[1] = 0;
     fence_barrier_init();
   }
-  __syncthreads();
+
+  // ------------------------------------------------------------- query rows
+  // Q^T fragments (B operand, f16), row n = nt*8 + lane/4, under the k permutation of
+  // the K fragments: k = 2c, 2c+1 <-> d = 16kk + 4c, +1; k = 8+2c, 9+2c <-> d = 16kk+4c+2, +3
+  // (c = lane % 4).  Row n is first scaled by 2^-e_n, e_n putting its largest |q| in
+  // [2^14, 2^15) (exact; e_n is folded back into the row's scores).
+  uint32_t qb[KC][NT][2];
+  {
+    const __nv_bfloat16* qblk = static_cast<const __nv_bfloat16*>(p.q) +
+                                ((((size_t)b * p.H_q + (size_t)g * p.group) * p.T_new) + r0) * D;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int row = nt * 8 + (lane >> 2);
+      float qv[KC][4];
+      float amax = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KC; ++kk) {
+        uint2 w = make_uint2(0u, 0u);
+        if (row < nr)
+          w = __ldg(reinterpret_cast<const uint2*>(qblk + (size_t)row * D + kk * 16 +
+                                                   (lane & 3) * 4));
+        qv[kk][0] = __uint_as_float(w.x << 16);
+        qv[kk][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        qv[kk][2] = __uint_as_float(w.y << 16);
+        qv[kk][3] = __uint_as_float(w.y & 0xFFFF0000u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[kk][e]));
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // e = exponent of amax - 14 (0 for a zero row), at least -126 so that 2^-e and 2^e
+      // are normal floats built by exponent arithmetic
+      const int e =
+          amax > 0.f ? max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14, -126) : 0;
+      const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+      for (int kk = 0; kk < KC; ++kk) {
+        qb[kk][nt][0] = f32x2_to_f16x2(qv[kk][0] * inv, qv[kk][1] * inv);
+        qb[kk][nt][1] = f32x2_to_f16x2(qv[kk][2] * inv, qv[kk][3] * inv);
+      }
+      if (warp == 0 && (lane & 3) == 0) qexp[row] = e;
+    }
+  }
+  __syncthreads();  // barriers initialised, row exponents published
 
   // ------------------------------------------------------- tile producer
   const bool producer = (threadIdx.x == 0);
@@ -180,58 +256,38 @@ __global__ void __launch_bounds__(Fp8Cfg<D>::kThreads)
     for (; issued < min(S, ntiles); ++issued) issue(issued);
 
   // ------------------------------------------------------------- consumers
-  // Q^T fragments (B operand of q.k): row n = nt*8 + lane/4, d = kk*16 + 2(lane%4) (+8)
-  uint32_t qb[C::kKSteps][NT][2];
-  {
-    const char* qblk =
-        static_cast<const char*>(p.q) + ((((size_t)b * p.H_q + (size_t)g * p.group) * p.T_new) +
-                                         r0) * D * 2;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int row = nt * 8 + (lane >> 2);
-#pragma unroll
-      for (int kk = 0; kk < C::kKSteps; ++kk) {
-        if (row < nr) {
-          const char* src = qblk + (size_t)row * D * 2 + (kk * 16 + (lane & 3) * 2) * 2;
-          qb[kk][nt][0] = __ldg(reinterpret_cast<const unsigned int*>(src));
-          qb[kk][nt][1] = __ldg(reinterpret_cast<const unsigned int*>(src + 16));
-        } else {
-          qb[kk][nt][0] = 0u;
-          qb[kk][nt][1] = 0u;
-        }
-      }
-    }
-  }
-  int vis[NT][2];  // this thread's score columns: rows nt*8 + 2(lane%4) + c
+  int vis[NT][2];    // this thread's score columns: rows nt*8 + 2(lane%4) + c
+  float fcol[NT][2];  // their score factors: scale * log2(e) * 2^e_row
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int rr = nt * 8 + (lane & 3) * 2 + c;
       vis[nt][c] = rr < nr ? L + (r0 + rr) % p.T_new + 1 : 0;
+      fcol[nt][c] = p.scale_log2 * __uint_as_float((uint32_t)(127 + qexp[rr]) << 23);
     }
 
-  float m[NT][2], l[NT][2];
-  float o[C::kMTiles][NT][4];
+  // per column: m / l for the softmax sum, mo for the weights of O (s + log2 v_scale)
+  float m[NT][2], l[NT][2], mo[NT][2];
+  float o[KC][NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     m[nt][0] = m[nt][1] = -INFINITY;
+    mo[nt][0] = mo[nt][1] = -INFINITY;
     l[nt][0] = l[nt][1] = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < C::kMTiles; ++mt)
+    for (int mt = 0; mt < KC; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
   }
 
-  const int mi = lane >> 3;
+  // ldmatrix row addresses: matrices (tokens 0-7 | 8-15) x (chunk j | j+1) of this warp
   const int wrow = warp * 16;
-  const int k_row = wrow + (mi & 1) * 8 + (lane & 7);
-  const int k_cs = mi >> 1;
-  const int v_row = wrow + (mi >> 1) * 8 + (lane & 7);
-  const int v_cs = mi & 1;
-  const uint32_t kb = smem_addr(bk);
-  const uint32_t vb = smem_addr(bv);
-  constexpr int kChunks = 16 * D / 16;  // 16-code chunks in this warp's 16 rows
+  const int mi = lane >> 3;
+  const int ld_row = wrow + (mi & 1) * 8 + (lane & 7);
+  const int ld_cs = mi >> 1;
+  const uint32_t ck_addr = smem_addr(ck);
+  const uint32_t cv_addr = smem_addr(cv);
 
   bool ok = true;
   int consumed = 0;
@@ -251,112 +307,110 @@ __global__ void __launch_bounds__(Fp8Cfg<D>::kThreads)
       break;
     }
     consumed = j + 1;
+    const uint32_t kb = ck_addr + st * C::kCodeBytes;
+    const uint32_t vb = cv_addr + st * C::kCodeBytes;
     const int t0 = sp.real(t_begin + j * C::kTile);
-
-    // this warp's 16 tokens: codes -> bf16 (swizzled), scales -> registers
-    {
-      const unsigned char* srck = ck + st * C::kCodeBytes + wrow * D;
-      const unsigned char* srcv = cv + st * C::kCodeBytes + wrow * D;
-#pragma unroll
-      for (int c = lane; c < kChunks; c += 32) {
-        const int row = wrow + c / (D / 16);
-        const int col = c % (D / 16);  // 16 codes = two 16-byte bf16 chunks
-        uint4 lo, hi;
-        e4m3x16_to_bf16(ld_shared_v4(srck + c * 16), lo, hi);
-        st_shared_v4(bk + swz<D>(row, 2 * col), lo);
-        st_shared_v4(bk + swz<D>(row, 2 * col + 1), hi);
-        e4m3x16_to_bf16(ld_shared_v4(srcv + c * 16), lo, hi);
-        st_shared_v4(bv + swz<D>(row, 2 * col), lo);
-        st_shared_v4(bv + swz<D>(row, 2 * col + 1), hi);
-      }
-    }
     const float* ssc = scl + st * (2 * C::kTile);
     const int ta = wrow + (lane >> 2);  // this thread's two tokens: ta and ta + 8
     const float ska = ssc[ta], skb = ssc[ta + 8];
-    const float sva = ssc[C::kTile + ta], svb = ssc[C::kTile + ta + 8];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);  // the codes are consumed: refill early
+    const float lva = __log2f(ssc[C::kTile + ta]), lvb = __log2f(ssc[C::kTile + ta + 8]);
 
-    // S^T = K . Q^T for this warp's 16 tokens
+    // S^T = K . Q^T for this warp's 16 tokens, K converted in registers
     float sacc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < C::kKSteps; ++kk) {
-      uint32_t a[4];
-      ldmatrix_x4(a, kb + swz<D>(k_row, 2 * kk + k_cs));
+    for (int kp = 0; kp < KC; kp += 2) {
+      uint32_t r[4];
+      ldmatrix_x4(r, kb + swz8<D>(ld_row, kp + ld_cs));
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816<T>(sacc[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+      for (int h = 0; h < 2; ++h) {  // chunk kp + h: registers r[2h] (tokens 0-7), r[2h+1]
+        const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * h]), e4m3x2_to_f16x2(r[2 * h + 1]),
+                               e4m3x2_to_f16x2(r[2 * h] >> 16),
+                               e4m3x2_to_f16x2(r[2 * h + 1] >> 16)};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816<__half>(sacc[nt], a, qb[kp + h][nt][0], qb[kp + h][nt][1]);
+      }
     }
 
-    // K scales and base-2 units, mask, online softmax per score column (query row)
+    // scores (base 2), mask, two running maxima per score column (query row)
     const int tok0 = t0 + ta;
     const bool unmasked = tile_fully_visible(t0, C::kTile, vis_min, n_blk, p.window, p.sink);
-    const float fa = p.scale_log2 * ska, fb = p.scale_log2 * skb;
     bool grew = false;
-    float alpha[NT][2];
+    float alpha_o[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        float s0 = sacc[nt][c] * fa;
-        float s1 = sacc[nt][2 + c] * fb;
+        float s0 = sacc[nt][c] * fcol[nt][c] * ska;
+        float s1 = sacc[nt][2 + c] * fcol[nt][c] * skb;
         if (!unmasked) {
           s0 = visible(tok0, vis[nt][c], p.window, p.sink) ? s0 : -INFINITY;
           s1 = visible(tok0 + 8, vis[nt][c], p.window, p.sink) ? s1 : -INFINITY;
         }
+        // the sum l, referenced to m
         float mx = fmaxf(s0, s1);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m[nt][c], mx);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[nt][c] = exp2f(m[nt][c] - mu);
-        grew |= (m_new > m[nt][c]);
+        l[nt][c] = fmaf(l[nt][c], exp2f(m[nt][c] - mu), exp2f(s0 - mu) + exp2f(s1 - mu));
         m[nt][c] = m_new;
-        const float p0 = exp2f(s0 - mu);
-        const float p1 = exp2f(s1 - mu);
-        l[nt][c] = fmaf(l[nt][c], alpha[nt][c], p0 + p1);
-        sacc[nt][c] = p0 * sva;  // the V scale enters the weight, not the sum
-        sacc[nt][2 + c] = p1 * svb;
+        // the weights of O, referenced to mo: 2^(s + log2 v_scale - mo) <= 1
+        const float w0 = s0 + lva, w1 = s1 + lvb;
+        float mxo = fmaxf(w0, w1);
+        mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 4));
+        mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 8));
+        mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 16));
+        const float mo_new = fmaxf(mo[nt][c], mxo);
+        const float muo = (mo_new == -INFINITY) ? 0.f : mo_new;
+        alpha_o[nt][c] = exp2f(mo[nt][c] - muo);
+        grew |= (mo_new > mo[nt][c]);
+        mo[nt][c] = mo_new;
+        sacc[nt][c] = exp2f(w0 - muo);
+        sacc[nt][2 + c] = exp2f(w1 - muo);
       }
     }
     if (__any_sync(0xffffffffu, grew)) {
 #pragma unroll
-      for (int mt = 0; mt < C::kMTiles; ++mt)
+      for (int mt = 0; mt < KC; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          o[mt][nt][0] *= alpha[nt][0];
-          o[mt][nt][1] *= alpha[nt][1];
-          o[mt][nt][2] *= alpha[nt][0];
-          o[mt][nt][3] *= alpha[nt][1];
+          o[mt][nt][0] *= alpha_o[nt][0];
+          o[mt][nt][1] *= alpha_o[nt][1];
+          o[mt][nt][2] *= alpha_o[nt][0];
+          o[mt][nt][3] *= alpha_o[nt][1];
         }
     }
-    // P^T fragments (bf16 hi and lo): transpose each 8x8 (token x row) block
-    uint32_t pb[NT][2], pl[NT][2];
+    // P^T fragments (f16): transpose each 8x8 (token x row) block
+    uint32_t pb[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t h0 = Elt<T>::pack2(sacc[nt][0], sacc[nt][1]);
-      const uint32_t h1 = Elt<T>::pack2(sacc[nt][2], sacc[nt][3]);
-      pb[nt][0] = movmatrix_trans(h0);
-      pb[nt][1] = movmatrix_trans(h1);
-      pl[nt][0] = movmatrix_trans(bf16_remainder2(sacc[nt][0], sacc[nt][1], h0));
-      pl[nt][1] = movmatrix_trans(bf16_remainder2(sacc[nt][2], sacc[nt][3], h1));
+      pb[nt][0] = movmatrix_trans(f32x2_to_f16x2(sacc[nt][0], sacc[nt][1]));
+      pb[nt][1] = movmatrix_trans(f32x2_to_f16x2(sacc[nt][2], sacc[nt][3]));
     }
-    // O^T += V^T . P^T
+    // O^T += V^T . P^T, V^T from the codes: convert, then transpose each 8x8 block
 #pragma unroll
-    for (int mt = 0; mt < C::kMTiles; ++mt) {
-      uint32_t a[4];
-      ldmatrix_x4_trans(a, vb + swz<D>(v_row, 2 * mt + v_cs));
+    for (int kp = 0; kp < KC; kp += 2) {
+      uint32_t r[4];
+      ldmatrix_x4(r, vb + swz8<D>(ld_row, kp + ld_cs));
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
-        mma_16816<T>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+      for (int h = 0; h < 2; ++h) {  // m-tile kp + h: d rows of chunk kp + h
+        const uint32_t a[4] = {movmatrix_trans(e4m3x2_to_f16x2(r[2 * h])),
+                               movmatrix_trans(e4m3x2_to_f16x2(r[2 * h] >> 16)),
+                               movmatrix_trans(e4m3x2_to_f16x2(r[2 * h + 1])),
+                               movmatrix_trans(e4m3x2_to_f16x2(r[2 * h + 1] >> 16))};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816<__half>(o[kp + h][nt], a, pb[nt][0], pb[nt][1]);
       }
     }
-    __syncwarp();  // this warp's bf16 rows are rewritten by its next tile
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
   }
   if (!ok) {
     atomicOr(&flags[0], 1);
@@ -377,15 +431,23 @@ __global__ void __launch_bounds__(Fp8Cfg<D>::kThreads)
     }
   named_barrier_sync(1, NTH);  // the rings are free
   if (flags[0]) return;
+  // O referenced to m: O * 2^(mo - m); V^T row rho of m-tile mt is d = 16 mt + vt_row_to_d(rho)
+  float f[NT][2];
 #pragma unroll
-  for (int mt = 0; mt < C::kMTiles; ++mt)
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      f[nt][c] = (m[nt][c] == -INFINITY || mo[nt][c] == -INFINITY) ? 0.f
+                                                                  : exp2f(mo[nt][c] - m[nt][c]);
+#pragma unroll
+  for (int mt = 0; mt < KC; ++mt)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int row = nt * 8 + (lane & 3) * 2 + (e & 1);
-        const int d = mt * 16 + (lane >> 2) + (e >> 1) * 8;
-        red_acc[(warp * R + row) * D + d] = o[mt][nt][e];
+        const int d = mt * 16 + vt_row_to_d((lane >> 2) + (e >> 1) * 8);
+        red_acc[(warp * R + row) * D + d] = o[mt][nt][e] * f[nt][e & 1];
       }
   if (lane < 4) {
 #pragma unroll

@@ -62,6 +62,9 @@ constexpr int kEltBytes = 2;
 #ifndef KVC_SPLIT_WAVES
 #define KVC_SPLIT_WAVES 4
 #endif
+#ifndef KVC_FP8_SPLIT_WAVES  // the FP8 kernel's tiles are cheaper to load: fewer, longer slices
+#define KVC_FP8_SPLIT_WAVES 4
+#endif
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -122,7 +125,9 @@ bool make_tmap(CUtensorMap* m, void* base, kvc_dtype dtype, int D, long long row
   return r == CUDA_SUCCESS;
 }
 
-// FP8 code pools: 2-D (rows, D) bytes, one D-byte row per box row, no swizzle.
+// FP8 code pools: 2-D (rows, D) bytes, one D-byte row per box row, swizzled across the
+// row's 16-byte chunks (128-byte swizzle for D = 128, 64-byte for D = 64) so that the
+// kernel's ldmatrix reads are conflict-free.
 bool make_tmap_fp8(CUtensorMap* m, void* base, int D, long long rows, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -131,7 +136,8 @@ bool make_tmap_fp8(CUtensorMap* m, void* base, int D, long long rows, int box_ro
   const cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1u, 1u};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                         KVC_TMA_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -440,7 +446,8 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
                                        tile);
   cap = std::max<long long>(cap, 1);
   const long long units = (long long)c->B * c->H_kv * pl.row_blocks;
-  const long long target = (long long)KVC_SPLIT_WAVES * c->num_sms * occ;
+  const long long target =
+      (long long)(pl.fp8 ? KVC_FP8_SPLIT_WAVES : KVC_SPLIT_WAVES) * c->num_sms * occ;
   // the merging CTA keeps one weight per (row, slice) in shared memory
   const long long max_ns = std::min<long long>((cap + tile - 1) / tile, scratch / pl.R);
   long long ns = std::min(std::max((target + units - 1) / units, 1LL), max_ns);
