@@ -46,6 +46,14 @@ METRIC = ("decode-attention KV HBM GB/s (% of B200 peak) and tokens/s per layer-
 KERNEL_SOURCES = {
     "attend_streamk_kernel": ("attend_streamk.cuh", "splitk_epilogue.cuh", "device_common.cuh",
                               "params.cuh"),
+    "attend_mma_kernel": ("attend_mma.cuh", "splitk_epilogue.cuh", "window.cuh",
+                          "device_common.cuh", "params.cuh"),
+    "attend_tc_kernel": ("attend_tc.cuh", "splitk_epilogue.cuh", "window.cuh",
+                         "device_common.cuh", "params.cuh"),
+    "attend_fp8_kernel": ("attend_fp8.cuh", "fp8.cuh", "splitk_epilogue.cuh", "window.cuh",
+                          "device_common.cuh", "params.cuh"),
+    "attend_decode_kernel": ("attend_decode.cuh", "splitk_epilogue.cuh", "window.cuh",
+                             "device_common.cuh", "params.cuh"),
 }
 
 
@@ -61,6 +69,8 @@ def kernel_source_sha256(kernel: str = "attend_streamk_kernel") -> str:
 
 def profiled_traffic(kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if its sources still match."""
+    if kernel.split("<")[0] not in KERNEL_SOURCES:
+        return None
     sha = kernel_source_sha256(kernel.split("<")[0])
     for f in sorted((ROOT / "profiles").glob("*.md")):
         kv = {}
@@ -79,6 +89,43 @@ def peaks():
         d = json.loads(p.read_text())
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a kernel timed on its own)."""
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        return float(json.loads(p.read_text())["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+L2_BYTES = 126e6
+
+
+def fp8_algorithmic_bytes(c: W.Case) -> int:
+    """Per layer-step on an FP8 cache: codes (1 B) and a K and a V scale (4 B) per
+    (token, KV head) read; q in and out in the 16-bit type; the new rows read in the
+    16-bit type and written as codes and scales."""
+    tokens = c.kv_read_bytes(True) // (2 * c.H_kv * c.D * c.elt)
+    kv = tokens * 2 * c.H_kv * (c.D + 4)
+    qo = 2 * c.B * c.H_q * c.T_new * c.D * c.elt
+    app = c.B * c.H_kv * c.T_new * 2 * (c.D * c.elt + c.D + 4)
+    return kv + qo + app
+
+
+def attend_kernel_name(c: W.Case, kv_format: str, split_tokens: int) -> str:
+    rows = (c.H_q // c.H_kv) * c.T_new
+    layout = "paged" if c.paged else "contiguous"
+    if kv_format == "fp8":
+        return f"attend_fp8_kernel<{c.D},{layout}>"
+    if rows >= 64 and c.D in (64, 128):
+        return f"attend_tc_kernel<{c.D},{c.dtype},{layout}>"
+    if split_tokens == 0:
+        nt = 1 if rows <= 8 else 2
+        return f"attend_streamk_kernel<{c.D},{nt},{c.dtype},{layout}>"
+    if rows >= 3 and c.D in (64, 128):
+        return f"attend_mma_kernel<{c.D},{c.dtype},{layout}>"
+    return f"attend_decode_kernel<{c.D},{c.dtype},{layout}>"
 
 
 # ---------------------------------------------------------------------------
@@ -179,9 +226,16 @@ def time_oracle(case: W.Case, requests: list[int], layers: list[int]) -> tuple[f
     return total, nbytes
 
 
-def cpu_baseline(case: W.Case, budget_s: float = 12.0) -> dict:
+def cpu_baseline(case: W.Case, budget_s: float = 12.0, max_elems: float = 6.4e7) -> dict:
     import oracle
-    reqs = list(range(case.B))
+    # requests in order while their K/V stays within max_elems host elements (one at least)
+    reqs, elems = [], 0
+    for b in range(case.B):
+        e = (int(case.seq_lens[b]) + case.T_new) * case.H_kv * case.D
+        if reqs and elems + e > max_elems:
+            break
+        reqs.append(b)
+        elems += e
     layers, t, nb = [], 0.0, 0
     for layer in range(case.layers):
         dt, b = time_oracle(case, reqs, [layer])
@@ -192,8 +246,8 @@ def cpu_baseline(case: W.Case, budget_s: float = 12.0) -> dict:
             break
     return {"value": nb / t / 1e9, "unit": "GB/s", "cores": oracle.threads_used(),
             "kind": "oracle",
-            "sample": f"{len(layers)} of {case.layers} layers x all {case.B} requests "
-                      f"({case.name}), fp64 C oracle, {t:.1f} s"}
+            "sample": f"{len(layers)} of {case.layers} layers x {len(reqs)} of {case.B} "
+                      f"requests ({case.name}), fp64 C oracle, {t:.1f} s"}
 
 
 def run_reference(args, case: W.Case) -> None:
@@ -283,14 +337,22 @@ def run_kvc(args, case: W.Case) -> None:
     barrier, max_over_ranks = reps.barrier, reps.max_over_ranks
 
     c = case
+    fp8 = args.kv_format == "fp8"
     tdt = {"fp16": torch.float16, "bf16": torch.bfloat16}[c.dtype]
-    cache = kvc.KVCache(c.B, c.H_kv, c.D, c.max_T, c.dtype, num_layers=c.layers)
+    cache = kvc.KVCache(c.B, c.H_kv, c.D, c.max_T, c.dtype, c.page_size, c.layers,
+                        c.num_pages, kv_format=args.kv_format)
+    bt = torch.from_numpy(c.block_table).cuda() if c.paged else None
+    max_pages = c.max_pages if c.paged else 0
     gen = torch.Generator(device="cuda")
     gen.manual_seed(c.seed * 1000 + rank)
     for layer in range(c.layers):
         for which in ("k", "v"):
             pool = cache.pool(layer, which)
-            pool.normal_(0.0, c.kv_std, generator=gen)
+            if fp8:  # any finite E4M3 codes, positive scales
+                pool.random_(0, 0x7E, generator=gen)
+                cache.scales(layer, which).uniform_(1e-3, 1e-2, generator=gen)
+            else:
+                pool.normal_(0.0, c.kv_std, generator=gen)
     qs = torch.randn((c.layers, c.B, c.H_q, c.T_new, c.D), device="cuda", dtype=tdt,
                      generator=gen) * c.q_std
     ks = torch.randn((c.layers, c.B, c.H_kv, c.T_new, c.D), device="cuda", dtype=tdt,
@@ -299,14 +361,14 @@ def run_kvc(args, case: W.Case) -> None:
                      generator=gen) * c.kv_std
     outs = torch.empty((c.layers, c.B, c.H_q, c.T_new, c.D), device="cuda", dtype=tdt)
     seq = torch.from_numpy(c.seq_lens).cuda()
-    cache.reserve(c.H_q, c.T_new)
-    ns, split_tokens = cache.plan(c.H_q, c.T_new)
+    cache.reserve(c.H_q, c.T_new, max_pages)
+    ns, split_tokens = cache.plan(c.H_q, c.T_new, max_pages)
     stream = torch.cuda.Stream()
     scale = c.scale
 
     def step(q=qs, k=ks, v=vs, o=outs):
         for layer in range(c.layers):
-            cache.append_attend(layer, k[layer], v[layer], q[layer], seq, scale=scale,
+            cache.append_attend(layer, k[layer], v[layer], q[layer], seq, bt, scale=scale,
                                 out=o[layer], stream=stream)
 
     # one launch per layer on the persistent path (append, attend and merge fused)
@@ -361,7 +423,7 @@ def run_kvc(args, case: W.Case) -> None:
         for _ in range(max(2, args.steps // 10)):
             for layer in range(c.layers):
                 evs[layer][0].record(stream)
-                cache.append_attend(layer, ks[layer], vs[layer], qs[layer], seq, scale=scale,
+                cache.append_attend(layer, ks[layer], vs[layer], qs[layer], seq, bt, scale=scale,
                                     out=outs[layer], stream=stream)
                 evs[layer][1].record(stream)
             stream.synchronize()
@@ -394,17 +456,36 @@ def run_kvc(args, case: W.Case) -> None:
     h2d = (hq.numel() + hk.numel() + hv.numel()) * c.elt
     d2h = ho.numel() * c.elt
 
-    step_bytes = c.layers * c.algorithmic_bytes()
+    layer_bytes = fp8_algorithmic_bytes(c) if fp8 else c.algorithmic_bytes()
+    step_bytes = c.layers * layer_bytes
     value = whole_job_gbs(world, step_bytes, ms)
-    # K/V read + q read + out written + k_new/v_new read + their rows written to the cache
-    attend_bytes = c.algorithmic_bytes() + 2 * c.B * c.H_kv * c.T_new * c.D * c.elt
+    # one call's bytes: K/V read + q read + out written + k_new/v_new read + rows written
+    # (the FP8 count already holds both sides of the append)
+    attend_bytes = layer_bytes + (0 if fp8 else 2 * c.B * c.H_kv * c.T_new * c.D * c.elt)
     achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
     tok_layer_step = world * c.B * c.T_new / (ms * 1e-3 / c.layers)
-
-    traffic = profiled_traffic(f"attend_streamk_kernel<{c.D},1,{c.dtype},contiguous>")
+    kernel = attend_kernel_name(c, args.kv_format, split_tokens)
+    rows = (c.H_q // c.H_kv) * c.T_new
+    # attention flops of one call: 4 per (query row, visible position, dimension); new row
+    # i of request b sees L_b + i + 1 positions
+    seen = float(sum(int(L) * c.T_new + c.T_new * (c.T_new + 1) // 2 for L in c.seq_lens))
+    flops = 4.0 * seen * c.H_q * c.D
+    if kernel.startswith("attend_tc_kernel"):
+        tpeak, tpeak_kind = tensor_peak()
+        achieved_tf = flops / (attend_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tpeak,
+                    "unit": "TFLOP/s", "frac": achieved_tf / tpeak, "traffic": None,
+                    "peak_source": tpeak_kind}
+    else:
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": profiled_traffic(kernel),
+                    "peak_source": peak_kind}
+    roofline["kernel"] = (kernel + (", fused: one launch per kvc_append_attend call (append, "
+                                    "split attend, merge)" if split_tokens == 0 else
+                                    ", after the append kernel"))
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         cpu = cpu_baseline(c)
 
     graph.reset()
@@ -417,20 +498,22 @@ def run_kvc(args, case: W.Case) -> None:
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": c.dtype, "data": "synthetic",
             "config": {"workload": c.name, "layers": c.layers, "B": c.B, "H_q": c.H_q,
-                       "H_kv": c.H_kv, "D": c.D, "T_past": int(c.seq_lens[0]),
-                       "T_new": c.T_new, "cache": "contiguous",
+                       "H_kv": c.H_kv, "D": c.D,
+                       "T_past": (int(c.seq_lens[0]) if len(set(c.seq_lens.tolist())) == 1
+                                  else [int(c.seq_lens.min()), int(c.seq_lens.max())]),
+                       "T_new": c.T_new,
+                       "cache": (f"paged P{c.page_size}" if c.paged else "contiguous") +
+                                (", FP8 E4M3 + per-row scales" if fp8 else ""),
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (8.6 GB of K/V per step)",
+                       "l2": (f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB read per "
+                              f"step over {c.layers} layer caches)"),
                        "split_k": {"num_splits": ns, "split_tokens": split_tokens},
-                       "timing": "CUDA graph of one 32-layer step, CUDA events"},
+                       "timing": f"CUDA graph of one {c.layers}-layer step, CUDA events"},
             "pct_of_peak": 100.0 * value / world / peak,
             "tokens_per_s_per_layer_step": tok_layer_step,
             "ms_per_step_eager": ms_eager,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "attend_streamk_kernel, fused: one launch per "
-                                   "kvc_append_attend call (append, split attend, merge)",
-                         "peak_source": peak_kind},
+            "roofline": roofline,
+            "attention_tflops": flops / (attend_ms * 1e-3) / 1e12,
             "e2e": {"value": whole_job_gbs(world, step_bytes, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
@@ -444,6 +527,11 @@ def run_kvc(args, case: W.Case) -> None:
 
 WORKLOADS = {
     "gqa_32layer": lambda: W.gqa_32layer(32),
+    "paged_gqa": lambda: W.paged_gqa(),
+    "mha_b4_L4096": lambda: W.mha_sweep(4096),
+    "mha_b4_L8192": lambda: W.mha_sweep(8192),
+    **{f"verify_g{g}_hkv{h}": (lambda g=g, h=h: W.spec_verify(g, h))
+       for g in (2, 4, 8) for h in (8, 1)},
 }
 
 
@@ -457,12 +545,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (a smaller case for profiling)")
+    ap.add_argument("--kv-format", default="native", choices=["native", "fp8"],
+                    help="K/V storage: the 16-bit type, or FP8 E4M3 with per-row scales")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     case = WORKLOADS[args.workload]()
     if args.layers:
         case.layers = args.layers
+    else:  # enough independent layer caches that a step reads more than 4x L2
+        case.layers = max(case.layers, -(-int(4 * L2_BYTES) // case.kv_read_bytes(True)))
     if args.impl == "reference":
         run_reference(args, case)
     else:
