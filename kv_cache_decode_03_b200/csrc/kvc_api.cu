@@ -52,6 +52,12 @@ constexpr int kEltBytes = 2;
 #define KVC_TMA_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
 #endif
 
+// Query rows per KV head from which the tensor-core kernels take over from the CUDA-core
+// kernel (where tensor maps exist: D 64 or 128, pages of 8 or more tokens).
+#ifndef KVC_MMA_MIN_ROWS
+#define KVC_MMA_MIN_ROWS 1
+#endif
+
 // Query rows per KV head from which the tcgen05 kernel (128-row blocks) takes over.
 #ifndef KVC_TC_MIN_ROWS
 #define KVC_TC_MIN_ROWS 64
@@ -393,7 +399,7 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
   // From KVC_TC_MIN_ROWS rows a 128-row block fills the tcgen05 MMA's M.
   pl.fp8 = c->fp8;
   pl.tc = !c->fp8 && c->tma && rows >= KVC_TC_MIN_ROWS;
-  pl.mma = !c->fp8 && c->tma && rows >= 3 && !pl.tc;
+  pl.mma = !c->fp8 && c->tma && rows >= KVC_MMA_MIN_ROWS && !pl.tc;
   int tile, occ, scratch = 1 << 30;
   if (pl.fp8) {
     pl.NT = rows <= 8 ? 1 : (rows <= 16 ? 2 : 4);

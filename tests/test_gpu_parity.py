@@ -413,8 +413,15 @@ FUSED = {
                                                  [62, 125, 1021], seed=44, max_T=1100),
     "d64_fp16_paged": lambda: W.paged_case("fz4", 4, 16, 4, 64, "fp16", 2, 0, 900, 16,
                                            seed=45, pool_seed=46),
+    # one and two query rows per KV head (MHA decode, MHA verify) on the same kernel
+    "mha_d64_decode": lambda: W.contig_case("fz7", 4, 12, 12, 64, "fp16", 1,
+                                            [4095, 0, 63, 1500], seed=50, max_T=4100),
+    "mha_d128_paged_t2": lambda: W.paged_case("fz8", 3, 8, 8, 128, "bf16", 2, 0, 1200, 16,
+                                              seed=51, pool_seed=52),
+    "gqa2_d64_paged": lambda: W.paged_case("fz9", 3, 8, 4, 64, "bf16", 1, 0, 900, 8,
+                                           seed=53, pool_seed=54),
     # other kernels: append then attend, two launches
-    "mha_simt": lambda: W.contig_case("fz5", 2, 8, 8, 64, "fp16", 1, [700, 33], seed=47),
+    "mha_simt_d32": lambda: W.contig_case("fz5", 2, 8, 8, 32, "fp16", 1, [700, 33], seed=47),
     "mqa_splitk": lambda: W.paged_case("fz6", 2, 32, 1, 128, "bf16", 4, 100, 2000, 16,
                                        seed=48, pool_seed=49),
 }
