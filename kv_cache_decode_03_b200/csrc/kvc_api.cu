@@ -71,6 +71,16 @@ constexpr int kEltBytes = 2;
 #ifndef KVC_FP8_SPLIT_WAVES  // the FP8 kernel's tiles are cheaper to load: fewer, longer slices
 #define KVC_FP8_SPLIT_WAVES 4
 #endif
+// A tcgen05 slice carries a large fixed cost (TMEM allocation, 32 KB of Q staged, the
+// pipeline fill, its part of the merge): plan two waves and slices of at least 16 tiles.
+// Measured against 4, 8 and 16 waves, 1 wave, and a model fitting whole waves, this was
+// best or close on the MQA verify and MHA prefill-chunk workloads.
+#ifndef KVC_TC_SPLIT_WAVES
+#define KVC_TC_SPLIT_WAVES 2
+#endif
+#ifndef KVC_TC_MIN_SLICE_TILES
+#define KVC_TC_MIN_SLICE_TILES 16
+#endif
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -453,10 +463,13 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
   cap = std::max<long long>(cap, 1);
   const long long units = (long long)c->B * c->H_kv * pl.row_blocks;
   const long long target =
-      (long long)(pl.fp8 ? KVC_FP8_SPLIT_WAVES : KVC_SPLIT_WAVES) * c->num_sms * occ;
+      (long long)(pl.fp8 ? KVC_FP8_SPLIT_WAVES : pl.tc ? KVC_TC_SPLIT_WAVES : KVC_SPLIT_WAVES) *
+      c->num_sms * occ;
   // the merging CTA keeps one weight per (row, slice) in shared memory
   const long long max_ns = std::min<long long>((cap + tile - 1) / tile, scratch / pl.R);
   long long ns = std::min(std::max((target + units - 1) / units, 1LL), max_ns);
+  if (pl.tc)
+    ns = std::max(1LL, std::min(ns, cap / ((long long)KVC_TC_MIN_SLICE_TILES * tile)));
   long long S = (cap + ns - 1) / ns;
   S = (S + tile - 1) / tile * tile;
   ns = (cap + S - 1) / S;

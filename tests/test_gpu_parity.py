@@ -124,10 +124,10 @@ def test_many_rows_page_sizes(P):
 
 
 def test_many_rows_long_context_split_cap():
-    """One request, one KV head, 30K positions: the split count hits the merge's
-    shared-memory cap."""
-    case = W.contig_case("rows_long", 1, 64, 1, 128, "bf16", 2, [30000], seed=90,
-                         max_T=30002)
+    """One request, one KV head, 100K positions: the split count hits the merge's
+    shared-memory cap (90 slices of 128 rows at D = 128)."""
+    case = W.contig_case("rows_long", 1, 64, 1, 128, "bf16", 2, [100000], seed=90,
+                         max_T=100002)
     run_case(case)
 
 
