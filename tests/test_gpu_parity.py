@@ -123,9 +123,9 @@ def test_many_rows_page_sizes(P):
     run_case(case)
 
 
-def test_many_rows_long_context_split_cap():
-    """One request, one KV head, 100K positions: the split count hits the merge's
-    shared-memory cap (90 slices of 128 rows at D = 128)."""
+def test_many_rows_long_context_many_slices():
+    """One request, one KV head, 100K positions: about a hundred slices of one row block,
+    merged by one CTA."""
     case = W.contig_case("rows_long", 1, 64, 1, 128, "bf16", 2, [100000], seed=90,
                          max_T=100002)
     run_case(case)
