@@ -30,7 +30,9 @@
 //
 // CUDA cores, not tensor cores: with R <= 4 rows per K/V element this is ~R
 // flop per K/V byte, far below the tensor ridge; the kernel is HBM-bound once
-// its instruction count per K/V row is low enough.
+// its instruction count per K/V row is low enough.  It serves the caches the
+// tensor-core kernels have no TMA tensor maps for: D = 32, pages of fewer than
+// 8 tokens.
 #pragma once
 
 #include <math.h>

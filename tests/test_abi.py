@@ -12,7 +12,8 @@ import kv_cache_decode_03_b200 as kvc
 from kv_cache_decode_03_b200 import build as kvc_build
 from tests import oracle_pins
 
-HEADER = Path(__file__).resolve().parents[1] / "include" / "kvc.h"
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "kvc.h"
 
 
 @pytest.fixture(scope="module")
@@ -73,3 +74,31 @@ def test_null_handle_calls_fail_cleanly(lib):
     assert lib.kvc_get_error(None) == kvc.KVC_ERR_INVALID_ARG
     assert kvc.kvc_bytes(0) == 0
     assert lib.kvc_destroy(None) == kvc.KVC_OK
+
+
+def test_missing_library_fails_loudly():
+    """Without libkvc.so the product path raises; there is no fallback."""
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from pathlib import Path\n"
+        "import kv_cache_decode_03_b200 as k\n"
+        "k.LIB_PATH = Path('/nonexistent/libkvc.so'); k._lib = None\n"
+        "try:\n"
+        "    k.KVCache(1, 1, 64, 8, 'bf16')\n"
+        "except ImportError as e:\n"
+        "    print('raised:', e)\n"
+    ) % str(ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert "raised:" in out.stdout, out.stdout + out.stderr
+
+
+def test_package_does_not_load_the_oracle():
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "import kv_cache_decode_03_b200\n"
+            "print('oracle' in sys.modules)\n") % str(ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert out.stdout.strip() == "False", out.stdout + out.stderr
