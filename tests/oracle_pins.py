@@ -317,8 +317,9 @@ def check_cached_equals_full_causal(o):
         q, K, V, _ = random_case(B, H, H, T, D, [0, 0], dtype, seed=77 + dtype)
         scale = float(np.float32(1 / math.sqrt(D)))
         full = o.attend(q, K, V, np.zeros(B, np.int32), scale, dtype, nthreads=2)
-        Kc = np.zeros_like(K)
-        Vc = np.zeros_like(V)
+        # two slack rows: a planted off-by-one writes there instead of past the array
+        Kc = np.zeros(K.shape[:2] + (T + 2, D), K.dtype)
+        Vc = np.zeros(V.shape[:2] + (T + 2, D), V.dtype)
         for t in range(T):
             L = np.full(B, t, np.int32)
             o.append_contig(Kc, np.ascontiguousarray(K[:, :, t:t + 1]), L)
@@ -326,7 +327,8 @@ def check_cached_equals_full_causal(o):
             step = o.attend(np.ascontiguousarray(q[:, :, t:t + 1]), Kc, Vc, L, scale, dtype,
                             nthreads=2)
             assert np.array_equal(step[:, :, 0], full[:, :, t]), f"step {t}"
-        assert np.array_equal(Kc, K) and np.array_equal(Vc, V)
+        assert np.array_equal(Kc[:, :, :T], K) and np.array_equal(Vc[:, :, :T], V)
+        assert not Kc[:, :, T:].any() and not Vc[:, :, T:].any()
 
 
 def check_chunked_equals_naive(o):
@@ -371,7 +373,9 @@ def check_paged_equals_contig(o):
     max_pages = int(-(-T_cap // P))
     num_pages = int(need.sum()) + 2
     perm = np.random.default_rng(5).permutation(num_pages).astype(np.int32)
-    bt = np.full((B, max_pages), -1, np.int32)
+    # entries the pages never reach name the spare page past the pool (see pool_mem):
+    # a planted mistake that reads them writes into memory the test owns
+    bt = np.full((B, max_pages), num_pages, np.int32)
     cur = 0
     for b in range(B):
         bt[b, :need[b]] = perm[cur:cur + need[b]]
@@ -387,7 +391,10 @@ def check_paged_equals_contig(o):
         assert np.array_equal(contig[b, :, L[b] + T_new:], hist[b, :, L[b] + T_new:])
     # paged: place the history rows by hand (page = table[pos // P], slot = pos % P)
     canary = np.uint16(0x7E01)
-    pool = np.full((num_pages, H_kv, P, D), canary, np.uint16)
+    # the pool is a view of one page more, so a planted mistake that writes past the
+    # pool lands in memory the test owns
+    pool_mem = np.full((num_pages + 1, H_kv, P, D), canary, np.uint16)
+    pool = pool_mem[:num_pages]
     for b in range(B):
         for pos in range(int(L[b])):
             pool[bt[b, pos // P], :, pos % P] = hist[b, :, pos]
