@@ -39,6 +39,26 @@
 
 namespace kvc {
 
+// L2 prefetch of one box: nothing lands in shared memory and nothing signals
+// completion, so it changes no result whatever the coordinates name.
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(tmap), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+// -------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the
+// grid ahead of it in the stream has finished.  griddep_wait() blocks until that
+// grid has completed and its writes are visible (it returns at once for a plain
+// launch); griddep_launch_dependents() lets the next such grid begin launching.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <int D>
 struct StreamKCfg {
   static constexpr int kWarps = 4;
@@ -141,77 +161,140 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
   const int lane = tid & 31;
   const int c = blockIdx.x;
 
-  // ---------------------------------------------- per-request tile prefix
-  int* P = reinterpret_cast<int*>(smem);  // [B + 1], in the ring before any copy
-  {
-    const int per = ceil_div(p.B, NTH);
-    const int b_lo = min(p.B, tid * per), b_hi = min(p.B, b_lo + per);
-    int sum = 0;
-    for (int b = b_lo; b < b_hi; ++b) {
-      const int L = p.seq_lens[b];
-      int t = 0;
-      if (length_ok(p, L, PAGED)) t = request_tiles<R>(p, L);
-      else flag_error(p.err, KVC_ERR_BOUNDS);
-      P[b] = t;
-      sum += t;
-    }
-    int incl = sum;  // inclusive scan across the block
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    int* wsum = flags + 4;  // [W]
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += wsum[w];
-    int run = base + incl - sum;
-    for (int b = b_lo; b < b_hi; ++b) {
-      const int t = P[b];
-      P[b] = run;
-      run += t;
-    }
-    if (tid == NTH - 1) P[p.B] = base + incl;
-    __syncthreads();
-  }
-  const long long Wt = P[p.B];
-  const int G = (int)(Wt < (long long)gridDim.x ? Wt : (long long)gridDim.x);
-  if (c >= G) return;
-  const long long lo = (long long)c * Wt / G;
-  const long long hi = (long long)(c + 1) * Wt / G;
-  const int ntiles = (int)(hi - lo);
+  // Programmatic dependent launch: the next grid in the stream may begin as
+  // this one's CTAs retire.  Before griddep_wait() this kernel writes no global
+  // memory and reads seq_lens and the block table only to aim L2 prefetches,
+  // which change no result; the pass that counts runs after the wait.
+  griddep_launch_dependents();
 
-  // starting position: request (binary search), KV head, row block
+  // ------------------------------------ per-request tile prefix and this CTA's range
+  int* P = reinterpret_cast<int*>(smem);  // [B + 1], in the ring before any copy
+  long long Wt = 0, lo = 0;
+  int G = 0, ntiles = 0;
   TileCursor<R> cur;
-  {
-    int a = 0, z = p.B;  // largest b with P[b] <= lo
-    while (z - a > 1) {
-      const int mid = (a + z) >> 1;
-      if (P[mid] <= lo) a = mid;
-      else z = mid;
-    }
-    while (P[a + 1] == P[a]) ++a;  // skip requests with no tiles
-    cur.b = a;
-    cur.L = p.seq_lens[a];
-    int local = (int)(lo - P[a]);
-    const int per_g = (P[a + 1] - P[a]) / p.H_kv;
-    cur.g = local / per_g;
-    local -= cur.g * per_g;
-    cur.rb = 0;
-    while (true) {
-      const int t = ceil_div(cur.L + row_block(cur.rb, R, p.rows, p.T_new).imax + 1, 64);
-      if (local < t) {
-        cur.seg_tiles = t;
-        break;
+  // Returns whether this CTA has tiles; ends with a barrier (P is then dead).
+  auto locate = [&](bool authoritative) -> bool {
+    {
+      const int per = ceil_div(p.B, NTH);
+      const int b_lo = min(p.B, tid * per), b_hi = min(p.B, b_lo + per);
+      int sum = 0;
+      for (int b = b_lo; b < b_hi; ++b) {
+        const int L = p.seq_lens[b];
+        int t = 0;
+        if (length_ok(p, L, PAGED)) t = request_tiles<R>(p, L);
+        else if (authoritative) flag_error(p.err, KVC_ERR_BOUNDS);
+        P[b] = t;
+        sum += t;
       }
-      local -= t;
-      ++cur.rb;
+      int incl = sum;  // inclusive scan across the block
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      int* wsum = flags + 4;  // [W]
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      int base = 0;
+      for (int w = 0; w < warp; ++w) base += wsum[w];
+      int run = base + incl - sum;
+      for (int b = b_lo; b < b_hi; ++b) {
+        const int t = P[b];
+        P[b] = run;
+        run += t;
+      }
+      if (tid == NTH - 1) P[p.B] = base + incl;
+      __syncthreads();
     }
-    cur.k = local;
-    cur.seg_start = lo - local;
+    Wt = P[p.B];
+    G = (int)(Wt < (long long)gridDim.x ? Wt : (long long)gridDim.x);
+    bool work = c < G;  // the same in every thread
+    if (work) {
+      lo = (long long)c * Wt / G;
+      ntiles = (int)((long long)(c + 1) * Wt / G - lo);
+      // starting position: request (binary search), KV head, row block
+      int a = 0, z = p.B;  // largest b with P[b] <= lo
+      while (z - a > 1) {
+        const int mid = (a + z) >> 1;
+        if (P[mid] <= lo) a = mid;
+        else z = mid;
+      }
+      while (P[a + 1] == P[a]) ++a;  // skip requests with no tiles
+      cur.b = a;
+      cur.L = p.seq_lens[a];
+      // a length read before the wait may be changing under this read
+      work = length_ok(p, cur.L, PAGED);
+      int local = (int)(lo - P[a]);
+      const int per_g = (P[a + 1] - P[a]) / p.H_kv;
+      cur.g = local / per_g;
+      local -= cur.g * per_g;
+      cur.rb = 0;
+      while (work) {
+        const int t = ceil_div(cur.L + row_block(cur.rb, R, p.rows, p.T_new).imax + 1, 64);
+        if (local < t || cur.rb == p.row_blocks - 1) {
+          cur.seg_tiles = t;
+          break;
+        }
+        local -= t;
+        ++cur.rb;
+      }
+      cur.k = local;
+      cur.seg_start = lo - local;
+    }
+    __syncthreads();  // P is dead: the ring may now be filled
+    return work;
+  };
+
+  // The TMA boxes of the tile under cursor pc: f(x, y, byte offset in the stage).
+  auto for_each_box = [&](const TileCursor<R>& pc, auto&& f) {
+    const int t0 = pc.k * C::kTile;
+    if (!PAGED) {
+      const int y = (pc.b * p.H_kv + pc.g) * p.max_T + t0;
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h) f(h * 64, y, h * C::kBoxBytes);
+    } else {
+      const int Pg = 1 << p.page_shift;
+      const int box_rows = Pg < C::kTile ? Pg : C::kTile;
+      const int n_seg = pc.L + row_block(pc.rb, R, p.rows, p.T_new).imax + 1;
+      const int32_t* bt = p.block_table + (size_t)pc.b * p.max_pages;
+      const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
+#pragma unroll 1
+      for (int t = t0; t < t0 + C::kTile; t += box_rows) {
+        int y = beyond;
+        if (t < n_seg) {
+          const int page = bt[t >> p.page_shift];
+          if (page >= 0 && page < p.num_pages)
+            y = (page * p.H_kv + pc.g) * Pg + (t & (Pg - 1));
+          else
+            f(-1, 0, 0);  // a bad page id: reported by the caller
+        }
+        const int off = (t - t0) * 128;
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) f(h * 64, y, h * C::kBoxBytes + off);
+      }
+    }
+  };
+
+  // Speculative pass: warm L2 with this CTA's first tiles while the grid ahead
+  // finishes.  Lengths or pages that change before the wait only waste a prefetch.
+  if (locate(false) && tid == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    // only boxes wholly inside the tensor: the cursor may walk off stale lengths
+    const int rows_total = PAGED ? p.num_pages * p.H_kv << p.page_shift : p.B * p.H_kv * p.max_T;
+    const int box_h = PAGED ? min(1 << p.page_shift, C::kTile) : C::kTile;
+    TileCursor<R> pc = cur;
+    for (int i = 0; i < min(C::kStages, ntiles) && pc.b < p.B; ++i) {
+      for_each_box(pc, [&](int x, int y, int) {
+        if (x < 0 || y < 0 || y + box_h > rows_total) return;
+        tma_prefetch_2d(&tmk, x, y);
+        tma_prefetch_2d(&tmv, x, y);
+      });
+      pc.next(p, PAGED);
+    }
   }
-  __syncthreads();  // P is dead: the ring may now be filled
+  griddep_wait();
+  if (!locate(true)) return;
 
   if (tid == 0) {
     prefetch_tmap(&tmk);
@@ -246,38 +329,14 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     }
     unsigned char* dk = sk + st * C::kTileBytes;
     unsigned char* dv = sv + st * C::kTileBytes;
-    const int t0 = pc.k * C::kTile;
-    if (!PAGED) {
-      const int y = (pc.b * p.H_kv + pc.g) * p.max_T + t0;
-#pragma unroll
-      for (int h = 0; h < C::kHalves; ++h) {
-        tma_load_2d(dk + h * C::kBoxBytes, &tmk, h * 64, y, &full[st], pol);
-        tma_load_2d(dv + h * C::kBoxBytes, &tmv, h * 64, y, &full[st], pol);
+    for_each_box(pc, [&](int x, int y, int off) {
+      if (x < 0) {
+        flag_error(p.err, KVC_ERR_BOUNDS);
+        return;
       }
-    } else {
-      const int Pg = 1 << p.page_shift;
-      const int box_rows = Pg < C::kTile ? Pg : C::kTile;
-      const int n_seg = pc.L + row_block(pc.rb, R, p.rows, p.T_new).imax + 1;
-      const int32_t* bt = p.block_table + (size_t)pc.b * p.max_pages;
-      const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
-#pragma unroll 1
-      for (int t = t0; t < t0 + C::kTile; t += box_rows) {
-        int y = beyond;
-        if (t < n_seg) {
-          const int page = bt[t >> p.page_shift];
-          if (page >= 0 && page < p.num_pages)
-            y = (page * p.H_kv + pc.g) * Pg + (t & (Pg - 1));
-          else
-            flag_error(p.err, KVC_ERR_BOUNDS);
-        }
-        const int off = (t - t0) * 128;
-#pragma unroll
-        for (int h = 0; h < C::kHalves; ++h) {
-          tma_load_2d(dk + h * C::kBoxBytes + off, &tmk, h * 64, y, &full[st], pol);
-          tma_load_2d(dv + h * C::kBoxBytes + off, &tmv, h * 64, y, &full[st], pol);
-        }
-      }
-    }
+      tma_load_2d(dk + off, &tmk, x, y, &full[st], pol);
+      tma_load_2d(dv + off, &tmv, x, y, &full[st], pol);
+    });
     ++issued;
     pc.next(p, PAGED);
   };

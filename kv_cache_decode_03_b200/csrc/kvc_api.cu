@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -553,14 +554,36 @@ kvc_status dispatch_mma(const kvc::AttendParams& p, int D, int NT, bool paged,
                : dispatch_mma_nt<128, T, false>(p, NT, tk, tv, s);
 }
 
+// Dependent launch of the stream-K kernel is on unless KVC_PDL=0 (read once).
+static bool dependent_launch_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("KVC_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 template <int D, int NT, typename T, bool PAGED>
 kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, const CUtensorMap& tk,
                                  const CUtensorMap& tv, cudaStream_t stream) {
   using C = kvc::StreamKCfg<D>;
   streamk_occupancy<D, NT, T, PAGED>();  // sets the shared-memory attribute once
   const size_t smem = C::template smem_bytes<NT>();
-  kvc::attend_streamk_kernel<D, NT, T, PAGED><<<grid, C::kThreads, smem, stream>>>(p, tk, tv);
-  return cuda_status(cudaGetLastError());
+  // Programmatic stream serialization: the kernel may start while the grid
+  // ahead of it retires; it waits for that grid (griddepcontrol.wait) before
+  // its first read that counts or any write.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent_launch_enabled() ? 1 : 0;
+  return cuda_status(
+      cudaLaunchKernelEx(&cfg, kvc::attend_streamk_kernel<D, NT, T, PAGED>, p, tk, tv));
 }
 
 template <typename T>
