@@ -153,6 +153,11 @@ kvc_status kvc_append(kvc_cache* cache, int layer, const void* k_new, const void
  * owned by the cache for split-K partial results; it grows on demand (a device
  * allocation, so the first call with a larger shape should precede any stream capture;
  * kvc_reserve sizes it up front).
+ * Launch: when the plan picks the persistent stream-K kernel (D 64/128, 1-16 query rows
+ * per KV head, no window), it is launched with programmatic stream serialization.  It
+ * may start while the kernel ahead of it on the stream retires, but reads no input that
+ * counts and writes nothing before that kernel has completed.  The environment variable
+ * KVC_PDL=0 (read once) turns this into a plain launch.
  */
 kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
                       const int32_t* block_table, int max_pages, const int32_t* seq_lens,
