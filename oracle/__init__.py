@@ -91,6 +91,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_encode_e4m3.restype = None
     lib.oracle_quantize_fp8.argtypes = [P, I64, I, P, P]
     lib.oracle_quantize_fp8.restype = None
+    lib.oracle_append_fp8_contig.argtypes = [I, I, I, I, I, I, P, P, P, P]
+    lib.oracle_append_fp8_contig.restype = None
+    lib.oracle_append_fp8_paged.argtypes = [I, I, I, I, I, I, P, P, P, P, P]
+    lib.oracle_append_fp8_paged.restype = None
     lib.oracle_gather_rows.argtypes = [I, I, I, I, I, I, P, P, P, P]
     lib.oracle_gather_rows.restype = None
     lib.oracle_attend_fp8.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, D, I, I, P, I]
@@ -218,23 +222,34 @@ class Oracle:
 
     def append_fp8(self, codes, scales, new_kv, seq_lens, block_table=None) -> None:
         """Quantise the new rows (B, H_kv, T_new, D) and write codes and scales into the
-        pool images in place: contiguous codes (B, H_kv, T_cap, D) with scales
-        (B, H_kv, T_pad); paged codes (num_pages, H_kv, P, D) with scales
-        (num_pages, H_kv, P); row L_b + i of (b, g) as for the 16-bit append."""
-        qc, qs = self.quantize_fp8(new_kv)
-        B, H_kv, T_new, _ = qc.shape
+        pool images in place (oracle.c: oracle_append_fp8_contig / _paged): contiguous
+        codes (B, H_kv, T_cap, D) with scales (B, H_kv, T_pad); paged codes
+        (num_pages, H_kv, P, D) with scales (num_pages, H_kv, P); row L_b + i of (b, g)
+        as for the 16-bit append."""
+        nk = _u16(new_kv)
+        B, H_kv, T_new, D = nk.shape
         sl = _i32(seq_lens)
-        for b in range(B):
-            for i in range(T_new):
-                pos = int(sl[b]) + i
-                if block_table is None:
-                    codes[b, :, pos] = qc[b, :, i]
-                    scales[b, :, pos] = qs[b, :, i]
-                else:
-                    P = codes.shape[2]
-                    page = int(block_table[b, pos // P])
-                    codes[page, :, pos % P] = qc[b, :, i]
-                    scales[page, :, pos % P] = qs[b, :, i]
+        assert codes.dtype == np.uint8 and codes.flags["C_CONTIGUOUS"]
+        assert scales.dtype == np.float32 and scales.flags["C_CONTIGUOUS"]
+        if block_table is None:
+            assert codes.shape[:2] == (B, H_kv) and codes.shape[3] == D
+            T_cap, T_pad = codes.shape[2], scales.shape[2]
+            assert scales.shape == (B, H_kv, T_pad) and T_pad >= T_cap
+            assert np.all((sl >= 0) & (sl + T_new <= T_cap))
+            self.lib.oracle_append_fp8_contig(B, H_kv, T_new, D, T_cap, T_pad, _ptr(nk),
+                                              _ptr(sl), _ptr(codes), _ptr(scales))
+            return
+        num_pages, hk, P, d = codes.shape
+        assert (hk, d) == (H_kv, D) and scales.shape == (num_pages, H_kv, P)
+        bt = _i32(block_table)
+        max_pages = bt.shape[1]
+        assert np.all((sl + T_new - 1) // P < max_pages)
+        rows = np.arange(B)
+        for j in range(int(T_new)):
+            pages = bt[rows, (sl + j) // P]
+            assert np.all((pages >= 0) & (pages < num_pages))
+        self.lib.oracle_append_fp8_paged(B, H_kv, T_new, D, P, max_pages, _ptr(nk), _ptr(sl),
+                                         _ptr(bt), _ptr(codes), _ptr(scales))
 
     def gather_rows(self, pool, block_table, n_visible, T_cap: int) -> np.ndarray:
         """Logical (B, H_kv, T_cap, ...) view of a paged pool (num_pages, H_kv, P, ...) of

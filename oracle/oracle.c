@@ -25,7 +25,7 @@
  *        section 9.6 (paged KV cache managed in blocks), section 9.7 (flash
  *        attention is exact up to floating-point rounding).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - causal within the new chunk: new row i of a request with committed
  *     length L sees positions 0 .. L+i (the project-11 snippet applies no
  *     mask, which is only right for one new row);
@@ -251,26 +251,68 @@ void oracle_encode_e4m3(const float* src, uint8_t* dst, int64_t n)
         dst[i] = encode_e4m3(src[i]);
 }
 
+/* One row x of D bf16 words -> D codes and its scale. */
+static void quantize_row(const uint16_t* x, int D, uint8_t* code, float* scale_out)
+{
+    float amax = 0.0f;
+    for (int d = 0; d < D; ++d) {
+        float v = (float)decode_bf16(x[d]);
+        float av = v < 0 ? -v : v;
+        if (av > amax)
+            amax = av;
+    }
+    float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    *scale_out = scale;
+    for (int d = 0; d < D; ++d) {
+        float v = (float)decode_bf16(x[d]);
+        code[d] = encode_e4m3(v / scale);
+    }
+}
+
 /* rows (n_rows, D) of bf16 words -> codes (n_rows, D) and scales (n_rows) */
 void oracle_quantize_fp8(const uint16_t* rows, int64_t n_rows, int D, uint8_t* codes,
                          float* scales)
 {
-    for (int64_t r = 0; r < n_rows; ++r) {
-        const uint16_t* x = rows + r * D;
-        float amax = 0.0f;
-        for (int d = 0; d < D; ++d) {
-            float v = (float)decode_bf16(x[d]);
-            float av = v < 0 ? -v : v;
-            if (av > amax)
-                amax = av;
-        }
-        float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
-        scales[r] = scale;
-        for (int d = 0; d < D; ++d) {
-            float v = (float)decode_bf16(x[d]);
-            codes[r * D + d] = encode_e4m3(v / scale);
-        }
-    }
+    for (int64_t r = 0; r < n_rows; ++r)
+        quantize_row(rows + r * D, D, codes + r * D, &scales[r]);
+}
+
+/* FP8 append into a contiguous cache: new row i of (b, g) (bf16 words,
+ * new_kv (B, H_kv, T_new, D)) is quantised and lands at position
+ * pos = seq_lens[b] + i -- its D codes in codes (B, H_kv, T_cap, D), its
+ * scale in scales (B, H_kv, T_pad), the scale rows being T_pad long. */
+void oracle_append_fp8_contig(int B, int H_kv, int T_new, int D, int T_cap, int T_pad,
+                              const uint16_t* new_kv, const int32_t* seq_lens,
+                              uint8_t* codes, float* scales)
+{
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < H_kv; ++g)
+            for (int i = 0; i < T_new; ++i) {
+                int64_t pos = (int64_t)seq_lens[b] + i;
+                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;
+                int64_t code_row = ((int64_t)b * H_kv + g) * T_cap + pos;
+                int64_t scale_at = ((int64_t)b * H_kv + g) * T_pad + pos;
+                quantize_row(src, D, codes + code_row * D, &scales[scale_at]);
+            }
+}
+
+/* FP8 append into a paged pool ([P3] 9.6): position pos of request b is slot
+ * pos % P of page block_table[b * max_pages + pos / P]; codes are
+ * (num_pages, H_kv, P, D), scales (num_pages, H_kv, P). */
+void oracle_append_fp8_paged(int B, int H_kv, int T_new, int D, int P, int max_pages,
+                             const uint16_t* new_kv, const int32_t* seq_lens,
+                             const int32_t* block_table, uint8_t* codes, float* scales)
+{
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < H_kv; ++g)
+            for (int i = 0; i < T_new; ++i) {
+                int64_t pos = (int64_t)seq_lens[b] + i;
+                int64_t page = block_table[(int64_t)b * max_pages + pos / P];
+                int64_t slot = pos % P;
+                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;
+                int64_t row = (page * H_kv + g) * P + slot;
+                quantize_row(src, D, codes + row * D, &scales[row]);
+            }
 }
 
 /* Logical rows of a paged pool of fixed-size rows (any element type): row pos of

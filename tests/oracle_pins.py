@@ -40,8 +40,11 @@ What pins what:
 * the FP8 (E4M3) cache -- decoding against torch's float8_e4m3fn over all 256
   codes, encoding against torch's round-to-nearest-even below 448 (plus exact
   ties between neighbours and saturation above), row quantisation against the
-  format's half-step error bound and its amax -> 448 property, and attention
-  over the dequantised values against torch's fp64 SDPA (causal and windowed).
+  format's half-step error bound and its amax -> 448 property, attention
+  over the dequantised values against torch's fp64 SDPA (causal and windowed),
+  the any-width paged gather against a loop written in the test and against
+  the 16-bit gather, and the FP8 append's placement of codes and scales by
+  hand (contiguous) and through a shuffled block table (paged).
 """
 from __future__ import annotations
 
@@ -619,6 +622,93 @@ def check_attend_fp8_vs_sdpa(o):
             assert_close(got[b], ref[0].numpy(), 1e-13, 1e-11, what=f"W={W} S={S} b={b}")
 
 
+
+def _shuffled_table(L, T_new, P, T_cap, seed):
+    """A block table over a shuffled pool: request b's first ceil((L_b + T_new) / P)
+    entries name distinct pages; every other entry names the spare page num_pages."""
+    need = -(-(L + T_new) // P)
+    max_pages = int(-(-T_cap // P))
+    num_pages = int(need.sum()) + 2
+    perm = np.random.default_rng(seed).permutation(num_pages).astype(np.int32)
+    bt = np.full((len(L), max_pages), num_pages, np.int32)
+    cur = 0
+    for b in range(len(L)):
+        bt[b, :need[b]] = perm[cur:cur + need[b]]
+        cur += need[b]
+    return bt, num_pages
+
+
+def check_gather_rows(o):
+    """gather_rows (any row width) reads position pos of (b, g) from slot pos % P of page
+    table[b][pos // P]: against a loop written here over 1-byte and 4-byte rows, and
+    byte for byte against gather_paged on a 16-bit pool ("9. 推理" section 9.6)."""
+    B, H_kv, D, P, T_new, T_cap = 3, 2, 8, 4, 3, 20
+    L = np.array([0, 9, 14], np.int32)
+    bt, num_pages = _shuffled_table(L, T_new, P, T_cap, 21)
+    n = L + T_new
+    r = np.random.default_rng(22)
+    # spare pages past the pool: a planted mistake that reads past it stays in test memory
+    codes_mem = r.integers(0, 256, size=(num_pages + 4, H_kv, P, D)).astype(np.uint8)
+    scales_mem = np.float32(r.uniform(-5, 5, size=(num_pages + 4, H_kv, P)))
+    words_mem = r.integers(0, 1 << 16, size=(num_pages + 4, H_kv, P, D)).astype(np.uint16)
+    for pool_mem in (codes_mem, scales_mem, words_mem):
+        pool = pool_mem[:num_pages]
+        got = o.gather_rows(pool, bt, n, T_cap)
+        ref = np.zeros((B, H_kv, T_cap) + pool.shape[3:], pool.dtype)
+        for b in range(B):
+            for g in range(H_kv):
+                for pos in range(int(n[b])):
+                    ref[b, g, pos] = pool[bt[b, pos // P], g, pos % P]
+        assert got.dtype == pool.dtype and got.shape == ref.shape
+        assert np.array_equal(got.view(np.uint8), ref.view(np.uint8))
+    words = words_mem[:num_pages]
+    assert np.array_equal(o.gather_rows(words, bt, n, T_cap), o.gather_paged(words, bt, n, T_cap))
+
+
+def check_append_fp8_placement(o):
+    """FP8 append: new row i of (b, g), quantised, lands at position L_b + i -- codes and
+    scale together -- in a contiguous cache (checked by hand, with scale rows padded past
+    the capacity), and through a shuffled block table the paged pool reads back (with
+    gather_rows) exactly as the contiguous cache; nothing else is written."""
+    B, H_kv, D, P, T_new, T_cap, T_pad = 3, 2, 16, 4, 3, 20, 64
+    L = np.array([0, 9, 14], np.int32)
+    r = np.random.default_rng(31)
+    x = r.standard_normal((B, H_kv, T_new, D)) * np.exp(r.uniform(-3, 3, (B, H_kv, T_new, 1)))
+    new = bf16_words(x)
+    qc, qs = o.quantize_fp8(new)
+    # history: arbitrary codes and scales at every slot
+    hist_c = r.integers(0, 256, size=(B, H_kv, T_cap, D)).astype(np.uint8)
+    hist_s = np.float32(r.uniform(1, 2, size=(B, H_kv, T_pad)))
+    codes, scales = hist_c.copy(), hist_s.copy()
+    o.append_fp8(codes, scales, new, L)
+    for b in range(B):
+        for i in range(T_new):
+            assert np.array_equal(codes[b, :, L[b] + i], qc[b, :, i]), (b, i)
+            assert np.array_equal(scales[b, :, L[b] + i], qs[b, :, i]), (b, i)
+    assert np.any(codes != hist_c, axis=-1).sum() <= B * H_kv * T_new
+    assert (scales != hist_s).sum() == B * H_kv * T_new
+    # paged: the same history placed by hand, then the append through the table
+    bt, num_pages = _shuffled_table(L, T_new, P, T_cap, 32)
+    pc_mem = np.full((num_pages + 4, H_kv, P, D), 0xA5, np.uint8)
+    ps_mem = np.full((num_pages + 4, H_kv, P), -7.0, np.float32)
+    pc, ps = pc_mem[:num_pages], ps_mem[:num_pages]
+    for b in range(B):
+        for pos in range(int(L[b])):
+            pc[bt[b, pos // P], :, pos % P] = hist_c[b, :, pos]
+            ps[bt[b, pos // P], :, pos % P] = hist_s[b, :, pos]
+    before_c, before_s = pc_mem.copy(), ps_mem.copy()
+    o.append_fp8(pc, ps, new, L, bt)
+    n = L + T_new
+    got_c = o.gather_rows(pc, bt, n, T_cap)
+    got_s = o.gather_rows(ps, bt, n, T_cap)
+    for b in range(B):
+        assert np.array_equal(got_c[b, :, :n[b]], codes[b, :, :n[b]]), b
+        assert np.array_equal(got_s[b, :, :n[b]], scales[b, :, :n[b]]), b
+    assert (ps_mem != before_s).sum() == B * H_kv * T_new
+    assert np.any(pc_mem != before_c, axis=-1).sum() <= B * H_kv * T_new
+    assert np.array_equal(pc_mem[num_pages:], before_c[num_pages:])
+
+
 ALL_CHECKS = [
     check_decode_fp16_exhaustive,
     check_decode_bf16_exhaustive,
@@ -641,5 +731,7 @@ ALL_CHECKS = [
     check_e4m3_decode_exhaustive,
     check_e4m3_encode,
     check_quantize_fp8,
+    check_gather_rows,
+    check_append_fp8_placement,
     check_attend_fp8_vs_sdpa,
 ]

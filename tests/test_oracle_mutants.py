@@ -69,6 +69,27 @@ MUTANTS = [
     ("fp8_scale_447", "amax / 448.0f", "amax / 447.0f", 0),
     ("fp8_attend_drops_v_scale", "* (double)Vs[j])", "* 1.0)", 0),
     ("fp8_attend_k_scale_from_v", "(double)Ks[j])", "(double)Vs[j])", 0),
+    ("gather_rows_page_slot_swapped",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint8_t* src = pool",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos % P];\n                int64_t slot = pos / P;\n                const uint8_t* src = pool", 0),
+    ("gather_rows_ignores_table",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint8_t* src = pool",
+     "int64_t page = pos / P;\n                int64_t slot = pos % P;\n                const uint8_t* src = pool", 0),
+    ("gather_rows_head_dropped", "const uint8_t* src = pool + ((page * H_kv + g) * P + slot)",
+     "const uint8_t* src = pool + ((page * H_kv) * P + slot)", 0),
+    ("fp8_append_contig_off_by_one",
+     "int64_t pos = (int64_t)seq_lens[b] + i;\n                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;\n                int64_t code_row",
+     "int64_t pos = (int64_t)seq_lens[b] + i + 1;\n                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;\n                int64_t code_row", 0),
+    ("fp8_append_contig_scale_stride", "int64_t scale_at = ((int64_t)b * H_kv + g) * T_pad + pos;",
+     "int64_t scale_at = ((int64_t)b * H_kv + g) * T_cap + pos;", 0),
+    ("fp8_append_paged_off_by_one",
+     "int64_t pos = (int64_t)seq_lens[b] + i;\n                int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;\n                int64_t row",
+     "int64_t pos = (int64_t)seq_lens[b] + i + 1;\n                int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;\n                int64_t row", 0),
+    ("fp8_append_paged_slot_swapped",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos / P];\n                int64_t slot = pos % P;\n                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;\n                int64_t row",
+     "int64_t page = block_table[(int64_t)b * max_pages + pos % P];\n                int64_t slot = pos / P;\n                const uint16_t* src = new_kv + (((int64_t)b * H_kv + g) * T_new + i) * D;\n                int64_t row", 0),
+    ("fp8_append_scale_in_logical_page", "quantize_row(src, D, codes + row * D, &scales[row]);",
+     "quantize_row(src, D, codes + row * D, &scales[((pos / P) * H_kv + g) * P + slot]);", 0),
 ]
 
 
