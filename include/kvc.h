@@ -156,8 +156,10 @@ kvc_status kvc_append(kvc_cache* cache, int layer, const void* k_new, const void
  * Launch: when the plan picks the persistent stream-K kernel (D 64/128, 1-16 query rows
  * per KV head, no window), it is launched with programmatic stream serialization.  It
  * may start while the kernel ahead of it on the stream retires, but reads no input that
- * counts and writes nothing before that kernel has completed.  The environment variable
- * KVC_PDL=0 (read once) turns this into a plain launch.
+ * counts and writes nothing before that kernel has completed (before that it only reads
+ * seq_lens and the block table to plan, and prefetches K/V lines into L2).  The
+ * environment variable KVC_PDL=0 (read at kvc_create) or kvc_set_dependent_launch
+ * turns this into a plain launch.
  */
 kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
                       const int32_t* block_table, int max_pages, const int32_t* seq_lens,
@@ -225,6 +227,32 @@ kvc_status kvc_reserve(kvc_cache* cache, int H_q, int T_new, int max_pages);
  * KVC_ERR_BOUNDS or KVC_ERR_TIMEOUT) and clear it.
  */
 kvc_status kvc_get_error(kvc_cache* cache);
+
+/*
+ * kvc_set_dependent_launch -- launch this cache's persistent stream-K attend kernel with
+ * programmatic stream serialization (on != 0; the default unless the environment
+ * variable KVC_PDL=0) or as a plain launch (on == 0).  Results are the same either way;
+ * see kvc_attend.
+ */
+kvc_status kvc_set_dependent_launch(kvc_cache* cache, int on);
+
+/*
+ * kvc_set_wait_limit -- bound, in nanoseconds of %globaltimer, of every pipeline wait in
+ * the later attend launches on this cache (0 restores the default of one second).  A wait
+ * that runs out never hangs or traps: the kernel records KVC_ERR_TIMEOUT in the sticky
+ * error word, finishes without waiting again, and kvc_get_error reports it.
+ */
+kvc_status kvc_set_wait_limit(kvc_cache* cache, unsigned long long ns);
+
+/*
+ * kvc_inject_stall -- failure-detection test hook.  The next attend call on this cache,
+ * if it runs the persistent stream-K or the tcgen05 kernel, issues none of its copies,
+ * so its first pipeline wait runs out after the wait limit (kvc_set_wait_limit) and
+ * kvc_get_error then returns KVC_ERR_TIMEOUT; that call's output is undefined, the
+ * cache and the device context stay usable.  Other kernels ignore it; the next call
+ * consumes it either way.
+ */
+kvc_status kvc_inject_stall(kvc_cache* cache);
 
 /* kvc_status_string -- static, human-readable name of a status. */
 const char* kvc_status_string(kvc_status status);

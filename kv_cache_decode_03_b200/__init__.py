@@ -76,6 +76,9 @@ def library() -> ctypes.CDLL:
         "kvc_commit": ([P, P, P, I, P], I),
         "kvc_rollback": ([P, P, P, P], I),
         "kvc_copy_pages": ([P, P, P, I, P], I),
+        "kvc_set_dependent_launch": ([P, I], I),
+        "kvc_set_wait_limit": ([P, ctypes.c_ulonglong], I),
+        "kvc_inject_stall": ([P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -223,6 +226,18 @@ def kvc_rollback(cache: int, seq_lens: int, drop: int, stream: int) -> None:
 def kvc_copy_pages(cache: int, src: int, dst: int, n: int, stream: int) -> None:
     _check(library().kvc_copy_pages(cache, src or None, dst or None, n, stream or None),
            "kvc_copy_pages")
+
+
+def kvc_set_dependent_launch(cache: int, on: bool) -> None:
+    _check(library().kvc_set_dependent_launch(cache, 1 if on else 0), "kvc_set_dependent_launch")
+
+
+def kvc_set_wait_limit(cache: int, ns: int) -> None:
+    _check(library().kvc_set_wait_limit(cache, int(ns)), "kvc_set_wait_limit")
+
+
+def kvc_inject_stall(cache: int) -> None:
+    _check(library().kvc_inject_stall(cache), "kvc_inject_stall")
 
 
 # ---------------------------------------------------------------------------
@@ -388,6 +403,15 @@ class KVCache:
 
     def plan(self, H_q: int, T_new: int, max_pages: int = 0) -> tuple[int, int]:
         return kvc_plan_splits(self.handle, H_q, T_new, max_pages)
+
+    def set_dependent_launch(self, on: bool) -> None:
+        kvc_set_dependent_launch(self.handle, on)
+
+    def set_wait_limit(self, ns: int) -> None:
+        kvc_set_wait_limit(self.handle, ns)
+
+    def inject_stall(self) -> None:
+        kvc_inject_stall(self.handle)
 
     def commit(self, seq_lens, accepted, T_new: int, stream=None) -> None:
         """seq_lens[b] += accepted[b] on the device (0 <= accepted[b] <= T_new)."""

@@ -12,9 +12,12 @@
 //   number of K/V bytes to within one tile, whatever the mix of lengths.
 //   Every CTA computes the per-request tile counts and their prefix sums from
 //   seq_lens itself (a block scan), so the host needs no lengths.
-// * Lane 0 of warp 0 keeps the 3-stage TMA ring full across segment
-//   boundaries; the first tile of each segment piece also carries that
-//   segment's q rows (one bulk copy into a per-stage q slot).
+// * Warp 0 keeps the 3-stage TMA ring full across segment boundaries; the
+//   first tile of each segment piece also carries that segment's q rows (one
+//   bulk copy into a per-stage q slot).  On a paged cache lane k of warp 0
+//   looks up and loads box k of a tile, and the page ids of the next tile are
+//   read while the current one is consumed, so a tile costs one lookup latency
+//   (hidden) rather than one per page.
 // * When a piece ends, the four warps merge their partial results inside the
 //   stage they just consumed, while the other stages keep streaming.  A piece
 //   that covers its whole segment writes the output directly.  A CTA has at
@@ -22,7 +25,14 @@
 //   (c, 0) and (c, 1) of the workspace, and the last CTA of a segment to
 //   finish merges the segment's pieces by log-sum-exp ("9. 推理" 9.7:
 //   exact up to rounding); an atomic ticket after a release fence decides
-//   who is last, so nothing ever waits on another CTA.
+//   who is last, so nothing ever waits on another CTA.  The merge spreads each
+//   output quad's pieces over up to eight threads, so all of its loads are in
+//   flight at once, and combines them with shuffles.
+// * Launched with programmatic stream serialization, a CTA sets up its
+//   barriers, plans its tile range from the lengths as they stand and
+//   prefetches the first tiles of that range into L2 while the grid ahead
+//   finishes; after the dependency wait it re-reads the lengths and keeps the
+//   plan when none changed.
 #pragma once
 
 #include <cuda.h>
@@ -35,6 +45,11 @@
 
 #ifndef KVC_SK_STAGES
 #define KVC_SK_STAGES 3
+#endif
+// Bytes of K/V that all CTAs together may prefetch into L2 before the dependency
+// wait (a part of the 126 MB L2, so the prefetched lines survive until they are read).
+#ifndef KVC_SK_PREFETCH_BYTES
+#define KVC_SK_PREFETCH_BYTES (48ll << 20)
 #endif
 
 namespace kvc {
@@ -136,6 +151,115 @@ struct TileCursor {
   }
 };
 
+// Stream-K ranges: CTA r streams the W tiles' range [r*W/G, (r+1)*W/G).
+struct RangeMap {
+  long long W;
+  int G;
+  __device__ __forceinline__ long long start(long long r) const { return r * W / G; }
+  __device__ __forceinline__ long long of(long long t) const {  // range holding tile t
+    return ((t + 1) * G - 1) / W;
+  }
+};
+
+// Merge the partial pieces rf..rl of one segment (the CTA's rows r0.., nr of them
+// valid, outputs from row_base) by log-sum-exp:
+//     out = sum_q 2^(lse_q - M) o_q / sum_q 2^(lse_q - M),   M = max_q lse_q.
+// Piece q lives in workspace slot 2*(rf+q) + 1 if it is the first piece and range rf
+// began before the segment (s0), else 2*(rf+q).  Each output quad (4 consecutive
+// elements of a row) is handled by tpq consecutive lanes (a power of two up to 8,
+// chosen so the CTA's threads cover the quads): lane `sub` of the group takes pieces
+// sub, sub + tpq, ..., issuing the lse and the float4 of four pieces before using
+// any, with a running maximum; the group then combines its lanes' (max, sum, acc)
+// with xor shuffles.  A merge is thus about one L2 round trip, not one per piece.
+template <typename T, int D, int R, int NTH>
+__device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const RangeMap& rm,
+                                                    long long rf, long long rl, long long s0,
+                                                    int nr, size_t row_base) {
+  constexpr int Q4 = D / 4;
+  const int tid = threadIdx.x;
+  const int npc = (int)(rl - rf + 1);
+  const bool rf_mid = rm.start(rf) < s0;
+  const int items = nr * Q4;
+  int tpq = 1;
+  while (tpq < 8 && tpq < npc && items * tpq * 2 <= NTH) tpq *= 2;
+  T* out = static_cast<T*>(p.out);
+#pragma unroll 1
+  for (int base = 0; base < items * tpq; base += NTH) {  // the same trip count in every thread
+    const int w = base + tid;
+    const bool act = w < items * tpq;
+    const int item = act ? w / tpq : 0;
+    const int sub = w & (tpq - 1);
+    const int rr = item / Q4;
+    const int d = (item - rr * Q4) * 4;
+    float m_run = -INFINITY, den = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int q0 = sub; act && q0 < npc; q0 += 4 * tpq) {
+      float ls[4];
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + u * tpq;
+        if (q < npc) {
+          const size_t slot = (size_t)(rf + q) * 2 + ((q == 0 && rf_mid) ? 1 : 0);
+          ls[u] = __ldcg(p.ws_lse + slot * R + rr);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (slot * R + rr) * D + d));
+        } else {
+          ls[u] = -INFINITY;
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mx = fmaxf(fmaxf(ls[0], ls[1]), fmaxf(ls[2], ls[3]));
+      const float m_new = fmaxf(m_run, mx);
+      if (m_new == -INFINITY) continue;  // nothing visible yet
+      const float f = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+      den *= f;
+      acc.x *= f;
+      acc.y *= f;
+      acc.z *= f;
+      acc.w *= f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float wq = ls[u] == -INFINITY ? 0.f : exp2f(ls[u] - m_new);
+        den += wq;
+        acc.x = fmaf(wq, v[u].x, acc.x);
+        acc.y = fmaf(wq, v[u].y, acc.y);
+        acc.z = fmaf(wq, v[u].z, acc.z);
+        acc.w = fmaf(wq, v[u].w, acc.w);
+      }
+      m_run = m_new;
+    }
+    // combine the group's lanes (consecutive lanes of one warp; every lane takes part)
+#pragma unroll 1
+    for (int off = 1; off < tpq; off <<= 1) {
+      const float m_o = __shfl_xor_sync(0xffffffffu, m_run, off);
+      const float den_o = __shfl_xor_sync(0xffffffffu, den, off);
+      float4 a_o;
+      a_o.x = __shfl_xor_sync(0xffffffffu, acc.x, off);
+      a_o.y = __shfl_xor_sync(0xffffffffu, acc.y, off);
+      a_o.z = __shfl_xor_sync(0xffffffffu, acc.z, off);
+      a_o.w = __shfl_xor_sync(0xffffffffu, acc.w, off);
+      const float m_new = fmaxf(m_run, m_o);
+      const float f1 = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+      const float f2 = m_o == -INFINITY ? 0.f : exp2f(m_o - m_new);
+      den = den * f1 + den_o * f2;
+      acc.x = acc.x * f1 + a_o.x * f2;
+      acc.y = acc.y * f1 + a_o.y * f2;
+      acc.z = acc.z * f1 + a_o.z * f2;
+      acc.w = acc.w * f1 + a_o.w * f2;
+      m_run = m_new;
+    }
+    if (act && sub == 0) {
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      T* o = out + (row_base + rr) * D + d;
+      store_elt<T>(o, acc.x * inv);
+      store_elt<T>(o + 1, acc.y * inv);
+      store_elt<T>(o + 2, acc.z * inv);
+      store_elt<T>(o + 3, acc.w * inv);
+    }
+  }
+}
+
 template <int D, int NT, typename T, bool PAGED>
 __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     attend_streamk_kernel(const AttendParams p, const __grid_constant__ CUtensorMap tmk,
@@ -163,23 +287,41 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
 
   // Programmatic dependent launch: the next grid in the stream may begin as
   // this one's CTAs retire.  Before griddep_wait() this kernel writes no global
-  // memory and reads seq_lens and the block table only to aim L2 prefetches,
-  // which change no result; the pass that counts runs after the wait.
+  // memory and reads seq_lens and the block table only to plan and to aim L2
+  // prefetches, which change no result; every read that counts comes after it.
   griddep_launch_dependents();
+
+  // CTA-local set-up (shared memory only): made visible by the first barrier of locate().
+  if (tid == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+#pragma unroll
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], W);
+    }
+    flags[0] = 0;
+    fence_barrier_init();
+  }
 
   // ------------------------------------ per-request tile prefix and this CTA's range
   int* P = reinterpret_cast<int*>(smem);  // [B + 1], in the ring before any copy
   long long Wt = 0, lo = 0;
   int G = 0, ntiles = 0;
   TileCursor<R> cur;
+  // this thread's requests in the scan, and a digest of the lengths it read there
+  const int per_thread = ceil_div(p.B, NTH);
+  const int b_lo = min(p.B, tid * per_thread), b_hi = min(p.B, b_lo + per_thread);
+  auto mix = [](uint32_t h, int L) { return (h ^ (uint32_t)L) * 0x9E3779B1u + 0x7F4A7C15u; };
+  uint32_t digest = 0;
   // Returns whether this CTA has tiles; ends with a barrier (P is then dead).
   auto locate = [&](bool authoritative) -> bool {
     {
-      const int per = ceil_div(p.B, NTH);
-      const int b_lo = min(p.B, tid * per), b_hi = min(p.B, b_lo + per);
       int sum = 0;
+      digest = 0;
       for (int b = b_lo; b < b_hi; ++b) {
         const int L = p.seq_lens[b];
+        digest = mix(digest, L);
         int t = 0;
         if (length_ok(p, L, PAGED)) t = request_tiles<R>(p, L);
         else if (authoritative) flag_error(p.err, KVC_ERR_BOUNDS);
@@ -245,100 +387,127 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     return work;
   };
 
-  // The TMA boxes of the tile under cursor pc: f(x, y, byte offset in the stage).
-  auto for_each_box = [&](const TileCursor<R>& pc, auto&& f) {
-    const int t0 = pc.k * C::kTile;
-    if (!PAGED) {
-      const int y = (pc.b * p.H_kv + pc.g) * p.max_T + t0;
-#pragma unroll
-      for (int h = 0; h < C::kHalves; ++h) f(h * 64, y, h * C::kBoxBytes);
-    } else {
-      const int Pg = 1 << p.page_shift;
-      const int box_rows = Pg < C::kTile ? Pg : C::kTile;
-      const int n_seg = pc.L + row_block(pc.rb, R, p.rows, p.T_new).imax + 1;
-      const int32_t* bt = p.block_table + (size_t)pc.b * p.max_pages;
-      const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
-#pragma unroll 1
-      for (int t = t0; t < t0 + C::kTile; t += box_rows) {
-        int y = beyond;
-        if (t < n_seg) {
-          const int page = bt[t >> p.page_shift];
-          if (page >= 0 && page < p.num_pages)
-            y = (page * p.H_kv + pc.g) * Pg + (t & (Pg - 1));
-          else
-            f(-1, 0, 0);  // a bad page id: reported by the caller
-        }
-        const int off = (t - t0) * 128;
-#pragma unroll
-        for (int h = 0; h < C::kHalves; ++h) f(h * 64, y, h * C::kBoxBytes + off);
-      }
-    }
+  // Paged tiles are loaded as boxes of min(page, 64) rows, one page lookup each.
+  const int Pg = PAGED ? (1 << p.page_shift) : C::kTile;
+  const int box_rows = Pg < C::kTile ? Pg : C::kTile;
+  const int nbox = C::kTile / box_rows;         // <= 8: pages of 8 or more tokens
+  const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
+  // Row of box `box` of the tile under cursor pc: -1 = the lookup is still to be done;
+  // returns `beyond` past the segment's last position.
+  auto box_page_row = [&](const TileCursor<R>& pc, int box, int page) -> int {
+    const int t = pc.k * C::kTile + box * box_rows;
+    if (t >= pc.L + row_block(pc.rb, R, p.rows, p.T_new).imax + 1) return beyond;
+    if (page < 0 || page >= p.num_pages) return -1;
+    return (page * p.H_kv + pc.g) * Pg + (t & (Pg - 1));
+  };
+  auto lookup_page = [&](const TileCursor<R>& pc, int box) -> int {
+    const int t = pc.k * C::kTile + box * box_rows;
+    if (pc.b >= p.B || box >= nbox ||
+        t >= pc.L + row_block(pc.rb, R, p.rows, p.T_new).imax + 1)
+      return 0;
+    return p.block_table[(size_t)pc.b * p.max_pages + (t >> p.page_shift)];
   };
 
-  // Speculative pass: warm L2 with this CTA's first tiles while the grid ahead
-  // finishes.  Lengths or pages that change before the wait only waste a prefetch.
-  if (locate(false) && tid == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
+  // Speculative pass: plan from the lengths as they stand and warm L2 with the
+  // first tiles of this CTA's range while the grid ahead finishes.  Lengths or
+  // pages that change before the wait only waste a prefetch.
+  const bool spec_work = locate(false);
+  const uint32_t spec_digest = digest;
+  const TileCursor<R> spec_cur = cur;
+  if (spec_work && warp == 0) {
     // only boxes wholly inside the tensor: the cursor may walk off stale lengths
-    const int rows_total = PAGED ? p.num_pages * p.H_kv << p.page_shift : p.B * p.H_kv * p.max_T;
-    const int box_h = PAGED ? min(1 << p.page_shift, C::kTile) : C::kTile;
+    const long long rows_total =
+        PAGED ? (long long)p.num_pages * p.H_kv * Pg : (long long)p.B * p.H_kv * p.max_T;
+    const long long budget = KVC_SK_PREFETCH_BYTES / ((long long)G * 2 * C::kTileBytes);
+    const int pf = (int)min((long long)ntiles, max((long long)C::kStages, budget));
     TileCursor<R> pc = cur;
-    for (int i = 0; i < min(C::kStages, ntiles) && pc.b < p.B; ++i) {
-      for_each_box(pc, [&](int x, int y, int) {
-        if (x < 0 || y < 0 || y + box_h > rows_total) return;
-        tma_prefetch_2d(&tmk, x, y);
-        tma_prefetch_2d(&tmv, x, y);
-      });
+#pragma unroll 1
+    for (int i = 0; i < pf && pc.b < p.B; ++i) {
+      if (!PAGED) {
+        const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
+        if (lane < C::kHalves && y + C::kTile <= rows_total) {
+          tma_prefetch_2d(&tmk, lane * 64, y);
+          tma_prefetch_2d(&tmv, lane * 64, y);
+        }
+      } else if (lane < nbox) {
+        const int y = box_page_row(pc, lane, lookup_page(pc, lane));
+        if (y >= 0 && y != beyond && y + box_rows <= rows_total)
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            tma_prefetch_2d(&tmk, h * 64, y);
+            tma_prefetch_2d(&tmv, h * 64, y);
+          }
+      }
       pc.next(p, PAGED);
     }
   }
   griddep_wait();
-  if (!locate(true)) return;
-
-  if (tid == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-#pragma unroll
-    for (int st = 0; st < C::kStages; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], W);
+  // The lengths now count: keep the speculative plan if none of them changed.
+  bool work;
+  {
+    uint32_t h = 0;
+    for (int b = b_lo; b < b_hi; ++b) {
+      const int L = p.seq_lens[b];
+      h = mix(h, L);
+      if (!length_ok(p, L, PAGED)) flag_error(p.err, KVC_ERR_BOUNDS);
     }
-    flags[0] = 0;
-    fence_barrier_init();
+    const bool same_first = !spec_work || p.seq_lens[spec_cur.b] == spec_cur.L;
+    if (__syncthreads_or(h != spec_digest || !same_first)) {
+      work = locate(true);
+    } else {
+      work = spec_work;
+      cur = spec_cur;
+    }
   }
-  __syncthreads();
+  if (!work) return;
 
   // ------------------------------------------------------- tile producer
-  const bool producer = (tid == 0);
+  // Warp 0 issues the copies (lane 0 the barrier and q; lane k box k).
+  const bool producer = (warp == 0) && !p.stall;
   const uint64_t pol = l2_policy_evict_first();
   TileCursor<R> pc = cur;  // producer's own cursor
   int issued = 0;
+  int page_ahead = PAGED && producer ? lookup_page(pc, lane) : 0;
   auto issue = [&]() {
     const int st = issued % C::kStages;
     const bool first = (issued == 0) || (pc.k == 0);
     const int r0 = pc.rb * R;
     const int nr = min(R, p.rows - r0);
     const uint32_t qbytes = first ? (uint32_t)nr * D * 2 : 0u;
-    mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes + qbytes);
-    if (first) {
-      const char* qsrc = static_cast<const char*>(p.q) +
-                         ((((size_t)pc.b * p.H_q + (size_t)pc.g * p.group) * p.T_new) + r0) *
-                             D * 2;
-      bulk_g2s(sq + st * R * D * 2, qsrc, qbytes, &full[st]);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes + qbytes);
+      if (first) {
+        const char* qsrc = static_cast<const char*>(p.q) +
+                           ((((size_t)pc.b * p.H_q + (size_t)pc.g * p.group) * p.T_new) + r0) *
+                               D * 2;
+        bulk_g2s(sq + st * R * D * 2, qsrc, qbytes, &full[st]);
+      }
     }
+    __syncwarp();
     unsigned char* dk = sk + st * C::kTileBytes;
     unsigned char* dv = sv + st * C::kTileBytes;
-    for_each_box(pc, [&](int x, int y, int off) {
-      if (x < 0) {
-        flag_error(p.err, KVC_ERR_BOUNDS);
-        return;
+    if (!PAGED) {
+      if (lane < C::kHalves) {
+        const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
+        tma_load_2d(dk + lane * C::kBoxBytes, &tmk, lane * 64, y, &full[st], pol);
+        tma_load_2d(dv + lane * C::kBoxBytes, &tmv, lane * 64, y, &full[st], pol);
       }
-      tma_load_2d(dk + off, &tmk, x, y, &full[st], pol);
-      tma_load_2d(dv + off, &tmv, x, y, &full[st], pol);
-    });
+    } else if (lane < nbox) {
+      int y = box_page_row(pc, lane, page_ahead);
+      if (y < 0) {  // a page id outside the pool: zero fill, reported
+        flag_error(p.err, KVC_ERR_BOUNDS);
+        y = beyond;
+      }
+      const int off = lane * box_rows * 128;
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h) {
+        tma_load_2d(dk + h * C::kBoxBytes + off, &tmk, h * 64, y, &full[st], pol);
+        tma_load_2d(dv + h * C::kBoxBytes + off, &tmv, h * 64, y, &full[st], pol);
+      }
+    }
     ++issued;
     pc.next(p, PAGED);
+    if (PAGED) page_ahead = lookup_page(pc, lane);  // consumed by the next issue
   };
   if (producer)
     while (issued < min(C::kStages, ntiles)) issue();
@@ -348,6 +517,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
   // return at once; the CTA finishes its loop (on garbage) instead of
   // stranding threads at a named barrier.
   volatile int* abort_word = flags;
+  const unsigned long long wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (*abort_word) return false;
 #pragma unroll 1
@@ -358,7 +528,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     while (true) {
       if (mbar_try_wait(bar, parity)) return true;
       if (*abort_word) return false;
-      if (global_timer_ns() - t_start > kWaitLimitNs) {
+      if (global_timer_ns() - t_start > wait_limit) {
         flag_error(p.err, KVC_ERR_TIMEOUT);
         *abort_word = 1;
         return false;
@@ -386,8 +556,9 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
   for (int j = 0; j < ntiles; ++j) {
     const int st = j % C::kStages;
     if (producer && j >= 1 && issued < ntiles) {
-      wait(&empty[(j - 1) % C::kStages], ((j - 1) / C::kStages) & 1);
-      issue();
+      bool ready = true;
+      if (lane == 0) ready = wait(&empty[(j - 1) % C::kStages], ((j - 1) / C::kStages) & 1);
+      if (__shfl_sync(0xffffffffu, ready, 0)) issue();
     }
     wait(&full[st], (j / C::kStages) & 1);
 
@@ -648,8 +819,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
       }
       named_barrier_sync(1, NTH);
       if (flags[1]) {
-        merge_pieces<T, D, R, NTH>(p, rm, rf, rl, s0, nr, row_base, red_acc, red_acc_hi,
-                                   C::kTileBytes / 4, [] { named_barrier_sync(1, NTH); });
+        merge_pieces_spread<T, D, R, NTH>(p, rm, rf, rl, s0, nr, row_base);
         if (tid == 0) *ticket = 0;
       }
     }
@@ -658,10 +828,10 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     cur.next(p, PAGED);
   }
   // After an abort, do not retire while copies may still be landing.
-  if (producer && *abort_word)
+  if (producer && lane == 0 && *abort_word)
 #pragma unroll 1
     for (int j = max(0, issued - C::kStages); j < issued; ++j)
-      if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.err)) break;
+      if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.err, wait_limit)) break;
 }
 
 }  // namespace kvc

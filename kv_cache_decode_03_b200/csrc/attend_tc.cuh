@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
   const uint32_t tO = tmem + C::kOCol;
 
   volatile int* abort_word = flags;
+  const unsigned long long wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (*abort_word) return false;
 #pragma unroll 1
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     while (true) {
       if (mbar_try_wait(bar, parity)) return true;
       if (*abort_word) return false;
-      if (global_timer_ns() - t_start > kWaitLimitNs) {
+      if (global_timer_ns() - t_start > wait_limit) {
         flag_error(p.err, KVC_ERR_TIMEOUT);
         *abort_word = 1;
         return false;
@@ -351,7 +352,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     const uint64_t pol = p.row_blocks > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
     if (lane_id == 0) prefetch_tmap(tm);
 #pragma unroll 1
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; j < ntiles && !p.stall; ++j) {  // a stall (test) issues nothing
       const int st = j % NS;
       if (j >= NS) {
         bool w = true;
@@ -541,11 +542,11 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
       const int NS = warp == C::kKWarp ? SK : SV;
       uint64_t* full = warp == C::kKWarp ? k_full : v_full;
       for (int j = max(0, issued - NS); j < issued; ++j)
-        if (!mbar_wait(&full[j % NS], (j / NS) & 1, p.err)) break;
+        if (!mbar_wait(&full[j % NS], (j / NS) & 1, p.err, wait_limit)) break;
     }
     if (warp == C::kMmaWarp && lane_id == 0 && mma_issued) {  // MMAs still in flight
       umma_commit(dbar);
-      mbar_wait(dbar, 0, p.err);
+      mbar_wait(dbar, 0, p.err, wait_limit);
     }
     tc_fence_before();
     __syncthreads();

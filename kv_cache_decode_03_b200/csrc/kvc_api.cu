@@ -41,6 +41,9 @@ struct kvc_cache {
   std::vector<CUtensorMap> tmv;
   int device;
   int num_sms;
+  bool dependent_launch;           // stream-K launches with programmatic stream serialization
+  unsigned long long wait_limit_ns;  // bound of the kernels' pipeline waits (0: 1 s)
+  bool stall_next;                 // failure-detection test: next attend issues no copies
 };
 
 namespace {
@@ -564,8 +567,9 @@ static bool dependent_launch_enabled() {
 }
 
 template <int D, int NT, typename T, bool PAGED>
-kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, cudaStream_t stream) {
+kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, bool pdl,
+                                 const CUtensorMap& tk, const CUtensorMap& tv,
+                                 cudaStream_t stream) {
   using C = kvc::StreamKCfg<D>;
   streamk_occupancy<D, NT, T, PAGED>();  // sets the shared-memory attribute once
   const size_t smem = C::template smem_bytes<NT>();
@@ -581,26 +585,27 @@ kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, const CUt
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = dependent_launch_enabled() ? 1 : 0;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cuda_status(
       cudaLaunchKernelEx(&cfg, kvc::attend_streamk_kernel<D, NT, T, PAGED>, p, tk, tv));
 }
 
 template <typename T>
 kvc_status dispatch_streamk(const kvc::AttendParams& p, int D, int NT, bool paged, int grid,
-                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+                            bool pdl, const CUtensorMap& tk, const CUtensorMap& tv,
+                            cudaStream_t s) {
   if (D == 64) {
     if (paged)
-      return NT == 1 ? launch_attend_streamk<64, 1, T, true>(p, grid, tk, tv, s)
-                     : launch_attend_streamk<64, 2, T, true>(p, grid, tk, tv, s);
-    return NT == 1 ? launch_attend_streamk<64, 1, T, false>(p, grid, tk, tv, s)
-                   : launch_attend_streamk<64, 2, T, false>(p, grid, tk, tv, s);
+      return NT == 1 ? launch_attend_streamk<64, 1, T, true>(p, grid, pdl, tk, tv, s)
+                     : launch_attend_streamk<64, 2, T, true>(p, grid, pdl, tk, tv, s);
+    return NT == 1 ? launch_attend_streamk<64, 1, T, false>(p, grid, pdl, tk, tv, s)
+                   : launch_attend_streamk<64, 2, T, false>(p, grid, pdl, tk, tv, s);
   }
   if (paged)
-    return NT == 1 ? launch_attend_streamk<128, 1, T, true>(p, grid, tk, tv, s)
-                   : launch_attend_streamk<128, 2, T, true>(p, grid, tk, tv, s);
-  return NT == 1 ? launch_attend_streamk<128, 1, T, false>(p, grid, tk, tv, s)
-                 : launch_attend_streamk<128, 2, T, false>(p, grid, tk, tv, s);
+    return NT == 1 ? launch_attend_streamk<128, 1, T, true>(p, grid, pdl, tk, tv, s)
+                   : launch_attend_streamk<128, 2, T, true>(p, grid, pdl, tk, tv, s);
+  return NT == 1 ? launch_attend_streamk<128, 1, T, false>(p, grid, pdl, tk, tv, s)
+                 : launch_attend_streamk<128, 2, T, false>(p, grid, pdl, tk, tv, s);
 }
 
 template <int D, int R, typename T, bool PAGED>
@@ -681,6 +686,47 @@ float* scale_pool(const kvc_cache* c, int layer, int which) {
   return c->scales + (size_t)(2 * layer + which) * c->scale_floats;
 }
 
+// The parameter block of an attend call on layer `layer` (no workspace yet).  A pending
+// stall (kvc_inject_stall) is taken by this call.
+kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q, int T_new,
+                                const int32_t* block_table, int max_pages,
+                                const int32_t* seq_lens, float scale, void* out,
+                                const Plan& pl) {
+  kvc::AttendParams p{};
+  p.k_pool = c->pool + (size_t)(2 * layer) * c->layer_bytes;
+  p.v_pool = c->pool + (size_t)(2 * layer + 1) * c->layer_bytes;
+  p.q = q;
+  p.out = out;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.max_pages = max_pages;
+  p.B = c->B;
+  p.H_q = H_q;
+  p.H_kv = c->H_kv;
+  p.T_new = T_new;
+  p.group = H_q / c->H_kv;
+  p.rows = p.group * T_new;
+  p.max_T = c->max_T;
+  p.page_shift = c->page_shift;
+  p.num_pages = c->num_pages;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.split_tokens = pl.split_tokens;
+  p.num_splits = pl.num_splits;
+  p.row_blocks = pl.row_blocks;
+  p.err = c->d_err;
+  p.wait_limit_ns = c->wait_limit_ns;
+  p.stall = c->stall_next ? 1 : 0;
+  c->stall_next = false;
+  return p;
+}
+
+// Where a plan's partial results start in a workspace of partial outputs then lse.
+float* lse_base(const kvc_cache* c, const Plan& pl, float* ws, int H_q, int T_new) {
+  if (!ws) return nullptr;
+  return pl.streamk ? ws + pl.slots * pl.R * c->D
+                    : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
+}
+
 // Launch the attend kernel a plan chose for layer `layer`.
 kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::AttendParams& p,
                     cudaStream_t s) {
@@ -698,9 +744,10 @@ kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::At
               : dispatch_tc<__half>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s);
   if (pl.streamk)
     return bf ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
-                                                c->tmk[layer], c->tmv[layer], s)
-              : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
-                                         c->tmv[layer], s);
+                                                c->dependent_launch, c->tmk[layer],
+                                                c->tmv[layer], s)
+              : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid,
+                                         c->dependent_launch, c->tmk[layer], c->tmv[layer], s);
   if (pl.mma)
     return bf ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
                                             c->tmv[layer], s)
@@ -787,6 +834,9 @@ static kvc_status create_cache(int B, int H_kv, int D, int max_T, kvc_dtype dtyp
                         : 0;
   c->device = dev;
   c->num_sms = sms;
+  c->dependent_launch = dependent_launch_enabled();
+  c->wait_limit_ns = 0;
+  c->stall_next = false;
   void* pool = nullptr;
   if (cudaMalloc(&pool, 2 * layer_bytes * (size_t)num_layers) != cudaSuccess) {
     cudaGetLastError();
@@ -1038,35 +1088,13 @@ kvc_status kvc_attend_window(kvc_cache* c, int layer, const void* q, int H_q, in
   const Plan pl = make_plan(c, H_q, T_new, max_pages, window, sink);
   kvc_status st = ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
   if (st != KVC_OK) return st;
-  kvc::AttendParams p{};
-  p.k_pool = kvc_k_pool(c, layer);
-  p.v_pool = kvc_v_pool(c, layer);
-  p.q = q;
-  p.out = out;
-  p.seq_lens = seq_lens;
-  p.block_table = block_table;
-  p.max_pages = max_pages;
-  p.B = c->B;
-  p.H_q = H_q;
-  p.H_kv = c->H_kv;
-  p.T_new = T_new;
-  p.group = H_q / c->H_kv;
-  p.rows = p.group * T_new;
-  p.max_T = c->max_T;
-  p.page_shift = c->page_shift;
-  p.num_pages = c->num_pages;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  kvc::AttendParams p =
+      attend_params(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, out, pl);
   p.window = window;
   p.sink = sink;
-  p.split_tokens = pl.split_tokens;
-  p.num_splits = pl.num_splits;
-  p.row_blocks = pl.row_blocks;
   p.ws_o = c->ws;
-  p.ws_lse = !c->ws ? nullptr
-             : pl.streamk ? c->ws + pl.slots * pl.R * c->D
-                          : c->ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
+  p.ws_lse = lse_base(c, pl, c->ws, H_q, T_new);
   p.counters = c->tickets;
-  p.err = c->d_err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return run_plan(c, layer, pl, p, s);
 }
@@ -1093,6 +1121,24 @@ kvc_status kvc_get_error(kvc_cache* c) {
     if (cudaDeviceSynchronize() != cudaSuccess) return KVC_ERR_CUDA;
   }
   return static_cast<kvc_status>(h);
+}
+
+kvc_status kvc_set_dependent_launch(kvc_cache* c, int on) {
+  if (!c) return KVC_ERR_INVALID_ARG;
+  c->dependent_launch = on != 0;
+  return KVC_OK;
+}
+
+kvc_status kvc_set_wait_limit(kvc_cache* c, unsigned long long ns) {
+  if (!c) return KVC_ERR_INVALID_ARG;
+  c->wait_limit_ns = ns;
+  return KVC_OK;
+}
+
+kvc_status kvc_inject_stall(kvc_cache* c) {
+  if (!c) return KVC_ERR_INVALID_ARG;
+  c->stall_next = true;
+  return KVC_OK;
 }
 
 }  // extern "C"
@@ -1149,6 +1195,12 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
     return KVC_ERR_INVALID_ARG;
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
   if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KVC_ERR_CUDA;
+  }
+  if (dev != c->device) return KVC_ERR_INVALID_ARG;  // the scratch must be on the cache's GPU
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
   // [tickets, padded to 256 bytes][partial outputs][lse]
   const size_t ticket_bytes = (pl.ws_counters * sizeof(int) + 255) & ~size_t(255);
@@ -1162,32 +1214,11 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
       cudaMemsetAsync(base, 0, pl.ws_counters * sizeof(int), s) != cudaSuccess)
     return cuda_status(cudaGetLastError());
   float* ws = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + ticket_bytes);
-  kvc::AttendParams p{};
-  p.k_pool = kvc_k_pool(c, layer);
-  p.v_pool = kvc_v_pool(c, layer);
-  p.q = q;
-  p.out = out;
-  p.seq_lens = seq_lens;
-  p.block_table = block_table;
-  p.max_pages = max_pages;
-  p.B = c->B;
-  p.H_q = H_q;
-  p.H_kv = c->H_kv;
-  p.T_new = T_new;
-  p.group = H_q / c->H_kv;
-  p.rows = p.group * T_new;
-  p.max_T = c->max_T;
-  p.page_shift = c->page_shift;
-  p.num_pages = c->num_pages;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.split_tokens = pl.split_tokens;
-  p.num_splits = pl.num_splits;
-  p.row_blocks = pl.row_blocks;
+  kvc::AttendParams p =
+      attend_params(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, out, pl);
   p.ws_o = ws;
-  p.ws_lse = pl.streamk ? ws + pl.slots * pl.R * c->D
-                        : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
+  p.ws_lse = lse_base(c, pl, ws, H_q, T_new);
   p.counters = static_cast<int*>(base);
-  p.err = c->d_err;
   return run_plan(c, layer, pl, p, s);
 }
 
@@ -1221,37 +1252,18 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   }
   kvc_status st = ensure_workspace(c, pl.ws_bytes, pl.ws_counters);
   if (st != KVC_OK) return st;
-  kvc::AttendParams p{};
-  p.k_pool = kvc_k_pool(c, layer);
-  p.v_pool = kvc_v_pool(c, layer);
-  p.q = q;
-  p.out = out;
-  p.seq_lens = seq_lens;
-  p.block_table = block_table;
-  p.max_pages = max_pages;
-  p.B = c->B;
-  p.H_q = H_q;
-  p.H_kv = c->H_kv;
-  p.T_new = T_new;
-  p.group = H_q / c->H_kv;
-  p.rows = p.group * T_new;
-  p.max_T = c->max_T;
-  p.page_shift = c->page_shift;
-  p.num_pages = c->num_pages;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.split_tokens = pl.split_tokens;
-  p.num_splits = pl.num_splits;
-  p.row_blocks = pl.row_blocks;
+  kvc::AttendParams p =
+      attend_params(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, out, pl);
   p.ws_o = c->ws;
-  p.ws_lse = c->ws + pl.slots * pl.R * c->D;
+  p.ws_lse = lse_base(c, pl, c->ws, H_q, T_new);
   p.counters = c->tickets;
   p.k_new = k_new;
   p.v_new = v_new;
-  p.err = c->d_err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return c->dtype == KVC_BF16
-             ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
+             ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
+                                               c->dependent_launch, c->tmk[layer],
                                                c->tmv[layer], s)
-             : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->tmk[layer],
-                                        c->tmv[layer], s);
+             : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->dependent_launch,
+                                        c->tmk[layer], c->tmv[layer], s);
 }

@@ -45,6 +45,9 @@ struct AttendParams {
   const void* k_new;  // fused append (stream-K kernel): (B, H_kv, T_new, D), else null
   const void* v_new;
   int* err;
+  unsigned long long wait_limit_ns;  // bound of every pipeline wait (0: the default, 1 s)
+  int stall;  // failure-detection test: the producers issue no copies, so the first
+              // wait runs out (stream-K and tcgen05 kernels)
 };
 
 }  // namespace kvc

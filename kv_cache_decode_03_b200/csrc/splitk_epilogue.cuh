@@ -140,115 +140,4 @@ __device__ __forceinline__ void finish_slice(const AttendParams& p, const float*
   if (tid == 0) *ticket = 0;  // ready for the next launch
 }
 
-// Stream-K ranges: CTA r streams the W tiles' range [r*W/G, (r+1)*W/G).
-struct RangeMap {
-  long long W;
-  int G;
-  __device__ __forceinline__ long long start(long long r) const { return r * W / G; }
-  __device__ __forceinline__ long long of(long long t) const {  // range holding tile t
-    return ((t + 1) * G - 1) / W;
-  }
-};
-
-// Merge the partial pieces rf..rl of one segment (the CTA's rows r0.., nr of them
-// valid, outputs from row_base) by log-sum-exp.  Piece q lives in workspace slot
-// 2*(rf+q) + 1 if it is the first piece and range rf began before the segment
-// (s0), else 2*(rf+q).  The (row, piece) weights are built once in shared memory
-// (`lo` then `hi`, `half` floats each); then every thread owns 4 consecutive
-// outputs of a row and issues the float4 loads of four pieces at a time before
-// accumulating, so a merge costs a few L2 round trips, not one per element.
-// `sync` is a barrier of the NTH participating threads.
-template <typename T, int D, int R, int NTH, typename Sync>
-__device__ __forceinline__ void merge_pieces(const AttendParams& p, const RangeMap& rm,
-                                             long long rf, long long rl, long long s0, int nr,
-                                             size_t row_base, float* lo, float* hi, int half,
-                                             Sync&& sync) {
-  const int tid = threadIdx.x;
-  const int npc = (int)(rl - rf + 1);
-  const bool rf_mid = rm.start(rf) < s0;
-  auto slot_of = [&](int q) -> size_t {
-    return (size_t)(rf + q) * 2 + ((q == 0 && rf_mid) ? 1 : 0);
-  };
-  auto w_at = [&](int rr, int q) -> float* {
-    const int i = rr * npc + q;
-    return i < half ? lo + i : hi + (i - half);
-  };
-  T* out = static_cast<T*>(p.out);
-  constexpr int Q4 = D / 4;
-  if (R * npc <= 2 * half) {
-#pragma unroll 1
-    for (int idx = tid; idx < R * npc; idx += NTH) {
-      const int rr = idx / npc;
-      const int q = idx - rr * npc;
-      *w_at(rr, q) = rr < nr ? __ldcg(p.ws_lse + slot_of(q) * R + rr) : -INFINITY;
-    }
-    sync();
-    if (tid < nr) {
-      float M = -INFINITY;
-      for (int q = 0; q < npc; ++q) M = fmaxf(M, *w_at(tid, q));
-      float den = 0.f;
-      for (int q = 0; q < npc; ++q) {
-        float* w = w_at(tid, q);
-        *w = (*w == -INFINITY) ? 0.f : exp2f(*w - M);
-        den += *w;
-      }
-      const float inv = 1.f / den;
-      for (int q = 0; q < npc; ++q) *w_at(tid, q) *= inv;
-    }
-    sync();
-#pragma unroll 1
-    for (int it = tid; it < nr * Q4; it += NTH) {
-      const int rr = it / Q4;
-      const int d = (it - rr * Q4) * 4;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      int q = 0;
-#pragma unroll 1
-      for (; q + 4 <= npc; q += 4) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          v[u] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (slot_of(q + u) * R + rr) * D + d));
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float w = *w_at(rr, q + u);
-          a.x = fmaf(w, v[u].x, a.x);
-          a.y = fmaf(w, v[u].y, a.y);
-          a.z = fmaf(w, v[u].z, a.z);
-          a.w = fmaf(w, v[u].w, a.w);
-        }
-      }
-      for (; q < npc; ++q) {
-        const float4 v =
-            __ldcg(reinterpret_cast<const float4*>(p.ws_o + (slot_of(q) * R + rr) * D + d));
-        const float w = *w_at(rr, q);
-        a.x = fmaf(w, v.x, a.x);
-        a.y = fmaf(w, v.y, a.y);
-        a.z = fmaf(w, v.z, a.z);
-        a.w = fmaf(w, v.w, a.w);
-      }
-      T* o = out + (row_base + rr) * D + d;
-      store_elt<T>(o, a.x);
-      store_elt<T>(o + 1, a.y);
-      store_elt<T>(o + 2, a.z);
-      store_elt<T>(o + 3, a.w);
-    }
-  } else {  // more (row, piece) weights than the buffers hold: two passes per output
-#pragma unroll 1
-    for (int idx = tid; idx < nr * D; idx += NTH) {
-      const int rr = idx / D;
-      const int d = idx - rr * D;
-      float M = -INFINITY;
-      for (int q = 0; q < npc; ++q) M = fmaxf(M, __ldcg(p.ws_lse + slot_of(q) * R + rr));
-      float den = 0.f, ov = 0.f;
-      for (int q = 0; q < npc; ++q) {
-        const float ls = __ldcg(p.ws_lse + slot_of(q) * R + rr);
-        const float w = (ls == -INFINITY) ? 0.f : exp2f(ls - M);
-        den += w;
-        ov = fmaf(w, __ldcg(p.ws_o + (slot_of(q) * R + rr) * D + d), ov);
-      }
-      store_elt<T>(out + (row_base + rr) * D + d, ov / den);
-    }
-  }
-}
-
 }  // namespace kvc
