@@ -326,25 +326,28 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, ms_per_step_max: float) 
     return world * bytes_per_rank_step / (ms_per_step_max * 1e-3) / 1e9
 
 
-def run_kvc(args, case: W.Case) -> None:
+class Measured(dict):
+    pass
+
+
+def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
+            reps: "Replicas", pdl_ab: bool = False, e2e: bool = False, clocks: bool = False):
+    """Time one workload: a CUDA graph of one step (every layer), K replays between CUDA
+    events (max over ranks); the same step eagerly; optionally the step with the
+    dependent launch off; the median duration of `samples` event-bracketed calls of
+    the step's kernel; and optionally the end-to-end step from pinned host buffers."""
     import torch
     import kv_cache_decode_03_b200 as kvc
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    reps = Replicas("nccl", torch.device("cuda", local))
-    world, rank = reps.world, reps.rank
-    barrier, max_over_ranks = reps.barrier, reps.max_over_ranks
-
     c = case
-    fp8 = args.kv_format == "fp8"
+    fp8 = kv_format == "fp8"
     tdt = {"fp16": torch.float16, "bf16": torch.bfloat16}[c.dtype]
     cache = kvc.KVCache(c.B, c.H_kv, c.D, c.max_T, c.dtype, c.page_size, c.layers,
-                        c.num_pages, kv_format=args.kv_format)
+                        c.num_pages, kv_format=kv_format)
     bt = torch.from_numpy(c.block_table).cuda() if c.paged else None
     max_pages = c.max_pages if c.paged else 0
     gen = torch.Generator(device="cuda")
-    gen.manual_seed(c.seed * 1000 + rank)
+    gen.manual_seed(c.seed * 1000 + reps.rank)
     for layer in range(c.layers):
         for which in ("k", "v"):
             pool = cache.pool(layer, which)
@@ -365,132 +368,215 @@ def run_kvc(args, case: W.Case) -> None:
     ns, split_tokens = cache.plan(c.H_q, c.T_new, max_pages)
     stream = torch.cuda.Stream()
     scale = c.scale
+    fused = split_tokens == 0 and not fp8  # kvc_append_attend is one launch
 
     def step(q=qs, k=ks, v=vs, o=outs):
         for layer in range(c.layers):
             cache.append_attend(layer, k[layer], v[layer], q[layer], seq, bt, scale=scale,
                                 out=o[layer], stream=stream)
 
-    # one launch per layer on the persistent path (append, attend and merge fused)
-    launches_per_step = c.layers * (1 if split_tokens == 0 else 2)
+    def capture():
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, warmup)):
+                step()
+            stream.synchronize()
+            if cache.get_error() != kvc.KVC_OK:
+                raise RuntimeError("device error during warm-up")
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step()
+            for _ in range(3):
+                g.replay()
+            stream.synchronize()
+        return g
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
-            step()
-        stream.synchronize()
-        if cache.get_error() != kvc.KVC_OK:
-            raise RuntimeError("device error during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-        # one step captured in a CUDA graph: the decode loop replays it
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            step()
-        for _ in range(3):
-            graph.replay()
-        stream.synchronize()
+    def time_graph(g, n, sampler=None):
+        reps.barrier()
+        torch.cuda.synchronize()
+        ctx = sampler if sampler is not None else _Null()
+        with ctx:
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(n):
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+        torch.cuda.synchronize()
+        reps.barrier()
+        return reps.max_over_ranks(e0.elapsed_time(e1) / n)
 
     # ---- timed region: K graph replays, device time by CUDA events
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.steps):
-                graph.replay()
-            e1.record(stream)
-        e1.synchronize()
-    torch.cuda.synchronize()
-    barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms)
-    clocks = clk.summary()
+    graph = capture()
+    clk = ClockSampler(torch.cuda.current_device()) if clocks else None
+    ms = time_graph(graph, steps, clk)
+    res = Measured(ms=ms, clocks=clk.summary() if clk else None)
 
     # ---- eager (no graph) step time, for reference
+    n_eager = max(3, steps // 4)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(max(3, args.steps // 4)):
+        for _ in range(n_eager):
             step()
         e1.record(stream)
     e1.synchronize()
-    ms_eager = e0.elapsed_time(e1) / max(3, args.steps // 4)
+    res["ms_eager"] = e0.elapsed_time(e1) / n_eager
 
-    # ---- per-launch duration of the step's kernel (kvc_append_attend) for the roofline
+    # ---- the same step with the dependent launch off (plain launches)
+    if pdl_ab and fused:
+        cache.set_dependent_launch(False)
+        g_plain = capture()
+        res["ms_no_dependent_launch"] = time_graph(g_plain, steps)
+        g_plain.reset()
+        del g_plain
+        cache.set_dependent_launch(True)
+
+    # ---- per-call duration of the step's kernel(s): median of `samples` bracketed calls
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(c.layers)]
     durs = []
     with torch.cuda.stream(stream):
-        for _ in range(max(2, args.steps // 10)):
+        while len(durs) < samples:
             for layer in range(c.layers):
                 evs[layer][0].record(stream)
-                cache.append_attend(layer, ks[layer], vs[layer], qs[layer], seq, bt, scale=scale,
-                                    out=outs[layer], stream=stream)
+                cache.append_attend(layer, ks[layer], vs[layer], qs[layer], seq, bt,
+                                    scale=scale, out=outs[layer], stream=stream)
                 evs[layer][1].record(stream)
             stream.synchronize()
             durs += [a.elapsed_time(b) for a, b in evs]
-    attend_ms = statistics.mean(durs)
+    res["call_ms_median"] = statistics.median(durs)
+    res["call_samples"] = len(durs)
     if cache.get_error() != kvc.KVC_OK:
         raise RuntimeError("device error in the timed region")
 
     # ---- e2e: pinned host buffers, copies inside the timed region
-    hq = qs.cpu().pin_memory()
-    hk = ks.cpu().pin_memory()
-    hv = vs.cpu().pin_memory()
-    ho = torch.empty(outs.shape, dtype=tdt).pin_memory()
-    dq, dk, dv = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
-    e2e_steps = max(3, args.steps // 4)
-    barrier()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            step(dq, dk, dv, outs)
-            ho.copy_(outs, non_blocking=True)
-        e1.record(stream)
-    e1.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-    h2d = (hq.numel() + hk.numel() + hv.numel()) * c.elt
-    d2h = ho.numel() * c.elt
+    if e2e:
+        hq = qs.cpu().pin_memory()
+        hk = ks.cpu().pin_memory()
+        hv = vs.cpu().pin_memory()
+        ho = torch.empty(outs.shape, dtype=tdt).pin_memory()
+        dq, dk, dv = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
+        e2e_steps = max(3, steps // 4)
+        reps.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                dq.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                step(dq, dk, dv, outs)
+                ho.copy_(outs, non_blocking=True)
+            e1.record(stream)
+        e1.synchronize()
+        reps.barrier()
+        res["e2e_ms"] = reps.max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+        res["h2d"] = (hq.numel() + hk.numel() + hv.numel()) * c.elt
+        res["d2h"] = ho.numel() * c.elt
+    graph.reset()
+    del graph
+    cache.close()
 
+    # ---- derived figures
     layer_bytes = fp8_algorithmic_bytes(c) if fp8 else c.algorithmic_bytes()
-    step_bytes = c.layers * layer_bytes
-    value = whole_job_gbs(world, step_bytes, ms)
+    res["layer_bytes"] = layer_bytes
+    res["step_bytes"] = c.layers * layer_bytes
+    res["launches_per_step"] = c.layers * (1 if fused else 2)
+    res["ns"], res["split_tokens"] = ns, split_tokens
     # one call's bytes: K/V read + q read + out written + k_new/v_new read + rows written
     # (the FP8 count already holds both sides of the append)
-    attend_bytes = layer_bytes + (0 if fp8 else 2 * c.B * c.H_kv * c.T_new * c.D * c.elt)
-    achieved = attend_bytes / (attend_ms * 1e-3) / 1e9
-    peak, peak_kind = peaks()
-    tok_layer_step = world * c.B * c.T_new / (ms * 1e-3 / c.layers)
-    kernel = attend_kernel_name(c, args.kv_format, split_tokens)
-    rows = (c.H_q // c.H_kv) * c.T_new
+    call_bytes = layer_bytes + (0 if fp8 else 2 * c.B * c.H_kv * c.T_new * c.D * c.elt)
+    res["call_bytes"] = call_bytes
+    kernel = attend_kernel_name(c, kv_format, split_tokens)
     # attention flops of one call: 4 per (query row, visible position, dimension); new row
     # i of request b sees L_b + i + 1 positions
     seen = float(sum(int(L) * c.T_new + c.T_new * (c.T_new + 1) // 2 for L in c.seq_lens))
     flops = 4.0 * seen * c.H_q * c.D
+    call_s = res["call_ms_median"] * 1e-3
+    step_call_s = ms * 1e-3 / c.layers  # one layer-step's share of the graph-timed step
+    peak, peak_kind = peaks()
     if kernel.startswith("attend_tc_kernel"):
         tpeak, tpeak_kind = tensor_peak()
-        achieved_tf = flops / (attend_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tpeak,
-                    "unit": "TFLOP/s", "frac": achieved_tf / tpeak, "traffic": None,
-                    "peak_source": tpeak_kind}
+        roof = {"bound": "tensor", "achieved": flops / call_s / 1e12, "peak": tpeak,
+                "unit": "TFLOP/s", "traffic": None, "peak_source": tpeak_kind,
+                "achieved_in_step": flops / step_call_s / 1e12}
     else:
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "traffic": profiled_traffic(kernel),
-                    "peak_source": peak_kind}
-    roofline["kernel"] = (kernel + (", fused: one launch per kvc_append_attend call (append, "
-                                    "split attend, merge)" if split_tokens == 0 else
-                                    ", after the append kernel"))
+        roof = {"bound": "hbm", "achieved": call_bytes / call_s / 1e9, "peak": peak,
+                "unit": "GB/s", "traffic": profiled_traffic(kernel), "peak_source": peak_kind,
+                "achieved_in_step": call_bytes / step_call_s / 1e9}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["frac_in_step"] = roof["achieved_in_step"] / roof["peak"]
+    roof["kernel"] = (kernel + (", fused: one launch per kvc_append_attend call (append, "
+                                "split attend, merge)" if fused else ", after the append kernel"))
+    roof["duration"] = (f"median of {len(durs)} event-bracketed kvc_append_attend calls "
+                        f"({res['call_ms_median'] * 1e3:.2f} us; each call alone, so without "
+                        f"the overlap of the dependent launch); achieved_in_step = the "
+                        f"graph-timed step / {c.layers} calls")
+    res["roofline"] = roof
+    res["kernel"] = kernel
+    res["tflops_call"] = flops / call_s / 1e12
+    res["tflops_step"] = flops / step_call_s / 1e12
+    res["peak"] = peak
+    return res
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def workload_summary(name: str, case: W.Case, kv_format: str, r: Measured, world: int) -> dict:
+    value = whole_job_gbs(world, r["step_bytes"], r["ms"])
+    d = {"workload": case.name, "kv_format": kv_format, "layers": case.layers,
+         "value_gbs": value, "pct_of_peak": 100.0 * value / world / r["peak"],
+         "ms_per_step": r["ms"], "ms_per_step_eager": r["ms_eager"],
+         "tokens_per_s_per_layer_step": world * case.B * case.T_new / (r["ms"] * 1e-3 / case.layers),
+         "attention_tflops_step": r["tflops_step"],
+         "call_us_median": r["call_ms_median"] * 1e3, "call_samples": r["call_samples"],
+         "frac": r["roofline"]["frac"], "frac_in_step": r["roofline"]["frac_in_step"],
+         "bound": r["roofline"]["bound"], "kernel": r["kernel"],
+         "split_k": {"num_splits": r["ns"], "split_tokens": r["split_tokens"]}}
+    if "ms_no_dependent_launch" in r:
+        d["ms_per_step_no_dependent_launch"] = r["ms_no_dependent_launch"]
+    return d
+
+
+def run_kvc(args, case: W.Case) -> None:
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    reps = Replicas("nccl", torch.device("cuda", local))
+    world, rank = reps.world, reps.rank
+    c = case
+    fp8 = args.kv_format == "fp8"
+    r = measure(c, args.kv_format, args.steps, args.warmup, args.launch_samples, reps,
+                pdl_ab=True, e2e=True, clocks=True)
+    ms = r["ms"]
+    value = whole_job_gbs(world, r["step_bytes"], ms)
+    peak = r["peak"]
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         cpu = cpu_baseline(c)
 
-    graph.reset()
-    del graph
-    cache.close()
+    # every other named configuration, bounded, on one GPU (the scaling runs time the
+    # headline only)
+    extra = {}
+    if world == 1 and args.workloads == "all":
+        for name, kvf in EXTRA_WORKLOADS:
+            if name == args.workload and kvf == args.kv_format:
+                continue
+            wc = sized_case(name, 0)
+            torch.cuda.empty_cache()
+            wr = measure(wc, kvf, max(5, min(args.steps, 10)), 3, args.launch_samples, reps,
+                         pdl_ab=(name.startswith("mha")))
+            key = name + ("_fp8" if kvf == "fp8" else "")
+            extra[key] = workload_summary(name, wc, kvf, wr, world)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -505,21 +591,23 @@ def run_kvc(args, case: W.Case) -> None:
                        "cache": (f"paged P{c.page_size}" if c.paged else "contiguous") +
                                 (", FP8 E4M3 + per-row scales" if fp8 else ""),
                        "parallelism": f"replicas x{world}",
-                       "l2": (f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB read per "
+                       "l2": (f"inputs larger than L2 ({r['step_bytes'] / 1e9:.2f} GB read per "
                               f"step over {c.layers} layer caches)"),
-                       "split_k": {"num_splits": ns, "split_tokens": split_tokens},
+                       "split_k": {"num_splits": r["ns"], "split_tokens": r["split_tokens"]},
                        "timing": f"CUDA graph of one {c.layers}-layer step, CUDA events"},
             "pct_of_peak": 100.0 * value / world / peak,
-            "tokens_per_s_per_layer_step": tok_layer_step,
-            "ms_per_step_eager": ms_eager,
-            "roofline": roofline,
-            "attention_tflops": flops / (attend_ms * 1e-3) / 1e12,
-            "e2e": {"value": whole_job_gbs(world, step_bytes, e2e_ms), "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks,
+            "tokens_per_s_per_layer_step": world * c.B * c.T_new / (ms * 1e-3 / c.layers),
+            "ms_per_step_eager": r["ms_eager"],
+            "ms_per_step_no_dependent_launch": r.get("ms_no_dependent_launch"),
+            "roofline": r["roofline"],
+            "attention_tflops": r["tflops_step"],
+            "e2e": {"value": whole_job_gbs(world, r["step_bytes"], r["e2e_ms"]), "unit": "GB/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                    "ms_per_step": r["e2e_ms"]},
+            "gpu_launches": r["launches_per_step"] * args.steps,
+            "clocks": r["clocks"],
             "cpu_baseline": cpu,
+            "workloads": extra or None,
         }
         print(json.dumps(line), flush=True)
     reps.close()
@@ -534,6 +622,23 @@ WORKLOADS = {
        for g in (2, 4, 8) for h in (8, 1)},
 }
 
+# the named configurations the default run also measures (bounded), beside the headline
+EXTRA_WORKLOADS = [("mha_b4_L4096", "native"), ("mha_b4_L8192", "native"),
+                   ("paged_gqa", "native"),
+                   *[(f"verify_g{g}_hkv{h}", "native") for h in (8, 1) for g in (2, 4, 8)],
+                   ("gqa_32layer", "fp8")]
+
+
+def sized_case(name: str, layers: int) -> W.Case:
+    """The named workload with `layers` layer caches, or by default enough independent
+    layer caches that a step reads more than 4x L2."""
+    case = WORKLOADS[name]()
+    if layers:
+        case.layers = layers
+    else:
+        case.layers = max(case.layers, -(-int(4 * L2_BYTES) // case.kv_read_bytes(True)))
+    return case
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -547,14 +652,15 @@ def main():
                     help="override the layer count (a smaller case for profiling)")
     ap.add_argument("--kv-format", default="native", choices=["native", "fp8"],
                     help="K/V storage: the 16-bit type, or FP8 E4M3 with per-row scales")
+    ap.add_argument("--launch-samples", type=int, default=64,
+                    help="event-bracketed calls whose median gives the per-call duration")
+    ap.add_argument("--workloads", default="all", choices=["all", "none"],
+                    help="also measure every other named configuration (one GPU only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    case = WORKLOADS[args.workload]()
-    if args.layers:
-        case.layers = args.layers
-    else:  # enough independent layer caches that a step reads more than 4x L2
-        case.layers = max(case.layers, -(-int(4 * L2_BYTES) // case.kv_read_bytes(True)))
+    args.launch_samples = max(50, args.launch_samples)
+    case = sized_case(args.workload, args.layers)
     if args.impl == "reference":
         run_reference(args, case)
     else:

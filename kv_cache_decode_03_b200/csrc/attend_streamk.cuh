@@ -6,10 +6,13 @@
 //
 // * Work is counted in 64-token tiles of "segments" s = (request b, KV head g,
 //   row block rb), in that order; segment s has ceil((L_b + i_max + 1) / 64)
-//   tiles, where i_max is the largest new-row index of the row block.  Each of
-//   the G persistent CTAs takes the contiguous tile range
-//   [c*W/G, (c+1)*W/G) of the W tiles in total, so every CTA streams the same
-//   number of K/V bytes to within one tile, whatever the mix of lengths.
+//   tiles, where i_max is the largest new-row index of the row block.  Each
+//   segment is preceded by `sk_penalty` virtual tiles that hold no work: a CTA
+//   pays a fixed cost (epilogue, ticket, a new q and a ring that restarts) for
+//   every segment it enters, and the virtual tiles charge that cost to it.
+//   Each of the G persistent CTAs takes the contiguous range [c*W/G,
+//   (c+1)*W/G) of the W virtual tiles in total, so every CTA streams the same
+//   work, costs included, whatever the mix of lengths.
 //   Every CTA computes the per-request tile counts and their prefix sums from
 //   seq_lens itself (a block scan), so the host needs no lengths.
 // * Warp 0 keeps the 3-stage TMA ring full across segment boundaries; the
@@ -62,6 +65,20 @@ __device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int c0, int c1
                : "memory");
 }
 
+// atomicAdd(ticket, 1) with release-acquire semantics at GPU scope: every write
+// this CTA made before the barrier that precedes it is visible to whoever reads the
+// new count, and the writes of the CTAs counted before it are visible to this one.
+__device__ __forceinline__ int ticket_add_acq_rel(int* ticket) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
+  return old;
+}
+
+// L2 prefetch of `bytes` (a multiple of 16) from a 16-byte aligned address.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // -------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start before the
 // grid ahead of it in the stream has finished.  griddep_wait() blocks until that
@@ -94,8 +111,15 @@ struct StreamKCfg {
            + kWarps * NT * 8 * 2 * sizeof(float)        // warp m and l
            + 2 * kStages * sizeof(uint64_t) + 64;       // barriers, flags
   }
-  // the block scan of per-request tile counts uses the ring before the first copy
-  static constexpr int kMaxBatch = kRing / (int)sizeof(int) - 1;
+  // resident CTAs an SM should hold (shared memory allows 4 at D = 64, 2 at D = 128):
+  // a register bound for the compiler
+  template <int NT>
+  static constexpr int min_blocks() {
+    return D == 64 ? (NT == 1 ? 4 : 3) : 2;
+  }
+  // the block scan of per-request tile counts and the lengths it read use the ring
+  // before the first copy
+  static constexpr int kMaxBatch = (kRing / (int)sizeof(int) - 1) / 2;
 };
 
 // Row-block geometry: new-row indices covered by row block rb.
@@ -116,26 +140,28 @@ __device__ __forceinline__ bool length_ok(const AttendParams& p, int L, bool pag
          (!paged || ((L + p.T_new - 1) >> p.page_shift) < p.max_pages);
 }
 
+// Virtual tiles of request b: its segments' tiles plus their penalty tiles.
 template <int R>
 __device__ __forceinline__ int request_tiles(const AttendParams& p, int L) {
   int t = 0;
   for (int rb = 0; rb < p.row_blocks; ++rb)
-    t += ceil_div(L + row_block(rb, R, p.rows, p.T_new).imax + 1, 64);
+    t += ceil_div(L + row_block(rb, R, p.rows, p.T_new).imax + 1, 64) + p.sk_penalty;
   return t * p.H_kv;
 }
 
-// Walks tiles in the global order: request, KV head, row block, tile.
+// Walks the real tiles in the global order: request, KV head, row block, tile.
 template <int R>
 struct TileCursor {
   int b, g, rb, L, k, seg_tiles;
-  long long seg_start;  // global index of the segment's first tile
+  long long seg_start;  // virtual index of the segment's first real tile
 
   __device__ __forceinline__ void enter_segment(const AttendParams& p) {
     seg_tiles = ceil_div(L + row_block(rb, R, p.rows, p.T_new).imax + 1, 64);
   }
-  __device__ __forceinline__ void next(const AttendParams& p, bool paged) {
+  // lens: the requests' lengths (seq_lens, or a copy of them in shared memory)
+  __device__ __forceinline__ void next(const AttendParams& p, bool paged, const int* lens) {
     if (++k < seg_tiles) return;
-    seg_start += seg_tiles;
+    seg_start += seg_tiles + p.sk_penalty;
     k = 0;
     if (++rb == p.row_blocks) {
       rb = 0;
@@ -143,11 +169,14 @@ struct TileCursor {
         g = 0;
         do {  // requests whose length is invalid contribute no tiles
           ++b;
-          L = b < p.B ? p.seq_lens[b] : 0;
+          L = b < p.B ? lens[b] : 0;
         } while (b < p.B && !length_ok(p, L, paged));
       }
     }
     enter_segment(p);
+  }
+  __device__ __forceinline__ void next(const AttendParams& p, bool paged) {
+    next(p, paged, p.seq_lens);
   }
 };
 
@@ -165,7 +194,7 @@ struct RangeMap {
 // valid, outputs from row_base) by log-sum-exp:
 //     out = sum_q 2^(lse_q - M) o_q / sum_q 2^(lse_q - M),   M = max_q lse_q.
 // Piece q lives in workspace slot 2*(rf+q) + 1 if it is the first piece and range rf
-// began before the segment (s0), else 2*(rf+q).  Each output quad (4 consecutive
+// began before the segment (its penalty tiles, before s0), else 2*(rf+q).  Each output quad (4 consecutive
 // elements of a row) is handled by tpq consecutive lanes (a power of two up to 8,
 // chosen so the CTA's threads cover the quads): lane `sub` of the group takes pieces
 // sub, sub + tpq, ..., issuing the lse and the float4 of four pieces before using
@@ -178,7 +207,9 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
   constexpr int Q4 = D / 4;
   const int tid = threadIdx.x;
   const int npc = (int)(rl - rf + 1);
-  const bool rf_mid = rm.start(rf) < s0;
+  // range rf streamed real tiles of an earlier segment first iff it began before this
+  // segment's penalty tiles
+  const bool rf_mid = rm.start(rf) < s0 - p.sk_penalty;
   const int items = nr * Q4;
   int tpq = 1;
   while (tpq < 8 && tpq < npc && items * tpq * 2 <= NTH) tpq *= 2;
@@ -261,7 +292,7 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
 }
 
 template <int D, int NT, typename T, bool PAGED>
-__global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
+__global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::template min_blocks<NT>())
     attend_streamk_kernel(const AttendParams p, const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv) {
   using C = StreamKCfg<D>;
@@ -306,6 +337,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
 
   // ------------------------------------ per-request tile prefix and this CTA's range
   int* P = reinterpret_cast<int*>(smem);  // [B + 1], in the ring before any copy
+  int* Ls = P + p.B + 1;                   // [B]: the lengths the scan read
   long long Wt = 0, lo = 0;
   int G = 0, ntiles = 0;
   TileCursor<R> cur;
@@ -314,7 +346,8 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
   const int b_lo = min(p.B, tid * per_thread), b_hi = min(p.B, b_lo + per_thread);
   auto mix = [](uint32_t h, int L) { return (h ^ (uint32_t)L) * 0x9E3779B1u + 0x7F4A7C15u; };
   uint32_t digest = 0;
-  // Returns whether this CTA has tiles; ends with a barrier (P is then dead).
+  // Returns whether this CTA has tiles; ends with a barrier.  P and Ls stay valid until
+  // the first copy into the ring.
   auto locate = [&](bool authoritative) -> bool {
     {
       int sum = 0;
@@ -322,6 +355,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
       for (int b = b_lo; b < b_hi; ++b) {
         const int L = p.seq_lens[b];
         digest = mix(digest, L);
+        Ls[b] = L;
         int t = 0;
         if (length_ok(p, L, PAGED)) t = request_tiles<R>(p, L);
         else if (authoritative) flag_error(p.err, KVC_ERR_BOUNDS);
@@ -363,8 +397,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
       }
       while (P[a + 1] == P[a]) ++a;  // skip requests with no tiles
       cur.b = a;
-      cur.L = p.seq_lens[a];
-      // a length read before the wait may be changing under this read
+      cur.L = Ls[a];
       work = length_ok(p, cur.L, PAGED);
       int local = (int)(lo - P[a]);
       const int per_g = (P[a + 1] - P[a]) / p.H_kv;
@@ -373,17 +406,34 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
       cur.rb = 0;
       while (work) {
         const int t = ceil_div(cur.L + row_block(cur.rb, R, p.rows, p.T_new).imax + 1, 64);
-        if (local < t || cur.rb == p.row_blocks - 1) {
+        if (local < t + p.sk_penalty || cur.rb == p.row_blocks - 1) {
           cur.seg_tiles = t;
           break;
         }
-        local -= t;
+        local -= t + p.sk_penalty;
         ++cur.rb;
       }
-      cur.k = local;
-      cur.seg_start = lo - local;
+      // local: the virtual offset in the segment; its penalty tiles are skipped
+      cur.seg_start = lo - local + p.sk_penalty;
+      cur.k = max(0, local - p.sk_penalty);
+      // the real tiles of [lo, hi): walk the segments the range reaches
+      const long long hi = (long long)(c + 1) * Wt / G;
+      ntiles = 0;
+      TileCursor<R> w = cur;
+#pragma unroll 1
+      while (work && w.b < p.B) {
+        const long long v = w.seg_start + w.k;
+        if (v >= hi) break;
+        const long long seg_end = w.seg_start + w.seg_tiles;
+        const long long stop = hi < seg_end ? hi : seg_end;
+        ntiles += (int)(stop - v);
+        if (stop < seg_end) break;
+        w.k = w.seg_tiles - 1;
+        w.next(p, PAGED, Ls);
+      }
+      work = work && ntiles > 0;
     }
-    __syncthreads();  // P is dead: the ring may now be filled
+    __syncthreads();
     return work;
   };
 
@@ -423,6 +473,13 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     TileCursor<R> pc = cur;
 #pragma unroll 1
     for (int i = 0; i < pf && pc.b < p.B; ++i) {
+      if ((i == 0 || pc.k == 0) && lane == 31) {  // the piece's q rows
+        const int r0 = pc.rb * R;
+        const char* qsrc = static_cast<const char*>(p.q) +
+                           ((((size_t)pc.b * p.H_q + (size_t)pc.g * p.group) * p.T_new) + r0) *
+                               D * 2;
+        bulk_prefetch_l2(qsrc, (uint32_t)min(R, p.rows - r0) * D * 2);
+      }
       if (!PAGED) {
         const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
         if (lane < C::kHalves && y + C::kTile <= rows_total) {
@@ -438,7 +495,22 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
             tma_prefetch_2d(&tmv, h * 64, y);
           }
       }
-      pc.next(p, PAGED);
+      pc.next(p, PAGED, Ls);
+    }
+  }
+  if (spec_work && warp == 1 && lane == 0 && p.k_new != nullptr) {
+    // the new rows of every segment this range ends: the fused append reads them
+    const long long hi = (long long)(c + 1) * Wt / G;
+    TileCursor<R> w = cur;
+#pragma unroll 1
+    while (w.b < p.B && w.seg_start < hi) {
+      if (w.seg_start + w.seg_tiles <= hi) {
+        const size_t off = ((size_t)w.b * p.H_kv + w.g) * p.T_new * D * 2;
+        bulk_prefetch_l2(static_cast<const char*>(p.k_new) + off, (uint32_t)p.T_new * D * 2);
+        bulk_prefetch_l2(static_cast<const char*>(p.v_new) + off, (uint32_t)p.T_new * D * 2);
+      }
+      w.k = w.seg_tiles - 1;
+      w.next(p, PAGED, Ls);
     }
   }
   griddep_wait();
@@ -536,6 +608,19 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     }
   };
 
+  // The producer keeps kStages tiles in flight: tile t goes into stage t % kStages
+  // once tile t - kStages has been released (`released` tiles are).  Warp 0 only.
+  auto refill = [&](int released) {
+#pragma unroll 1
+    while (issued < ntiles && issued < released + C::kStages) {
+      const int t = issued - C::kStages;
+      bool ready = true;
+      if (lane == 0) ready = wait(&empty[t % C::kStages], (t / C::kStages) & 1);
+      if (!__shfl_sync(0xffffffffu, ready, 0)) break;  // aborted: issue nothing more
+      issue();
+    }
+  };
+
   // ------------------------------------------------------------- consumers
   const int mi = lane >> 3;
   const int wrow = warp * 16;
@@ -551,15 +636,50 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
   int r0 = 0, nr = 0, vis_min = 0, piece_first_j = 0;
   float m[NT][2], l[NT][2];
   float o[C::kMTiles][NT][4];
+  // fresh running state; reset again at the end of every piece
+  auto reset_state = [&]() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        m[nt][cc] = -INFINITY;
+        l[nt][cc] = 0.f;
+      }
+#pragma unroll
+      for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+    }
+  };
+  reset_state();
+
+  // A partial piece's ticket (see the end of a piece) and what its merge needs.
+  constexpr int kTicketThread = 32;  // warp 1: the producer warp never waits on it
+  RangeMap rm;
+  rm.W = Wt;
+  rm.G = G;
+  bool pend = false;
+  long long pend_rf = 0, pend_rl = 0, pend_s0 = 0;
+  int pend_nr = 0, pend_count = 0;
+  size_t pend_row_base = 0;
+  int* pend_ticket = nullptr;
+  // Every thread: if the pending ticket was the segment's last, merge its pieces.
+  auto settle = [&]() {
+    if (tid == kTicketThread) flags[1] = pend_count == (int)(pend_rl - pend_rf);
+    named_barrier_sync(1, NTH);
+    if (flags[1]) {
+      merge_pieces_spread<T, D, R, NTH>(p, rm, pend_rf, pend_rl, pend_s0, pend_nr,
+                                        pend_row_base);
+      if (tid == 0) *pend_ticket = 0;
+    }
+    named_barrier_sync(1, NTH);  // flags[1] is read by every thread before it is reused
+    pend = false;
+  };
 
 #pragma unroll 1
   for (int j = 0; j < ntiles; ++j) {
     const int st = j % C::kStages;
-    if (producer && j >= 1 && issued < ntiles) {
-      bool ready = true;
-      if (lane == 0) ready = wait(&empty[(j - 1) % C::kStages], ((j - 1) / C::kStages) & 1);
-      if (__shfl_sync(0xffffffffu, ready, 0)) issue();
-    }
+    if (producer && j >= 1) refill(j);
     wait(&full[st], (j / C::kStages) & 1);
 
     if (j == 0 || cur.k == 0) {  // a new piece: its q rows, visibility, fresh state
@@ -586,13 +706,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
         for (int cc = 0; cc < 2; ++cc) {
           const int rr = nt * 8 + (lane & 3) * 2 + cc;
           vis[nt][cc] = rr < nr ? cur.L + (r0 + rr) % p.T_new + 1 : 0;
-          m[nt][cc] = -INFINITY;
-          l[nt][cc] = 0.f;
         }
-#pragma unroll
-        for (int mt = 0; mt < C::kMTiles; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
       }
     }
 
@@ -729,8 +843,10 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     }
 
     // -------------------------------------------- end of a segment piece
-    // The four warps merge inside this stage's K/V buffers (every warp is
-    // done reading them after the barrier); other stages keep streaming.
+    // The four warps merge inside this stage's K/V buffers (every warp is done
+    // reading them after the barrier) into registers; then the stage is released
+    // and refilled at once, so the ring keeps streaming while the piece's result
+    // is written and its ticket taken.
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -743,8 +859,9 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
     float* red_acc = reinterpret_cast<float*>(sk + st * C::kTileBytes);
     float* red_acc_hi = reinterpret_cast<float*>(sv + st * C::kTileBytes);
     auto acc_at = [&](int w, int row, int d) -> float* {
-      // W*R*D floats spread over this stage's K then V buffers
-      const int idx = (w * R + row) * D + d;
+      // W*R*D floats spread over this stage's K then V buffers; the column is
+      // swizzled by row bits 1-2 so that the fragment stores hit 32 distinct banks
+      const int idx = (w * R + row) * D + (d ^ (((row >> 1) & 3) << 3));
       constexpr int kHalfFloats = C::kTileBytes / 4;
       return idx < kHalfFloats ? red_acc + idx : red_acc_hi + (idx - kHalfFloats);
     };
@@ -768,7 +885,49 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
           red_l[warp * R + row] = l[nt][cc];
         }
     }
+    reset_state();
     named_barrier_sync(1, NTH);
+    // per row, once: warp w's weight 2^(m_w - M) / l in red_m, the row's base-2
+    // log-sum-exp M + log2 l in red_l[row] (a row that saw nothing: weights 0, -inf)
+    if (tid < R) {
+      const int rr = tid;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W; ++w) M = fmaxf(M, red_m[w * R + rr]);
+      float f[W];
+      float lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        f[w] = M == -INFINITY ? 0.f : exp2f(red_m[w * R + rr] - M);
+        lsum = fmaf(red_l[w * R + rr], f[w], lsum);
+      }
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) red_m[w * R + rr] = f[w] * inv;
+      red_l[rr] = lsum > 0.f ? M + log2f(lsum) : -INFINITY;
+    }
+    named_barrier_sync(1, NTH);
+
+    // element k of this thread: row (tid + k*NTH) / D, column (tid + k*NTH) % D
+    constexpr int PER = R * D / NTH;
+    float res[PER];  // the row's output (whole piece) or normalised partial
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int idx = tid + k * NTH;
+      const int rr = idx / D;
+      const int d = idx - rr * D;
+      float ov = 0.f;
+      if (rr < nr) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) ov = fmaf(*acc_at(w, rr, d), red_m[w * R + rr], ov);
+      }
+      res[k] = ov;
+    }
+    named_barrier_sync(1, NTH);  // the stage is read: release and refill it
+    if (lane == 0) mbar_arrive(&empty[st]);
+    if (producer) refill(j + 1);
+    // a ticket taken at an earlier piece end is settled now, while the ring streams
+    if (pend) settle();
 
     const bool whole = (piece_first_j == j - cur.k) && (cur.k == cur.seg_tiles - 1);
     const int slot = (piece_first_j == 0) ? 0 : 1;
@@ -777,56 +936,39 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads)
         ((size_t)cur.b * p.H_q + (size_t)cur.g * p.group) * p.T_new + r0;
     float* wso = p.ws_o + ((size_t)c * 2 + slot) * R * D;
     float* wsl = p.ws_lse + ((size_t)c * 2 + slot) * R;
-#pragma unroll 1
-    for (int idx = tid; idx < R * D; idx += NTH) {
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int idx = tid + k * NTH;
       const int rr = idx / D;
       const int d = idx - rr * D;
-      if (rr >= nr) break;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < W; ++w) M = fmaxf(M, red_m[w * R + rr]);
-      float lsum = 0.f, ov = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < W; ++w) {
-          const float f = exp2f(red_m[w * R + rr] - M);
-          lsum = fmaf(red_l[w * R + rr], f, lsum);
-          ov = fmaf(*acc_at(w, rr, d), f, ov);
+      if (rr < nr) {
+        if (whole) {
+          store_elt<T>(out + (row_base + rr) * D + d, res[k]);
+        } else {
+          wso[rr * D + d] = res[k];
+          if (d == 0) wsl[rr] = red_l[rr];
         }
-      }
-      if (whole) {
-        store_elt<T>(out + (row_base + rr) * D + d, ov / lsum);
-      } else {
-        wso[rr * D + d] = M == -INFINITY ? 0.f : ov / lsum;
-        if (d == 0) wsl[rr] = M == -INFINITY ? -INFINITY : M + log2f(lsum);
       }
     }
     if (!whole) {
-      // hand the piece to the segment's last finisher: the barrier orders every
-      // thread's partial stores before thread 0's fence and ticket
+      // Hand the piece to the segment's last finisher: the barrier orders every
+      // thread's partial stores before the release-acquire ticket, whose result is
+      // read only at the next piece end or after the loop (settle()), so nobody
+      // waits for it here.
       named_barrier_sync(1, NTH);
-      const long long s0 = cur.seg_start, s1 = cur.seg_start + cur.seg_tiles - 1;
-      RangeMap rm;
-      rm.W = Wt;
-      rm.G = G;
-      const long long rf = rm.of(s0), rl = rm.of(s1);
-      int* ticket = p.counters + ((size_t)cur.b * p.H_kv + cur.g) * p.row_blocks + cur.rb;
-      if (tid == 0) {
-        __threadfence();
-        const bool last = atomicAdd(ticket, 1) == (int)(rl - rf);
-        if (last) __threadfence();  // acquire the other pieces before the barrier
-        flags[1] = last;
-      }
-      named_barrier_sync(1, NTH);
-      if (flags[1]) {
-        merge_pieces_spread<T, D, R, NTH>(p, rm, rf, rl, s0, nr, row_base);
-        if (tid == 0) *ticket = 0;
-      }
+      pend = true;
+      pend_s0 = cur.seg_start;
+      const long long s1 = cur.seg_start + cur.seg_tiles - 1;
+      pend_rf = rm.of(pend_s0);
+      pend_rl = rm.of(s1);
+      pend_nr = nr;
+      pend_row_base = row_base;
+      pend_ticket = p.counters + ((size_t)cur.b * p.H_kv + cur.g) * p.row_blocks + cur.rb;
+      if (tid == kTicketThread) pend_count = ticket_add_acq_rel(pend_ticket);
     }
-    named_barrier_sync(1, NTH);  // the stage's buffers are free again
-    if (lane == 0) mbar_arrive(&empty[st]);
     cur.next(p, PAGED);
   }
+  if (pend) settle();
   // After an abort, do not retire while copies may still be landing.
   if (producer && lane == 0 && *abort_word)
 #pragma unroll 1

@@ -85,6 +85,15 @@ constexpr int kEltBytes = 2;
 #ifndef KVC_TC_MIN_SLICE_TILES
 #define KVC_TC_MIN_SLICE_TILES 16
 #endif
+// Stream-K: virtual tiles charged per segment a CTA enters (the fixed cost of a piece:
+// epilogue, ticket, a fresh q and a ring restart, measured at about two to four tiles'
+// streaming time), so CTAs that cross segment boundaries get fewer real tiles.
+#ifndef KVC_SK_PENALTY_D128
+#define KVC_SK_PENALTY_D128 3
+#endif
+#ifndef KVC_SK_PENALTY_D64
+#define KVC_SK_PENALTY_D64 2
+#endif
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -715,6 +724,7 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
   p.row_blocks = pl.row_blocks;
   p.err = c->d_err;
   p.wait_limit_ns = c->wait_limit_ns;
+  p.sk_penalty = !pl.streamk ? 0 : c->D == 128 ? KVC_SK_PENALTY_D128 : KVC_SK_PENALTY_D64;
   p.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   return p;

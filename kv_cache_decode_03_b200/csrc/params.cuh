@@ -46,6 +46,7 @@ struct AttendParams {
   const void* v_new;
   int* err;
   unsigned long long wait_limit_ns;  // bound of every pipeline wait (0: the default, 1 s)
+  int sk_penalty;  // stream-K: virtual tiles charged for each segment a CTA enters
   int stall;  // failure-detection test: the producers issue no copies, so the first
               // wait runs out (stream-K and tcgen05 kernels)
 };
