@@ -15,6 +15,12 @@
 //   work, costs included, whatever the mix of lengths.
 //   Every CTA computes the per-request tile counts and their prefix sums from
 //   seq_lens itself (a block scan), so the host needs no lengths.
+// * Stage layout: K (and V) rows of 128-byte, 128-byte-swizzled chunks.  Contiguous
+//   caches and pages of 64+ tokens: one 64-row box per 64-element half ([half][row]).
+//   Paged D = 128 with smaller pages: the tensor maps are 4-D (64 elements, page
+//   tokens, 2 halves, page blocks) so that one box brings a whole (page, head) block,
+//   laid out [page][half][row in page] -- half the copies of per-half boxes, and the
+//   same conflict-free ldmatrix pattern (8 consecutive rows of one half).
 // * Warp 0 keeps the 3-stage TMA ring full across segment boundaries; the
 //   first tile of each segment piece also carries that segment's q rows (one
 //   bulk copy into a per-stage q slot).  On a paged cache lane k of warp 0
@@ -49,10 +55,16 @@
 #ifndef KVC_SK_STAGES
 #define KVC_SK_STAGES 3
 #endif
-// Bytes of K/V that all CTAs together may prefetch into L2 before the dependency
-// wait (a part of the 126 MB L2, so the prefetched lines survive until they are read).
-#ifndef KVC_SK_PREFETCH_BYTES
-#define KVC_SK_PREFETCH_BYTES (48ll << 20)
+// Tiles of its range a CTA prefetches into L2 before the dependency wait (measured:
+// 2 beats 0, 1, 3 and 5: more delays the CTAs that start late and competes with the
+// grid ahead for HBM).
+// Paged: tiles ahead of the next copy whose page ids are already being read (measured:
+// 3 is no faster than 1 once a page is one box).
+#ifndef KVC_SK_LOOKAHEAD
+#define KVC_SK_LOOKAHEAD 1
+#endif
+#ifndef KVC_SK_PREFETCH_TILES
+#define KVC_SK_PREFETCH_TILES 2
 #endif
 
 namespace kvc {
@@ -72,6 +84,22 @@ __device__ __forceinline__ int ticket_add_acq_rel(int* ticket) {
   int old;
   asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
   return old;
+}
+
+// 4-D tiled load / L2 prefetch of one box (the blocked paged layout), no multicast.
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int c0, int c1, int c2,
+                                            int c3, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;"
+      ::"r"(smem_addr(dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_4d(const void* tmap, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+               ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 
 // L2 prefetch of `bytes` (a multiple of 16) from a 16-byte aligned address.
@@ -442,6 +470,17 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
   const int box_rows = Pg < C::kTile ? Pg : C::kTile;
   const int nbox = C::kTile / box_rows;         // <= 8: pages of 8 or more tokens
   const int beyond = p.num_pages * p.H_kv * Pg;  // first row past the pool: zero fill
+  const bool blocked = PAGED && D == 128 && p.sk_blocked != 0;
+  // byte offset in a stage of tile row `row` (its half 0, chunk 0 before the swizzle)
+  auto row_part = [&](int row) -> int {
+    return blocked ? (row >> p.page_shift) * (box_rows * 256) + (row & (box_rows - 1)) * 128
+                   : row * 128;
+  };
+  const int half_stride = blocked ? box_rows * 128 : C::kBoxBytes;
+  // byte offset of 16-byte chunk `chunk` (of D/8) of tile row `row`, swizzled
+  auto tile_off = [&](int row, int chunk) -> uint32_t {
+    return row_part(row) + (chunk >> 3) * half_stride + (((chunk & 7) ^ (row & 7)) << 4);
+  };
   // Row of box `box` of the tile under cursor pc: -1 = the lookup is still to be done;
   // returns `beyond` past the segment's last position.
   auto box_page_row = [&](const TileCursor<R>& pc, int box, int page) -> int {
@@ -468,11 +507,10 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
     // only boxes wholly inside the tensor: the cursor may walk off stale lengths
     const long long rows_total =
         PAGED ? (long long)p.num_pages * p.H_kv * Pg : (long long)p.B * p.H_kv * p.max_T;
-    const long long budget = KVC_SK_PREFETCH_BYTES / ((long long)G * 2 * C::kTileBytes);
-    const int pf = (int)min((long long)ntiles, max((long long)C::kStages, budget));
+    const int pf = min(ntiles, KVC_SK_PREFETCH_TILES);
     TileCursor<R> pc = cur;
 #pragma unroll 1
-    for (int i = 0; i < pf && pc.b < p.B; ++i) {
+    for (int i = 0; i < max(pf, 1) && pc.b < p.B; ++i) {
       if ((i == 0 || pc.k == 0) && lane == 31) {  // the piece's q rows
         const int r0 = pc.rb * R;
         const char* qsrc = static_cast<const char*>(p.q) +
@@ -480,6 +518,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
                                D * 2;
         bulk_prefetch_l2(qsrc, (uint32_t)min(R, p.rows - r0) * D * 2);
       }
+      if (i >= pf) break;  // no tiles prefetched: q only
       if (!PAGED) {
         const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
         if (lane < C::kHalves && y + C::kTile <= rows_total) {
@@ -488,12 +527,18 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
         }
       } else if (lane < nbox) {
         const int y = box_page_row(pc, lane, lookup_page(pc, lane));
-        if (y >= 0 && y != beyond && y + box_rows <= rows_total)
+        if (y >= 0 && y != beyond && y + box_rows <= rows_total) {
+          if (blocked) {
+            tma_prefetch_4d(&tmk, 0, 0, 0, y >> p.page_shift);
+            tma_prefetch_4d(&tmv, 0, 0, 0, y >> p.page_shift);
+          } else {
 #pragma unroll
-          for (int h = 0; h < C::kHalves; ++h) {
-            tma_prefetch_2d(&tmk, h * 64, y);
-            tma_prefetch_2d(&tmv, h * 64, y);
+            for (int h = 0; h < C::kHalves; ++h) {
+              tma_prefetch_2d(&tmk, h * 64, y);
+              tma_prefetch_2d(&tmv, h * 64, y);
+            }
           }
+        }
       }
       pc.next(p, PAGED, Ls);
     }
@@ -539,7 +584,19 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
   const uint64_t pol = l2_policy_evict_first();
   TileCursor<R> pc = cur;  // producer's own cursor
   int issued = 0;
-  int page_ahead = PAGED && producer ? lookup_page(pc, lane) : 0;
+  // Paged: lane k < nbox holds the page ids of box k of the next kLookahead tiles to
+  // issue (ids[0] for tile pc); a second cursor, kLookahead - 1 tiles ahead of pc, reads
+  // them, so a lookup has that many tiles' time to land.
+  constexpr int kLookahead = KVC_SK_LOOKAHEAD;
+  int ids[kLookahead];
+  TileCursor<R> pa = cur;
+  if (PAGED && producer) {
+#pragma unroll
+    for (int i = 0; i < kLookahead; ++i) {
+      if (i > 0) pa.next(p, PAGED);
+      ids[i] = lookup_page(pa, lane);
+    }
+  }
   auto issue = [&]() {
     const int st = issued % C::kStages;
     const bool first = (issued == 0) || (pc.k == 0);
@@ -565,21 +622,32 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
         tma_load_2d(dv + lane * C::kBoxBytes, &tmv, lane * 64, y, &full[st], pol);
       }
     } else if (lane < nbox) {
-      int y = box_page_row(pc, lane, page_ahead);
+      int y = box_page_row(pc, lane, ids[0]);
       if (y < 0) {  // a page id outside the pool: zero fill, reported
         flag_error(p.err, KVC_ERR_BOUNDS);
         y = beyond;
       }
-      const int off = lane * box_rows * 128;
+      if (blocked) {  // one box: the page's block, both halves
+        const int off = lane * box_rows * 256;
+        tma_load_4d(dk + off, &tmk, 0, 0, 0, y >> p.page_shift, &full[st], pol);
+        tma_load_4d(dv + off, &tmv, 0, 0, 0, y >> p.page_shift, &full[st], pol);
+      } else {
+        const int off = lane * box_rows * 128;
 #pragma unroll
-      for (int h = 0; h < C::kHalves; ++h) {
-        tma_load_2d(dk + h * C::kBoxBytes + off, &tmk, h * 64, y, &full[st], pol);
-        tma_load_2d(dv + h * C::kBoxBytes + off, &tmv, h * 64, y, &full[st], pol);
+        for (int h = 0; h < C::kHalves; ++h) {
+          tma_load_2d(dk + h * C::kBoxBytes + off, &tmk, h * 64, y, &full[st], pol);
+          tma_load_2d(dv + h * C::kBoxBytes + off, &tmv, h * 64, y, &full[st], pol);
+        }
       }
     }
     ++issued;
     pc.next(p, PAGED);
-    if (PAGED) page_ahead = lookup_page(pc, lane);  // consumed by the next issue
+    if (PAGED) {  // shift the lookahead queue and read the ids kLookahead - 1 tiles ahead
+#pragma unroll
+      for (int i = 0; i + 1 < kLookahead; ++i) ids[i] = ids[i + 1];
+      pa.next(p, PAGED);
+      ids[kLookahead - 1] = lookup_page(pa, lane);
+    }
   };
   if (producer)
     while (issued < min(C::kStages, ntiles)) issue();
@@ -630,6 +698,8 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
   const int v_cs = mi & 1;
   const uint32_t sk_addr = smem_addr(sk);
   const uint32_t sv_addr = smem_addr(sv);
+  const int k_rp = row_part(k_row), k_sw = k_row & 7;
+  const int v_rp = row_part(v_row), v_sw = v_row & 7;
 
   uint32_t qb[C::kKSteps][NT][2];
   int vis[NT][2];
@@ -731,7 +801,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
               ((((size_t)cur.b * p.H_kv + cur.g) * p.T_new + (pos - cur.L)) * D + ch * 8) * 2;
           const uint4 kv = ld_global_nc_v4(static_cast<const char*>(p.k_new) + src);
           const uint4 vv = ld_global_nc_v4(static_cast<const char*>(p.v_new) + src);
-          const uint32_t off = swz<D>(pos - ta, ch);
+          const uint32_t off = tile_off(pos - ta, ch);
           st_shared_v4(dk + off, kv);
           st_shared_v4(dv + off, vv);
           if (cur.rb == 0) {
@@ -766,7 +836,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
 #pragma unroll
     for (int kk = 0; kk < C::kKSteps; ++kk) {
       uint32_t a[4];
-      ldmatrix_x4(a, kb + swz<D>(k_row, 2 * kk + k_cs));
+      ldmatrix_x4(a, kb + k_rp + (kk >> 2) * half_stride + ((((2 * kk + k_cs) & 7) ^ k_sw) << 4));
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_16816<T>(sacc[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
     }
@@ -826,7 +896,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
 #pragma unroll
     for (int mt = 0; mt < C::kMTiles; ++mt) {
       uint32_t a[4];
-      ldmatrix_x4_trans(a, vb + swz<D>(v_row, 2 * mt + v_cs));
+      ldmatrix_x4_trans(a, vb + v_rp + (mt >> 2) * half_stride + ((((2 * mt + v_cs) & 7) ^ v_sw) << 4));
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);

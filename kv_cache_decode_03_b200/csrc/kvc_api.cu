@@ -39,6 +39,9 @@ struct kvc_cache {
   bool tma;                        // tensor maps built: the tensor-core path is available
   std::vector<CUtensorMap> tmk;    // per layer: K pool as a 2-D (rows, D) tensor
   std::vector<CUtensorMap> tmv;
+  bool tma4;                       // 4-D paged maps for the stream-K kernel (D 128, pages < 64)
+  std::vector<CUtensorMap> tmk4;   // per layer: (64 elements, page tokens, 2 halves, blocks)
+  std::vector<CUtensorMap> tmv4;
   int device;
   int num_sms;
   bool dependent_launch;           // stream-K launches with programmatic stream serialization
@@ -93,6 +96,10 @@ constexpr int kEltBytes = 2;
 #endif
 #ifndef KVC_SK_PENALTY_D64
 #define KVC_SK_PENALTY_D64 2
+#endif
+// Stream-K on paged D = 128 caches with pages under 64 tokens: one 4-D box per page.
+#ifndef KVC_SK_BLOCKED_PAGES
+#define KVC_SK_BLOCKED_PAGES 1
 #endif
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -154,6 +161,26 @@ bool make_tmap(CUtensorMap* m, void* base, kvc_dtype dtype, int D, long long row
   return r == CUDA_SUCCESS;
 }
 
+// Paged pools with D = 128 and pages of fewer than 64 tokens, for the stream-K kernel: a
+// 4-D view (64 elements, P tokens, 2 halves, num_pages x H_kv blocks) whose box is a whole
+// (page, head) block, landing in shared memory as [half][token] rows of 128 bytes.
+bool make_tmap_blocked(CUtensorMap* m, void* base, kvc_dtype dtype, int P, long long blocks) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {64u, (cuuint64_t)P, 2u, (cuuint64_t)blocks};
+  const cuuint64_t strides[3] = {128u * kEltBytes, 64u * kEltBytes,
+                                 (cuuint64_t)P * 128u * kEltBytes};
+  const cuuint32_t box[4] = {64u, (cuuint32_t)P, 2u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult r = fn(m,
+                        dtype == KVC_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, KVC_TMA_L2_PROMOTION,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // FP8 code pools: 2-D (rows, D) bytes, one D-byte row per box row, swizzled across the
 // row's 16-byte chunks (128-byte swizzle for D = 128, 64-byte for D = 64) so that the
 // kernel's ldmatrix reads are conflict-free.
@@ -205,6 +232,19 @@ void build_tmaps(kvc_cache* c) {
       return;
   }
   c->tma = true;
+  c->tma4 = false;
+  if (KVC_SK_BLOCKED_PAGES && c->paged && c->D == 128 && c->page_size < 64) {
+    const long long blocks = (long long)c->num_pages * c->H_kv;
+    c->tmk4.resize(c->num_layers);
+    c->tmv4.resize(c->num_layers);
+    for (int l = 0; l < c->num_layers; ++l)
+      if (!make_tmap_blocked(&c->tmk4[l], c->pool + (size_t)(2 * l) * c->layer_bytes, c->dtype,
+                             c->page_size, blocks) ||
+          !make_tmap_blocked(&c->tmv4[l], c->pool + (size_t)(2 * l + 1) * c->layer_bytes,
+                             c->dtype, c->page_size, blocks))
+        return;  // the stream-K kernel keeps the 2-D maps
+    c->tma4 = true;
+  }
 }
 
 template <int D, int NT, typename T, bool PAGED>
@@ -725,6 +765,7 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
   p.err = c->d_err;
   p.wait_limit_ns = c->wait_limit_ns;
   p.sk_penalty = !pl.streamk ? 0 : c->D == 128 ? KVC_SK_PENALTY_D128 : KVC_SK_PENALTY_D64;
+  p.sk_blocked = pl.streamk && c->tma4 ? 1 : 0;
   p.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   return p;
@@ -752,12 +793,14 @@ kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::At
   if (pl.tc)
     return bf ? dispatch_tc<__nv_bfloat16>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s)
               : dispatch_tc<__half>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s);
-  if (pl.streamk)
+  if (pl.streamk) {
+    const CUtensorMap& tk = p.sk_blocked ? c->tmk4[layer] : c->tmk[layer];
+    const CUtensorMap& tv = p.sk_blocked ? c->tmv4[layer] : c->tmv[layer];
     return bf ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
-                                                c->dependent_launch, c->tmk[layer],
-                                                c->tmv[layer], s)
+                                                c->dependent_launch, tk, tv, s)
               : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid,
-                                         c->dependent_launch, c->tmk[layer], c->tmv[layer], s);
+                                         c->dependent_launch, tk, tv, s);
+  }
   if (pl.mma)
     return bf ? dispatch_mma<__nv_bfloat16>(p, c->D, pl.NT, c->paged, c->tmk[layer],
                                             c->tmv[layer], s)
@@ -1270,10 +1313,11 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   p.k_new = k_new;
   p.v_new = v_new;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CUtensorMap& tk = p.sk_blocked ? c->tmk4[layer] : c->tmk[layer];
+  const CUtensorMap& tv = p.sk_blocked ? c->tmv4[layer] : c->tmv[layer];
   return c->dtype == KVC_BF16
              ? dispatch_streamk<__nv_bfloat16>(p, c->D, pl.NT, c->paged, pl.grid,
-                                               c->dependent_launch, c->tmk[layer],
-                                               c->tmv[layer], s)
+                                               c->dependent_launch, tk, tv, s)
              : dispatch_streamk<__half>(p, c->D, pl.NT, c->paged, pl.grid, c->dependent_launch,
-                                        c->tmk[layer], c->tmv[layer], s);
+                                        tk, tv, s);
 }
