@@ -50,6 +50,8 @@ KERNEL_SOURCES = {
                           "device_common.cuh", "params.cuh"),
     "attend_tc_kernel": ("attend_tc.cuh", "splitk_epilogue.cuh", "window.cuh",
                          "device_common.cuh", "params.cuh"),
+    "attend_tc_streamk_kernel": ("attend_tc_streamk.cuh", "attend_tc.cuh", "attend_streamk.cuh",
+                                 "device_common.cuh", "params.cuh"),
     "attend_fp8_kernel": ("attend_fp8.cuh", "fp8.cuh", "splitk_epilogue.cuh", "window.cuh",
                           "device_common.cuh", "params.cuh"),
     "attend_decode_kernel": ("attend_decode.cuh", "splitk_epilogue.cuh", "window.cuh",
@@ -119,6 +121,8 @@ def attend_kernel_name(c: W.Case, kv_format: str, split_tokens: int) -> str:
     if kv_format == "fp8":
         return f"attend_fp8_kernel<{c.D},{layout}>"
     if rows >= 64 and c.D in (64, 128):
+        if split_tokens == 0:
+            return f"attend_tc_streamk_kernel<{c.D},{c.dtype},{layout}>"
         return f"attend_tc_kernel<{c.D},{c.dtype},{layout}>"
     if split_tokens == 0:
         nt = 1 if rows <= 8 else 2
@@ -496,7 +500,7 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     call_s = res["call_ms_median"] * 1e-3
     step_call_s = ms * 1e-3 / c.layers  # one layer-step's share of the graph-timed step
     peak, peak_kind = peaks()
-    if kernel.startswith("attend_tc_kernel"):
+    if kernel.startswith("attend_tc"):
         tpeak, tpeak_kind = tensor_peak()
         roof = {"bound": "tensor", "achieved": flops / call_s / 1e12, "peak": tpeak,
                 "unit": "TFLOP/s", "traffic": None, "peak_source": tpeak_kind,

@@ -54,6 +54,13 @@
 #include "splitk_epilogue.cuh"
 
 
+#ifndef KVC_TC_KSTAGES_D128
+#define KVC_TC_KSTAGES_D128 3
+#endif
+#ifndef KVC_TC_VSTAGES_D128
+#define KVC_TC_VSTAGES_D128 2
+#endif
+
 namespace kvc {
 
 template <int D>
@@ -70,8 +77,8 @@ struct TcCfg {
   static constexpr int kBoxBytes = kTile * 128;  // one box of a K/V tile
   static constexpr int kTileBytes = kTile * D * 2;
   // stages sized so that two CTAs share an SM (<= 113 KB of shared memory each)
-  static constexpr int kKStages = D == 128 ? 3 : 4;
-  static constexpr int kVStages = D == 128 ? 2 : 4;
+  static constexpr int kKStages = D == 128 ? KVC_TC_KSTAGES_D128 : 4;
+  static constexpr int kVStages = D == 128 ? KVC_TC_VSTAGES_D128 : 4;
   static constexpr int kKRing = kKStages * kTileBytes;
   static constexpr int kVRing = kVStages * kTileBytes;
   static constexpr int kQBox = kRows * 128;      // one 64-element box of Q
@@ -85,8 +92,8 @@ struct TcCfg {
   static constexpr int kScratchOff = kAccBytes + 2 * kRows * 4;
   static constexpr int kScratchFloats = (kData - kScratchOff) / 4;
   static_assert(kScratchOff + kRows * 4 <= kData, "result area too small");
-  // K full/empty, V full/empty, s_full x2, p_full x2, o_done, drain
-  static constexpr int kBarriers = 2 * kKStages + 2 * kVStages + 6;
+  // K full/empty, V full/empty, s_full x2, p_full x2, o_done x2, drain
+  static constexpr int kBarriers = 2 * kKStages + 2 * kVStages + 7;
 
   // The dynamic shared memory starts 1024-byte aligned (checked at run time).
   static constexpr size_t smem_bytes() { return kData + kBarriers * sizeof(uint64_t) + 16; }
@@ -221,8 +228,11 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
   uint64_t* v_empty = v_full + SV;   // V stage consumed by its P.V MMA
   uint64_t* s_full = v_empty + SV;   // [2] S buffer holds Q.K^T
   uint64_t* p_full = s_full + 2;     // [2] S buffer holds P (128 arrivals)
-  uint64_t* o_done = p_full + 2;     // O += P.V of the last issued tile done
-  uint64_t* dbar = o_done + 1;       // drain after an abort
+  // [2] O += P(j).V(j) done, on o_done[j & 1]: each completes a phase every other tile,
+  // so a waiter is never more than one phase behind (a single barrier could be two
+  // phases past a P.V still pending, and a parity wait would then match the wrong phase)
+  uint64_t* o_done = p_full + 2;
+  uint64_t* dbar = o_done + 2;       // drain after an abort
   uint32_t* tslot = reinterpret_cast<uint32_t*>(dbar + 1);
   int* flags = reinterpret_cast<int*>(tslot + 1);  // [0] abort [1] last
   float* red_acc = reinterpret_cast<float*>(smem);  // operand area, after the loop
@@ -291,7 +301,8 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
       mbar_init(&s_full[k], 1);
       mbar_init(&p_full[k], NSM);
     }
-    mbar_init(o_done, 1);
+    mbar_init(&o_done[0], 1);
+    mbar_init(&o_done[1], 1);
     mbar_init(dbar, 1);
     flags[0] = 0;
     flags[1] = 0;
@@ -422,7 +433,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
       for (int j = 0; ok && j < ntiles; ++j) {
         if (j + 1 < ntiles) {
           // buffer (j+1)&1 still holds P(j-1) until its P.V MMA is done
-          if (j >= 1 && !wait(o_done, (j - 1) & 1)) {
+          if (j >= 1 && !wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
             ok = false;
             break;
           }
@@ -446,7 +457,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
           if constexpr (kSplitP) umma_f16_tmem_a(tO, tP + 32 + kk * 8, bv, idesc_o, true);
         }
         umma_commit(&v_empty[st]);
-        umma_commit(o_done);
+        umma_commit(&o_done[j & 1]);
       }
     }
     __syncwarp();
@@ -486,7 +497,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
       const float alpha = (move && m_ref != -INFINITY) ? ex2_approx(m_ref - mx) : 1.f;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {  // the warp's 32 rows together
         // O must hold P(j-1).V(j-1) first
-        ok = __all_sync(0xffffffffu, wait(o_done, (j - 1) & 1));
+        ok = __all_sync(0xffffffffu, wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
@@ -533,7 +544,9 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
       tc_fence_before();
       mbar_arrive(&p_full[buf]);
     }
-    if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, wait(o_done, (ntiles - 1) & 1));
+    if (ok && ntiles > 0)
+      ok = __all_sync(0xffffffffu,
+                      wait(&o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1));
   }
 
   const bool bad = __syncthreads_or(*abort_word != 0);

@@ -17,6 +17,7 @@
 #include "attend_mma.cuh"
 #include "attend_streamk.cuh"
 #include "attend_tc.cuh"
+#include "attend_tc_streamk.cuh"
 #include "cache_ops.cuh"
 #include "fp8.cuh"
 #include "kvc.h"
@@ -96,6 +97,20 @@ constexpr int kEltBytes = 2;
 #endif
 #ifndef KVC_SK_PENALTY_D64
 #define KVC_SK_PENALTY_D64 2
+#endif
+// tcgen05 rows (64+ per KV head) without a window run on the persistent stream-K
+// tcgen05 kernel; its penalty tiles charge a piece's Q reload, TMEM readout and partial.
+#ifndef KVC_TC_STREAMK
+#define KVC_TC_STREAMK 1
+#endif
+// Resident CTAs per SM the persistent tcgen05 grid assumes at least: the occupancy query
+// reports 1 for this 224-thread kernel although registers, shared memory and TMEM hold two,
+// and two do co-reside (MQA verify gamma 8: 24.6 % of HBM with 296 CTAs, 17.6 % with 148).
+#ifndef KVC_TC_MIN_OCC
+#define KVC_TC_MIN_OCC 2
+#endif
+#ifndef KVC_TC_SK_PENALTY
+#define KVC_TC_SK_PENALTY 3
 #endif
 // Stream-K on paged D = 128 caches with pages under 64 tokens: one 4-D box per page.
 #ifndef KVC_SK_BLOCKED_PAGES
@@ -336,6 +351,31 @@ int tc_occ(int D, bool paged) {
   return paged ? tc_occupancy<128, T, true>() : tc_occupancy<128, T, false>();
 }
 
+template <int D, typename T, bool PAGED>
+int tc_sk_occupancy() {
+  static int occ = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const size_t smem = kvc::TcSkCfg<D>::smem_bytes();
+    cudaFuncSetAttribute(kvc::attend_tc_streamk_kernel<D, T, PAGED>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, kvc::attend_tc_streamk_kernel<D, T, PAGED>, kvc::TcCfg<D>::kThreads, smem) !=
+        cudaSuccess)
+      n = 1;
+    // every resident CTA holds TMEM columns: never more than the 512 an SM has
+    occ = std::max(1, std::min(std::max(n, KVC_TC_MIN_OCC), 512 / kvc::TcCfg<D>::kTmemCols));
+  });
+  return occ;
+}
+
+template <typename T>
+int tc_sk_occ(int D, bool paged) {
+  if (D == 64) return paged ? tc_sk_occupancy<64, T, true>() : tc_sk_occupancy<64, T, false>();
+  return paged ? tc_sk_occupancy<128, T, true>() : tc_sk_occupancy<128, T, false>();
+}
+
 template <int D, int NT, bool PAGED>
 int fp8_occupancy() {
   static int occ = 0;
@@ -493,6 +533,27 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
   pl.row_blocks = kvc::ceil_div(rows, pl.R);
   // Persistent stream-K for up to 16 rows per KV head: the per-CTA partial
   // slots need no split size and every CTA streams the same bytes.
+  long long cap = c->max_T;
+  if (c->paged) cap = std::min<long long>(cap, (long long)max_pages * c->page_size);
+  const int tc_max_batch = c->D == 64 ? kvc::TcSkCfg<64>::kMaxBatch
+                                      : kvc::TcSkCfg<128>::kMaxBatch;
+  if (KVC_TC_STREAMK && pl.tc && c->B <= tc_max_batch && window == 0) {
+    pl.streamk = true;
+    const int socc = c->dtype == KVC_BF16 ? tc_sk_occ<__nv_bfloat16>(c->D, c->paged)
+                                          : tc_sk_occ<__half>(c->D, c->paged);
+    // no more CTAs than there can be tiles (penalties included)
+    const long long wt_max = (long long)c->B * c->H_kv * pl.row_blocks *
+                             ((cap + tile - 1) / tile + KVC_TC_SK_PENALTY);
+    pl.grid = (int)std::max<long long>(1, std::min<long long>((long long)c->num_sms * socc,
+                                                              wt_max));
+    pl.slots = (size_t)pl.grid * 2;
+    pl.split_tokens = 1 << 30;
+    pl.num_splits = 1;
+    pl.ws_partial_floats = (size_t)pl.grid * 2 * pl.R * (c->D + 1);
+    pl.ws_counters = (size_t)c->B * c->H_kv * pl.row_blocks;
+    pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
+    return pl;
+  }
   const int max_batch = c->D == 64 ? kvc::StreamKCfg<64>::kMaxBatch
                                    : kvc::StreamKCfg<128>::kMaxBatch;
   if (pl.mma && pl.NT <= 2 && c->B <= max_batch && window == 0) {
@@ -508,8 +569,6 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
     pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
     return pl;
   }
-  long long cap = c->max_T;
-  if (c->paged) cap = std::min<long long>(cap, (long long)max_pages * c->page_size);
   if (window > 0)  // a block reads at most its sink tiles and W + T_new positions (+ a tile)
     cap = std::min<long long>(cap, (long long)(sink + tile - 1) / tile * tile + window + T_new +
                                        tile);
@@ -700,6 +759,35 @@ kvc_status launch_attend_tc(const kvc::AttendParams& p, const CUtensorMap& tk,
   return cuda_status(cudaGetLastError());
 }
 
+template <int D, typename T, bool PAGED>
+kvc_status launch_attend_tc_streamk(const kvc::AttendParams& p, int grid, bool pdl,
+                                    const CUtensorMap& tk, const CUtensorMap& tv,
+                                    cudaStream_t stream) {
+  tc_sk_occupancy<D, T, PAGED>();  // sets the shared-memory attribute once
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kvc::TcCfg<D>::kThreads);
+  cfg.dynamicSmemBytes = kvc::TcSkCfg<D>::smem_bytes();
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cuda_status(
+      cudaLaunchKernelEx(&cfg, kvc::attend_tc_streamk_kernel<D, T, PAGED>, p, tk, tv));
+}
+
+template <typename T>
+kvc_status dispatch_tc_streamk(const kvc::AttendParams& p, int D, bool paged, int grid, bool pdl,
+                               const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  if (D == 64)
+    return paged ? launch_attend_tc_streamk<64, T, true>(p, grid, pdl, tk, tv, s)
+                 : launch_attend_tc_streamk<64, T, false>(p, grid, pdl, tk, tv, s);
+  return paged ? launch_attend_tc_streamk<128, T, true>(p, grid, pdl, tk, tv, s)
+               : launch_attend_tc_streamk<128, T, false>(p, grid, pdl, tk, tv, s);
+}
+
 template <typename T>
 kvc_status dispatch_tc(const kvc::AttendParams& p, int D, bool paged, const CUtensorMap& tk,
                        const CUtensorMap& tv, cudaStream_t s) {
@@ -764,8 +852,11 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
   p.row_blocks = pl.row_blocks;
   p.err = c->d_err;
   p.wait_limit_ns = c->wait_limit_ns;
-  p.sk_penalty = !pl.streamk ? 0 : c->D == 128 ? KVC_SK_PENALTY_D128 : KVC_SK_PENALTY_D64;
-  p.sk_blocked = pl.streamk && c->tma4 ? 1 : 0;
+  p.sk_penalty = !pl.streamk ? 0
+                 : pl.tc      ? KVC_TC_SK_PENALTY
+                 : c->D == 128 ? KVC_SK_PENALTY_D128
+                              : KVC_SK_PENALTY_D64;
+  p.sk_blocked = pl.streamk && !pl.tc && c->tma4 ? 1 : 0;
   p.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   return p;
@@ -790,6 +881,12 @@ kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::At
                     : dispatch_fp8_nt<128, false>(p, sc, pl.NT, c->tmk[layer], c->tmv[layer], s);
   }
   const bool bf = c->dtype == KVC_BF16;
+  if (pl.tc && pl.streamk)
+    return bf ? dispatch_tc_streamk<__nv_bfloat16>(p, c->D, c->paged, pl.grid,
+                                                   c->dependent_launch, c->tmk[layer],
+                                                   c->tmv[layer], s)
+              : dispatch_tc_streamk<__half>(p, c->D, c->paged, pl.grid, c->dependent_launch,
+                                            c->tmk[layer], c->tmv[layer], s);
   if (pl.tc)
     return bf ? dispatch_tc<__nv_bfloat16>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s)
               : dispatch_tc<__half>(p, c->D, c->paged, c->tmk[layer], c->tmv[layer], s);
@@ -1296,7 +1393,7 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
   if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
-  if (!pl.streamk) {
+  if (!pl.streamk || pl.tc) {  // only the mma.sync stream-K kernel fuses the append
     kvc_status st = kvc_append(c, layer, k_new, v_new, T_new, block_table, max_pages,
                                seq_lens, stream);
     if (st != KVC_OK) return st;

@@ -7,8 +7,8 @@ allocation can fail or fragment its pool), a latency-bound loop that cannot take
 the synchronisation a free implies.  It runs the same plan and the same kernels as
 kvc_attend with its split-K scratch in a fixed 16 MiB device array of the library.
 
-Here every kernel family -- persistent stream-K, fixed split-K on mma.sync
-tensor cores, tcgen05, the CUDA-core kernel and the FP8 kernel -- is called twice
+Here every kernel family -- persistent stream-K on mma.sync and on tcgen05, fixed
+split-K on mma.sync, the CUDA-core kernel and the FP8 kernel -- is called twice
 in a row through the new entry point.  Each case first checks that the plan takes
 the intended kernel with more than one slice (so the scratch is really used).  The
 two outputs must be byte-identical to kvc_attend's (same plan, same kernels,
@@ -58,9 +58,9 @@ CASES = {
     # fixed split-K on mma.sync: 32 rows per KV head (a GQA verify chunk)
     "splitk_mma_verify": (lambda: W.paged_case("na_mma", 4, 16, 2, 128, "bf16", 4, 1000, 4000,
                                                16, seed=93, pool_seed=94), "native", "split"),
-    # tcgen05: MQA verify, 128 rows per KV head, about 2K tokens of context
-    "splitk_tcgen05_mqa": (lambda: W.contig_case("na_tc", 2, 32, 1, 128, "bf16", 4, 2100,
-                                                 seed=97), "native", "split"),
+    # persistent stream-K on tcgen05: MQA verify, 128 rows per KV head, about 2K tokens
+    "streamk_tcgen05_mqa": (lambda: W.contig_case("na_tc", 2, 32, 1, 128, "bf16", 4, 2100,
+                                                  seed=97), "native", "streamk"),
     # CUDA-core kernel (D = 32 has no tensor maps), several slices per head
     "splitk_simt_d32": (lambda: W.contig_case("na_simt", 2, 16, 16, 32, "fp16", 1, 6000,
                                               seed=95), "native", "split"),
@@ -143,8 +143,9 @@ def test_noalloc_matches_attend_twice_in_a_row(name):
 
 
 def test_noalloc_rejects_plans_beyond_its_scratch():
-    """MQA verify of 64 requests over 32K-token page tables needs 17-25 MB of split-K
-    scratch (by occupancy): rejected with KVC_ERR_SCRATCH on the host, before any launch."""
+    """MQA verify of 64 requests over 32K-token page tables needs about 39 MB of partial
+    slots (two 128-row slots for each of the 296 persistent CTAs): rejected with
+    KVC_ERR_SCRATCH on the host, before any launch."""
     B, H_q, T_new, max_pages = 64, 32, 8, 2049
     cache = kvc.KVCache(B, 1, 128, max_pages * 16, "bf16", page_size=16, num_layers=1,
                         num_pages=64)
