@@ -120,7 +120,7 @@ def attend_kernel_name(c: W.Case, kv_format: str, split_tokens: int) -> str:
     layout = "paged" if c.paged else "contiguous"
     if kv_format == "fp8":
         return f"attend_fp8_kernel<{c.D},{layout}>"
-    if rows >= 64 and c.D in (64, 128):
+    if rows >= 17 and c.D in (64, 128):
         if split_tokens == 0:
             return f"attend_tc_streamk_kernel<{c.D},{c.dtype},{layout}>"
         return f"attend_tc_kernel<{c.D},{c.dtype},{layout}>"

@@ -219,7 +219,7 @@ struct RangeMap {
 };
 
 // Merge the partial pieces rf..rl of one segment (the CTA's rows r0.., nr of them
-// valid, outputs from row_base) by log-sum-exp:
+// valid, outputs from row_base; slots of p.sk_slot_rows rows) by log-sum-exp:
 //     out = sum_q 2^(lse_q - M) o_q / sum_q 2^(lse_q - M),   M = max_q lse_q.
 // Piece q lives in workspace slot 2*(rf+q) + 1 if it is the first piece and range rf
 // began before the segment (its penalty tiles, before s0), else 2*(rf+q).  Each output quad (4 consecutive
@@ -261,8 +261,9 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
         const int q = q0 + u * tpq;
         if (q < npc) {
           const size_t slot = (size_t)(rf + q) * 2 + ((q == 0 && rf_mid) ? 1 : 0);
-          ls[u] = __ldcg(p.ws_lse + slot * R + rr);
-          v[u] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (slot * R + rr) * D + d));
+          ls[u] = __ldcg(p.ws_lse + slot * p.sk_slot_rows + rr);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (slot * p.sk_slot_rows + rr) * D +
+                                                        d));
         } else {
           ls[u] = -INFINITY;
           v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1004,8 +1005,8 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
     T* out = static_cast<T*>(p.out);
     const size_t row_base =
         ((size_t)cur.b * p.H_q + (size_t)cur.g * p.group) * p.T_new + r0;
-    float* wso = p.ws_o + ((size_t)c * 2 + slot) * R * D;
-    float* wsl = p.ws_lse + ((size_t)c * 2 + slot) * R;
+    float* wso = p.ws_o + ((size_t)c * 2 + slot) * p.sk_slot_rows * D;
+    float* wsl = p.ws_lse + ((size_t)c * 2 + slot) * p.sk_slot_rows;
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int idx = tid + k * NTH;

@@ -43,9 +43,17 @@ struct TcSkCfg {
   using C = TcCfg<D>;
   // K full/empty, V full/empty, s_full x2, p_full x2, o_done x2, q_full, drain
   static constexpr int kBarriers = 2 * C::kKStages + 2 * C::kVStages + 8;
+  // after the barriers: the TMEM slot (16 bytes), then 32 ints of flags: [0] abort,
+  // [1] last finisher, [2] final merge pending, [4..7] two merge mbarriers, [8..14] scan
+  // sums, [16..23] the final merge's parameters
   static constexpr size_t smem_bytes() {
-    return C::kData + kBarriers * sizeof(uint64_t) + 16 + 16 * sizeof(int);
+    return C::kData + kBarriers * sizeof(uint64_t) + 16 + 32 * sizeof(int);
   }
+  // the final merge's weights: up to kMergeMaxPieces pieces of 128 rows at the end of the
+  // operand area; the rest holds two windows of partial rows
+  static constexpr int kMergeMaxPieces = 32;
+  static constexpr int kMergeWeightBytes = C::kRows * kMergeMaxPieces * (int)sizeof(float);
+  static constexpr int kMergeHalf = ((C::kData - kMergeWeightBytes) / 2) & ~15;
   // the plan's scan (tile prefix and lengths, 2B + 1 ints) uses the K/V rings before any copy
   static constexpr int kMaxBatch = ((C::kKRing + C::kVRing) / (int)sizeof(int) - 1) / 2;
 };
@@ -149,6 +157,106 @@ __device__ __forceinline__ SkRange<R> sk_plan(const AttendParams& p, int* P, int
   return r;
 }
 
+// The last finisher's merge of a segment's pieces rf..rl at the end of its range, by all
+// of the CTA's threads, with the operand area (`smem`, TcCfg<D>::kData bytes) free:
+//   1. every (row, piece) weight 2^(lse - M) / sum, once, into the area's last bytes;
+//   2. the pieces' partial rows streamed through two shared-memory windows of bulk copies
+//      (each window RC rows of every piece), the next window loading while this one is
+//      summed.
+// More pieces than the weight area holds fall back to merge_pieces_spread.  Waits are
+// bounded; after one runs out the merge finishes on garbage and KVC_ERR_TIMEOUT stands.
+template <typename T, int D>
+__device__ __forceinline__ void tc_merge_final(const AttendParams& p, const RangeMap& rm,
+                                               long long rf, long long rl, long long s0, int nr,
+                                               size_t row_base, unsigned char* smem,
+                                               uint64_t* mbar, unsigned long long wait_limit) {
+  using C = TcCfg<D>;
+  using S = TcSkCfg<D>;
+  constexpr int R = C::kRows;
+  constexpr int NTH = C::kThreads;
+  constexpr int Q4 = D / 4;
+  const int tid = threadIdx.x;
+  const int npc = (int)(rl - rf + 1);
+  if (npc > S::kMergeMaxPieces) {
+    merge_pieces_spread<T, D, R, NTH>(p, rm, rf, rl, s0, nr, row_base);
+    return;
+  }
+  const bool rf_mid = rm.start(rf) < s0 - p.sk_penalty;
+  auto slot_of = [&](int q) -> size_t {
+    return (size_t)(rf + q) * 2 + ((q == 0 && rf_mid) ? 1 : 0);
+  };
+  float* w = reinterpret_cast<float*>(smem + C::kData - S::kMergeWeightBytes);  // [row][piece]
+  // 1. weights
+#pragma unroll 1
+  for (int idx = tid; idx < nr * npc; idx += NTH) {
+    const int rr = idx / npc, q = idx - rr * npc;
+    w[idx] = __ldcg(p.ws_lse + slot_of(q) * p.sk_slot_rows + rr);
+  }
+  __syncthreads();
+  if (tid < nr) {
+    float* wr = w + tid * npc;
+    float M = -INFINITY;
+    for (int q = 0; q < npc; ++q) M = fmaxf(M, wr[q]);
+    float den = 0.f;
+    for (int q = 0; q < npc; ++q) {
+      wr[q] = wr[q] == -INFINITY ? 0.f : exp2f(wr[q] - M);
+      den += wr[q];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int q = 0; q < npc; ++q) wr[q] *= inv;
+  }
+  // 2. the partial rows, RC rows of every piece per window
+  const int RC = min(nr, S::kMergeHalf / (npc * D * (int)sizeof(float)));
+  const int nwin = ceil_div(nr, RC);
+  auto issue = [&](int win) {  // thread 0
+    const int half = win & 1;
+    const int r0 = win * RC;
+    const uint32_t bytes = (uint32_t)min(RC, nr - r0) * D * sizeof(float);
+    mbar_arrive_expect_tx(&mbar[half], bytes * npc);
+    for (int q = 0; q < npc; ++q)
+      bulk_g2s(smem + half * S::kMergeHalf + (size_t)q * RC * D * sizeof(float),
+               p.ws_o + (slot_of(q) * p.sk_slot_rows + r0) * D, bytes, &mbar[half]);
+  };
+  if (tid == 0) {
+    // the partials were written by other CTAs through the generic proxy and acquired by
+    // the ticket: order them before the bulk copies' async-proxy reads
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    issue(0);
+    if (nwin > 1) issue(1);
+  }
+  __syncthreads();  // the weights are complete
+  T* out = static_cast<T*>(p.out);
+#pragma unroll 1
+  for (int win = 0; win < nwin; ++win) {
+    const int half = win & 1;
+    const int r0 = win * RC;
+    const int rows = min(RC, nr - r0);
+    mbar_wait(&mbar[half], (win >> 1) & 1, p.err, wait_limit);
+    const float* buf = reinterpret_cast<const float*>(smem + half * S::kMergeHalf);
+#pragma unroll 1
+    for (int e = tid; e < rows * Q4; e += NTH) {
+      const int rr = e / Q4;
+      const int d = (e - rr * Q4) * 4;
+      const float* wr = w + (r0 + rr) * npc;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int q = 0; q < npc; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(buf + ((size_t)q * RC + rr) * D + d);
+        const float wq = wr[q];
+        a.x = fmaf(wq, v.x, a.x);
+        a.y = fmaf(wq, v.y, a.y);
+        a.z = fmaf(wq, v.z, a.z);
+        a.w = fmaf(wq, v.w, a.w);
+      }
+      T* o = out + (row_base + r0 + rr) * D + d;
+      const uint2 packed = make_uint2(Elt<T>::pack2(a.x, a.y), Elt<T>::pack2(a.z, a.w));
+      *reinterpret_cast<uint2*>(o) = packed;
+    }
+    __syncthreads();  // the window is read: it may be refilled
+    if (tid == 0 && win + 2 < nwin) issue(win + 2);
+  }
+}
+
 template <int D, typename T, bool PAGED>
 __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     attend_tc_streamk_kernel(const AttendParams p, const __grid_constant__ CUtensorMap tmk,
@@ -174,7 +282,9 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
   uint64_t* q_full = o_done + 2;    // a piece's Q is staged (NSM arrivals; O was read)
   uint64_t* dbar = q_full + 1;      // drain after an abort
   uint32_t* tslot = reinterpret_cast<uint32_t*>(dbar + 1);
-  int* flags = reinterpret_cast<int*>(tslot + 4);  // [0] abort [1] last [8..14] scan sums
+  int* flags = reinterpret_cast<int*>(tslot + 4);  // see TcSkCfg::smem_bytes
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(flags + 4);      // [2] final merge windows
+  long long* fm = reinterpret_cast<long long*>(flags + 16);     // final merge parameters
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -210,6 +320,9 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     mbar_init(dbar, 1);
     flags[0] = 0;
     flags[1] = 0;
+    flags[2] = 0;
+    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[1], 1);
     fence_barrier_init();
   }
   tc_fence_before();
@@ -495,7 +608,7 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
         const size_t row_base =
             ((size_t)sc.b * p.H_q + (size_t)sc.g * p.group) * p.T_new + r0;
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float* wso = p.ws_o + (((size_t)c * 2 + slot) * R + tid) * D;
+        float* wso = p.ws_o + (((size_t)c * 2 + slot) * p.sk_slot_rows + tid) * D;
         T* orow = out + (row_base + tid) * D;
 #pragma unroll 1
         for (int c16 = 0; c16 < D / 16; ++c16) {
@@ -518,7 +631,8 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
           }
         }
         if (!whole && tid < nr)
-          p.ws_lse[((size_t)c * 2 + slot) * R + tid] = l > 0.f ? m_ref + log2f(l) : -INFINITY;
+          p.ws_lse[((size_t)c * 2 + slot) * p.sk_slot_rows + tid] =
+              l > 0.f ? m_ref + log2f(l) : -INFINITY;
         // The row's O is read: staging the next piece's Q hands TMEM back to the MMA issuer.
         if (j + 1 < rg.ntiles) {
           TileCursor<R> nc = sc;
@@ -534,11 +648,21 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
           int* ticket = p.counters + ((size_t)sc.b * p.H_kv + sc.g) * p.row_blocks + sc.rb;
           if (tid == 0) flags[1] = ticket_add_acq_rel(ticket) == (int)(rl - rf);
           named_barrier_sync(1, NSM);
-          if (flags[1]) {
-            merge_pieces_spread<T, D, R, NSM>(p, rm, rf, rl, s0, nr, row_base);
-            if (tid == 0) *ticket = 0;
+          if (j + 1 < rg.ntiles) {  // mid-range: the softmax threads merge at once
+            if (flags[1]) {
+              merge_pieces_spread<T, D, R, NSM>(p, rm, rf, rl, s0, nr, row_base);
+              if (tid == 0) *ticket = 0;
+            }
+            named_barrier_sync(1, NSM);  // flags[1] is read by every thread before reuse
+          } else if (tid == 0 && flags[1]) {
+            // the range's last piece: every thread of the CTA merges after the loops, with
+            // the operand area free for staging (tc_merge_final)
+            flags[2] = 1;
+            fm[0] = s0;
+            fm[1] = (long long)row_base;
+            fm[2] = rf | (rl << 32);
+            fm[3] = nr | ((long long)(ticket - p.counters) << 32);
           }
-          named_barrier_sync(1, NSM);  // flags[1] is read by every thread before it is reused
         }
       }
       sc.next(p, PAGED);
@@ -546,6 +670,14 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
   }
 
   const bool bad = __syncthreads_or(*abort_word != 0);
+  if (!bad && flags[2]) {  // every copy and MMA has completed: the operand area is free
+    RangeMap frm;
+    frm.W = rg.Wt;
+    frm.G = rg.G;
+    tc_merge_final<T, D>(p, frm, fm[2] & 0xffffffffll, fm[2] >> 32, fm[0],
+                         (int)(fm[3] & 0xffffffffll), (size_t)fm[1], smem, mbar, wait_limit);
+    if (tid == 0) p.counters[fm[3] >> 32] = 0;  // the ticket, ready for the next launch
+  }
   if (bad) {
     if ((warp == C::kKWarp || warp == C::kVWarp) && lane_id == 0) {  // loads in flight
       const int NS = warp == C::kKWarp ? SK : SV;

@@ -66,9 +66,12 @@ constexpr int kEltBytes = 2;
 #define KVC_MMA_MIN_ROWS 1
 #endif
 
-// Query rows per KV head from which the tcgen05 kernel (128-row blocks) takes over.
+// Query rows per KV head from which the tcgen05 kernel (128-row blocks) takes over.  From
+// 17 rows the persistent tcgen05 kernel beats the mma.sync kernels even with most of the
+// MMA's 128 rows idle (GQA verify gamma 8, 32 rows: 69 % of HBM against 33 % on the
+// fixed-split mma.sync kernel); up to 16 rows the mma.sync stream-K kernel is faster.
 #ifndef KVC_TC_MIN_ROWS
-#define KVC_TC_MIN_ROWS 64
+#define KVC_TC_MIN_ROWS 17
 #endif
 
 // Split-K sizing: aim for this many waves of resident CTAs, so that the last
@@ -435,7 +438,8 @@ struct Plan {
   bool mma;          // mma.sync tensor-core kernel (else the CUDA-core kernel)
   bool streamk;      // mma: persistent stream-K kernel (grid = resident CTAs)
   int grid;          // streamk: persistent CTAs
-  size_t slots;      // streamk: partial-result slots (R rows x D each) in the workspace
+  size_t slots;      // streamk: partial-result slots (slot_rows rows x D each) in the workspace
+  int slot_rows;     // streamk: rows of a slot
   int NT;            // mma: 8-row n-tiles per CTA
   int R;             // query rows per CTA
   int row_blocks;    // CTAs per KV head along the rows
@@ -497,9 +501,8 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
                int sink = 0) {
   Plan pl{};
   const int rows = (H_q / c->H_kv) * T_new;
-  // Three or more query rows per K/V row make q.k and p.v a dense contraction
-  // worth the tensor cores; one or two rows stay on CUDA cores.
-  // From KVC_TC_MIN_ROWS rows a 128-row block fills the tcgen05 MMA's M.
+  // Tensor cores from KVC_MMA_MIN_ROWS query rows per K/V row (mma.sync), tcgen05 from
+  // KVC_TC_MIN_ROWS (a 128-row block as the MMA's M).
   pl.fp8 = c->fp8;
   pl.tc = !c->fp8 && c->tma && rows >= KVC_TC_MIN_ROWS;
   pl.mma = !c->fp8 && c->tma && rows >= KVC_MMA_MIN_ROWS && !pl.tc;
@@ -547,9 +550,10 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
     pl.grid = (int)std::max<long long>(1, std::min<long long>((long long)c->num_sms * socc,
                                                               wt_max));
     pl.slots = (size_t)pl.grid * 2;
+    pl.slot_rows = std::min(pl.R, rows);  // no more rows of a block can be valid
     pl.split_tokens = 1 << 30;
     pl.num_splits = 1;
-    pl.ws_partial_floats = (size_t)pl.grid * 2 * pl.R * (c->D + 1);
+    pl.ws_partial_floats = pl.slots * pl.slot_rows * (c->D + 1);
     pl.ws_counters = (size_t)c->B * c->H_kv * pl.row_blocks;
     pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
     return pl;
@@ -562,9 +566,10 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
                                           : streamk_occ<__half>(c->D, pl.NT, c->paged);
     pl.grid = c->num_sms * socc;
     pl.slots = (size_t)pl.grid * 2;
+    pl.slot_rows = pl.R;
     pl.split_tokens = 1 << 30;  // unused by the stream-K kernel
     pl.num_splits = 1;
-    pl.ws_partial_floats = (size_t)pl.grid * 2 * pl.R * (c->D + 1);
+    pl.ws_partial_floats = pl.slots * pl.slot_rows * (c->D + 1);
     pl.ws_counters = (size_t)c->B * c->H_kv * pl.row_blocks;
     pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
     return pl;
@@ -857,6 +862,7 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
                  : c->D == 128 ? KVC_SK_PENALTY_D128
                               : KVC_SK_PENALTY_D64;
   p.sk_blocked = pl.streamk && !pl.tc && c->tma4 ? 1 : 0;
+  p.sk_slot_rows = pl.slot_rows;
   p.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   return p;
@@ -865,7 +871,7 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
 // Where a plan's partial results start in a workspace of partial outputs then lse.
 float* lse_base(const kvc_cache* c, const Plan& pl, float* ws, int H_q, int T_new) {
   if (!ws) return nullptr;
-  return pl.streamk ? ws + pl.slots * pl.R * c->D
+  return pl.streamk ? ws + pl.slots * pl.slot_rows * c->D
                     : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
 }
 

@@ -47,6 +47,8 @@ struct AttendParams {
   int* err;
   unsigned long long wait_limit_ns;  // bound of every pipeline wait (0: the default, 1 s)
   int sk_penalty;  // stream-K: virtual tiles charged for each segment a CTA enters
+  int sk_slot_rows;  // stream-K: rows of one partial-result slot (the rows of a row block
+                     // that can be valid: min(rows per CTA, query rows per KV head))
   int sk_blocked;  // stream-K, paged, D = 128, pages < 64 tokens: the tensor maps are 4-D
                    // (64 elements, page tokens, 2 halves, page blocks), one box a page
   int stall;  // failure-detection test: the producers issue no copies, so the first

@@ -7,9 +7,10 @@ allocation can fail or fragment its pool), a latency-bound loop that cannot take
 the synchronisation a free implies.  It runs the same plan and the same kernels as
 kvc_attend with its split-K scratch in a fixed 16 MiB device array of the library.
 
-Here every kernel family -- persistent stream-K on mma.sync and on tcgen05, fixed
-split-K on mma.sync, the CUDA-core kernel and the FP8 kernel -- is called twice
-in a row through the new entry point.  Each case first checks that the plan takes
+Here every kernel family an unwindowed attend can take -- persistent stream-K on
+mma.sync and on tcgen05, the CUDA-core kernel and the FP8 kernel (the fixed-split
+mma.sync and tcgen05 kernels serve only windowed calls) -- is called twice in a row
+through the new entry point.  Each case first checks that the plan takes
 the intended kernel with more than one slice (so the scratch is really used).  The
 two outputs must be byte-identical to kvc_attend's (same plan, same kernels,
 deterministic merge order), and within the parity tolerance of the fp64 oracle.  The
@@ -55,9 +56,11 @@ CASES = {
     "streamk_paged_gqa": (lambda: W.paged_case("na_sk", 8, 32, 8, 128, "bf16", 1, 300, 5000,
                                                16, seed=91, pool_seed=92, share_frac=0.25,
                                                share_tokens=256), "native", "streamk"),
-    # fixed split-K on mma.sync: 32 rows per KV head (a GQA verify chunk)
-    "splitk_mma_verify": (lambda: W.paged_case("na_mma", 4, 16, 2, 128, "bf16", 4, 1000, 4000,
-                                               16, seed=93, pool_seed=94), "native", "split"),
+    # persistent stream-K on tcgen05 with a quarter of the 128-row block used: 32 rows per
+    # KV head (a GQA verify chunk), paged
+    "streamk_tcgen05_gqa": (lambda: W.paged_case("na_gqa", 4, 16, 2, 128, "bf16", 4, 1000,
+                                                 4000, 16, seed=93, pool_seed=94), "native",
+                            "streamk"),
     # persistent stream-K on tcgen05: MQA verify, 128 rows per KV head, about 2K tokens
     "streamk_tcgen05_mqa": (lambda: W.contig_case("na_tc", 2, 32, 1, 128, "bf16", 4, 2100,
                                                   seed=97), "native", "streamk"),
