@@ -44,8 +44,8 @@ METRIC = ("decode-attention KV HBM GB/s (% of B200 peak) and tokens/s per layer-
 # The sources each profiled kernel is compiled from: a committed ncu summary stays
 # valid while these files are unchanged.
 KERNEL_SOURCES = {
-    "attend_streamk_kernel": ("attend_streamk.cuh", "splitk_epilogue.cuh", "device_common.cuh",
-                              "params.cuh"),
+    "attend_streamk_kernel": ("attend_streamk.cuh", "attend_fp8.cuh", "fp8.cuh",
+                              "splitk_epilogue.cuh", "device_common.cuh", "params.cuh"),
     "attend_mma_kernel": ("attend_mma.cuh", "splitk_epilogue.cuh", "window.cuh",
                           "device_common.cuh", "params.cuh"),
     "attend_tc_kernel": ("attend_tc.cuh", "splitk_epilogue.cuh", "window.cuh",
@@ -119,6 +119,8 @@ def attend_kernel_name(c: W.Case, kv_format: str, split_tokens: int) -> str:
     rows = (c.H_q // c.H_kv) * c.T_new
     layout = "paged" if c.paged else "contiguous"
     if kv_format == "fp8":
+        if split_tokens == 0:  # E4M3 stages in the stream-K kernel
+            return f"attend_streamk_kernel<{c.D},1,bf16,{layout},fp8>"
         return f"attend_fp8_kernel<{c.D},{layout}>"
     if rows >= 17 and c.D in (64, 128):
         if split_tokens == 0:

@@ -47,6 +47,7 @@
 #include <cuda.h>
 #include <math.h>
 
+#include "attend_fp8.cuh"
 #include "attend_mma.cuh"
 #include "device_common.cuh"
 #include "params.cuh"
@@ -54,6 +55,18 @@
 
 #ifndef KVC_SK_STAGES
 #define KVC_SK_STAGES 3
+#endif
+#ifndef KVC_SK_FP8_CHAINS  // FP8: independent S accumulator chains
+#define KVC_SK_FP8_CHAINS 2
+#endif
+#ifndef KVC_SK_FP8_MIN_BLOCKS  // FP8, D = 128: resident CTAs an SM (a register bound)
+#define KVC_SK_FP8_MIN_BLOCKS 3
+#endif
+#ifndef KVC_SK_STAGES_FP8  // FP8, D = 128: stages (3 CTAs of 3 stages fit an SM)
+#define KVC_SK_STAGES_FP8 3
+#endif
+#ifndef KVC_SK_STAGES_D64
+#define KVC_SK_STAGES_D64 KVC_SK_STAGES
 #endif
 // Tiles of its range a CTA prefetches into L2 before the dependency wait (measured:
 // 2 beats 0, 1, 3 and 5: more delays the CTAs that start late and competes with the
@@ -119,18 +132,25 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-template <int D>
+// FP8 = true: the cache holds E4M3 codes (one byte an element) and one fp32 scale per
+// (token, KV head); a stage then holds the K and V codes of a tile and their scales, and
+// twice as many stages keep the same bytes in flight.
+template <int D, bool FP8 = false>
 struct StreamKCfg {
   static constexpr int kWarps = 4;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kTile = 64;
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = kTile * 128;
-  static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStages = KVC_SK_STAGES;
+  static constexpr int kTileBytes = kTile * D * (FP8 ? 1 : 2);  // K (equally V) of a stage
+  static constexpr int kScaleBytes = FP8 ? 2 * kTile * 4 : 0;   // K and V scales of a stage
+  // FP8: half-size stages; the conversions make the tile arithmetic latency-bound, so
+  // D = 128 trades depth for a third resident CTA (3 x 3 stages an SM)
+  static constexpr int kStages =
+      FP8 ? (D == 128 ? KVC_SK_STAGES_FP8 : 6) : (D == 64 ? KVC_SK_STAGES_D64 : KVC_SK_STAGES);
   static constexpr int kKSteps = D / 16;
   static constexpr int kMTiles = D / 16;
-  static constexpr int kRing = 2 * kStages * kTileBytes;
+  static constexpr int kRing = 2 * kStages * kTileBytes + kStages * kScaleBytes;
 
   template <int NT>
   static constexpr size_t smem_bytes() {
@@ -143,11 +163,15 @@ struct StreamKCfg {
   // a register bound for the compiler
   template <int NT>
   static constexpr int min_blocks() {
-    return D == 64 ? (NT == 1 ? 4 : 3) : 2;
+    return FP8 ? (D == 64 ? 3 : KVC_SK_FP8_MIN_BLOCKS) : D == 64 ? (KVC_SK_STAGES_D64 <= 3 ? (NT == 1 ? 4 : 3) : 2) : 2;
   }
   // the block scan of per-request tile counts and the lengths it read use the ring
   // before the first copy
   static constexpr int kMaxBatch = (kRing / (int)sizeof(int) - 1) / 2;
+  // the piece epilogue's W x 8NT x D fp32 partials live in one stage's K and V buffers
+  static_assert(!FP8 || kWarps * 8 * D * 4 <= 2 * kTileBytes, "FP8: one row group of 8");
+  static_assert(!FP8 || D == 64 || KVC_SK_FP8_MIN_BLOCKS * (smem_bytes<1>() + 1024) <= 233472,
+                "FP8 D = 128: the resident CTAs must fit an SM's shared memory");
 };
 
 // Row-block geometry: new-row indices covered by row block rb.
@@ -320,11 +344,16 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
   }
 }
 
-template <int D, int NT, typename T, bool PAGED>
-__global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::template min_blocks<NT>())
+// FP8 = true (NT 1, bf16 q and out): the stages carry E4M3 codes and scales and the
+// tile arithmetic is that of attend_fp8.cuh (codes converted in registers, two running
+// maxima); planning, the ring, pieces, epilogue and merge are the same.
+template <int D, int NT, typename T, bool PAGED, bool FP8 = false>
+__global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
+                                  StreamKCfg<D, FP8>::template min_blocks<NT>())
     attend_streamk_kernel(const AttendParams p, const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv) {
-  using C = StreamKCfg<D>;
+  using C = StreamKCfg<D, FP8>;
+  static_assert(!FP8 || (NT == 1 && Elt<T>::kCode == KVC_BF16), "FP8: 1-8 rows, bf16");
   constexpr int W = C::kWarps;
   constexpr int NTH = C::kThreads;
   constexpr int R = NT * 8;
@@ -333,6 +362,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sk = smem;
   unsigned char* sv = smem + C::kStages * C::kTileBytes;
+  float* scl = reinterpret_cast<float*>(smem + 2 * C::kStages * C::kTileBytes);  // FP8: [st][K|V]
   unsigned char* sq = smem + C::kRing;  // [stage][R][D]
   float* red_m = reinterpret_cast<float*>(sq + C::kStages * R * D * 2);
   float* red_l = red_m + W * R;
@@ -522,14 +552,18 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
       if (i >= pf) break;  // no tiles prefetched: q only
       if (!PAGED) {
         const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
-        if (lane < C::kHalves && y + C::kTile <= rows_total) {
+        // FP8 code maps: one box of D bytes a row
+        if (lane < (FP8 ? 1 : C::kHalves) && y + C::kTile <= rows_total) {
           tma_prefetch_2d(&tmk, lane * 64, y);
           tma_prefetch_2d(&tmv, lane * 64, y);
         }
       } else if (lane < nbox) {
         const int y = box_page_row(pc, lane, lookup_page(pc, lane));
         if (y >= 0 && y != beyond && y + box_rows <= rows_total) {
-          if (blocked) {
+          if (FP8) {
+            tma_prefetch_2d(&tmk, 0, y);
+            tma_prefetch_2d(&tmv, 0, y);
+          } else if (blocked) {
             tma_prefetch_4d(&tmk, 0, 0, 0, y >> p.page_shift);
             tma_prefetch_4d(&tmv, 0, 0, 0, y >> p.page_shift);
           } else {
@@ -605,7 +639,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
     const int nr = min(R, p.rows - r0);
     const uint32_t qbytes = first ? (uint32_t)nr * D * 2 : 0u;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes + qbytes);
+      mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes + C::kScaleBytes + qbytes);
       if (first) {
         const char* qsrc = static_cast<const char*>(p.q) +
                            ((((size_t)pc.b * p.H_q + (size_t)pc.g * p.group) * p.T_new) + r0) *
@@ -616,7 +650,33 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
     __syncwarp();
     unsigned char* dk = sk + st * C::kTileBytes;
     unsigned char* dv = sv + st * C::kTileBytes;
-    if (!PAGED) {
+    if constexpr (FP8) {  // codes: one box of D bytes a row; scales: 1-D bulk copies
+      float* ds = scl + st * 2 * C::kTile;
+      if (!PAGED) {
+        const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
+        if (lane == 0) {
+          tma_load_2d(dk, &tmk, 0, y, &full[st], pol);
+          tma_load_2d(dv, &tmv, 0, y, &full[st], pol);
+        } else if (lane == 1) {  // T_pad holds whole tiles
+          const size_t srow = ((size_t)pc.b * p.H_kv + pc.g) * p.T_pad + pc.k * C::kTile;
+          bulk_g2s_hint(ds, p.k_scales + srow, C::kTile * 4, &full[st], pol);
+          bulk_g2s_hint(ds + C::kTile, p.v_scales + srow, C::kTile * 4, &full[st], pol);
+        }
+      } else if (lane < nbox) {
+        int y = box_page_row(pc, lane, ids[0]);
+        if (y < 0) {  // a page id outside the pool: zero fill, reported
+          flag_error(p.err, KVC_ERR_BOUNDS);
+          y = beyond;
+        }
+        // past the segment (zero codes): any finite scales, row 0's
+        const size_t srow = y == beyond ? 0 : (size_t)y;
+        const int off = lane * box_rows;
+        tma_load_2d(dk + off * D, &tmk, 0, y, &full[st], pol);
+        tma_load_2d(dv + off * D, &tmv, 0, y, &full[st], pol);
+        bulk_g2s_hint(ds + off, p.k_scales + srow, box_rows * 4, &full[st], pol);
+        bulk_g2s_hint(ds + C::kTile + off, p.v_scales + srow, box_rows * 4, &full[st], pol);
+      }
+    } else if (!PAGED) {
       if (lane < C::kHalves) {
         const int y = (pc.b * p.H_kv + pc.g) * p.max_T + pc.k * C::kTile;
         tma_load_2d(dk + lane * C::kBoxBytes, &tmk, lane * 64, y, &full[st], pol);
@@ -706,6 +766,8 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
   int vis[NT][2];
   int r0 = 0, nr = 0, vis_min = 0, piece_first_j = 0;
   float m[NT][2], l[NT][2];
+  float mo[NT][2];    // FP8: the running maximum of s + log2(v_scale), the weights' reference
+  float fcol[NT][2];  // FP8: score factor of the column's row: scale * log2(e) * 2^e_row
   float o[C::kMTiles][NT][4];
   // fresh running state; reset again at the end of every piece
   auto reset_state = [&]() {
@@ -714,6 +776,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         m[nt][cc] = -INFINITY;
+        mo[nt][cc] = -INFINITY;
         l[nt][cc] = 0.f;
       }
 #pragma unroll
@@ -762,15 +825,51 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int row = nt * 8 + (lane >> 2);
+        if constexpr (FP8) {
+          // f16 fragments of row / 2^e (e puts the row's largest |q| in [2^14, 2^15);
+          // exact), under the k permutation of the converted K codes (attend_fp8.cuh):
+          // k = 2c, 2c+1 <-> d = 16kk + 4c, +1; k = 8+2c, 9+2c <-> d = 16kk + 4c + 2, +3
+          float qv[C::kKSteps][4];
+          float amax = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < C::kKSteps; ++kk) {
-          if (row < nr) {
-            const unsigned char* src = qs + row * D * 2 + (kk * 16 + (lane & 3) * 2) * 2;
-            qb[kk][nt][0] = *reinterpret_cast<const uint32_t*>(src);
-            qb[kk][nt][1] = *reinterpret_cast<const uint32_t*>(src + 16);
-          } else {
-            qb[kk][nt][0] = 0u;
-            qb[kk][nt][1] = 0u;
+          for (int kk = 0; kk < C::kKSteps; ++kk) {
+            uint2 w = make_uint2(0u, 0u);
+            if (row < nr)
+              w = *reinterpret_cast<const uint2*>(qs + row * D * 2 + (kk * 16 + (lane & 3) * 4) * 2);
+            qv[kk][0] = __uint_as_float(w.x << 16);
+            qv[kk][1] = __uint_as_float(w.x & 0xFFFF0000u);
+            qv[kk][2] = __uint_as_float(w.y << 16);
+            qv[kk][3] = __uint_as_float(w.y & 0xFFFF0000u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[kk][e]));
+          }
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+          const int e =
+              amax > 0.f ? max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14, -126) : 0;
+          const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk) {
+            qb[kk][nt][0] = f32x2_to_f16x2(qv[kk][0] * inv, qv[kk][1] * inv);
+            qb[kk][nt][1] = f32x2_to_f16x2(qv[kk][2] * inv, qv[kk][3] * inv);
+          }
+          // the exponent of column row nt*8 + 2(lane%4) + cc is held by lane 4 (row % 8)
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int ec = __shfl_sync(0xffffffffu, e, (((lane & 3) * 2 + cc) & 7) << 2);
+            fcol[nt][cc] = p.scale_log2 * __uint_as_float((uint32_t)(127 + ec) << 23);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk) {
+            if (row < nr) {
+              const unsigned char* src = qs + row * D * 2 + (kk * 16 + (lane & 3) * 2) * 2;
+              qb[kk][nt][0] = *reinterpret_cast<const uint32_t*>(src);
+              qb[kk][nt][1] = *reinterpret_cast<const uint32_t*>(src + 16);
+            } else {
+              qb[kk][nt][0] = 0u;
+              qb[kk][nt][1] = 0u;
+            }
           }
         }
 #pragma unroll
@@ -784,7 +883,7 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
     // Fused append: the tile that holds the new positions takes them from
     // k_new / v_new (its copy from the pool may predate them) and the first row
     // block writes them into the cache; every other tile is untouched.
-    if (p.k_new != nullptr) {
+    if (!FP8 && p.k_new != nullptr) {
       const int ta = cur.k * C::kTile;
       const int n_lo = max(cur.L, ta), n_hi = min(cur.L + p.T_new, ta + C::kTile);
       if (n_lo < n_hi) {  // the same decision in every thread of the CTA
@@ -829,79 +928,192 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
     const uint32_t kb = sk_addr + st * C::kTileBytes;
     const uint32_t vb = sv_addr + st * C::kTileBytes;
     const int t0 = cur.k * C::kTile;
-    float sacc[NT][4];
+    if constexpr (FP8) {
+      // E4M3 tile: scores and weights as in attend_fp8.cuh
+      const float* ssc = scl + st * 2 * C::kTile;
+      const int ta = wrow + (lane >> 2);  // this thread's two tokens: ta and ta + 8
+      const float ska = ssc[ta], skb = ssc[ta + 8];
+      const float lva = __log2f(ssc[C::kTile + ta]), lvb = __log2f(ssc[C::kTile + ta + 8]);
+      // KVC_SK_FP8_CHAINS independent accumulator chains (chunk % chains), summed after:
+      // shorter dependent MMA chains for the one n-tile
+      constexpr int NCH = KVC_SK_FP8_CHAINS;
+      float sacc[NT][4];
+      float sch[NCH][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int kk = 0; kk < C::kKSteps; ++kk) {
-      uint32_t a[4];
-      ldmatrix_x4(a, kb + k_rp + (kk >> 2) * half_stride + ((((2 * kk + k_cs) & 7) ^ k_sw) << 4));
+          for (int e = 0; e < 4; ++e) sch[ch][nt][e] = 0.f;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816<T>(sacc[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
-    }
-    const int tok0 = t0 + wrow + (lane >> 2);
-    const bool unmasked = (t0 + C::kTile <= vis_min);
-    bool grew = false;
-    float alpha[NT][2];
+      for (int kp = 0; kp < C::kKSteps; kp += 2) {
+        uint32_t r[4];
+        ldmatrix_x4(r, kb + swz8<D>(k_row, kp + k_cs));
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+        for (int h = 0; h < 2; ++h) {  // chunk kp + h: r[2h] tokens 0-7, r[2h+1] tokens 8-15
+          const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * h]), e4m3x2_to_f16x2(r[2 * h + 1]),
+                                 e4m3x2_to_f16x2(r[2 * h] >> 16),
+                                 e4m3x2_to_f16x2(r[2 * h + 1] >> 16)};
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        float s0 = sacc[nt][cc] * p.scale_log2;
-        float s1 = sacc[nt][2 + cc] * p.scale_log2;
-        if (!unmasked) {
-          s0 = (tok0 < vis[nt][cc]) ? s0 : -INFINITY;
-          s1 = (tok0 + 8 < vis[nt][cc]) ? s1 : -INFINITY;
+          for (int nt = 0; nt < NT; ++nt)
+            mma_16816<__half>(sch[(kp + h) % NCH][nt], a, qb[kp + h][nt][0], qb[kp + h][nt][1]);
         }
-        float mx = fmaxf(s0, s1);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m[nt][cc], mx);
-        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[nt][cc] = exp2f(m[nt][cc] - mu);
-        grew |= (m_new > m[nt][cc]);
-        m[nt][cc] = m_new;
-        const float p0 = exp2f(s0 - mu);
-        const float p1 = exp2f(s1 - mu);
-        l[nt][cc] = fmaf(l[nt][cc], alpha[nt][cc], p0 + p1);
-        sacc[nt][cc] = p0;
-        sacc[nt][2 + cc] = p1;
       }
-    }
-    if (__any_sync(0xffffffffu, grew)) {
 #pragma unroll
-      for (int mt = 0; mt < C::kMTiles; ++mt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          o[mt][nt][0] *= alpha[nt][0];
-          o[mt][nt][1] *= alpha[nt][1];
-          o[mt][nt][2] *= alpha[nt][0];
-          o[mt][nt][3] *= alpha[nt][1];
+        for (int e = 0; e < 4; ++e) {
+          float v = sch[0][nt][e];
+#pragma unroll
+          for (int ch = 1; ch < NCH; ++ch) v += sch[ch][nt][e];
+          sacc[nt][e] = v;
         }
-    }
-    uint32_t pb[NT][2], pl[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t h0 = Elt<T>::pack2(sacc[nt][0], sacc[nt][1]);
-      const uint32_t h1 = Elt<T>::pack2(sacc[nt][2], sacc[nt][3]);
-      pb[nt][0] = movmatrix_trans(h0);
-      pb[nt][1] = movmatrix_trans(h1);
-      if constexpr (SplitP<T>::kOn) {  // bf16: the weights' rounding remainders
-        pl[nt][0] = movmatrix_trans(bf16_remainder2(sacc[nt][0], sacc[nt][1], h0));
-        pl[nt][1] = movmatrix_trans(bf16_remainder2(sacc[nt][2], sacc[nt][3], h1));
-      }
-    }
-#pragma unroll
-    for (int mt = 0; mt < C::kMTiles; ++mt) {
-      uint32_t a[4];
-      ldmatrix_x4_trans(a, vb + v_rp + (mt >> 2) * half_stride + ((((2 * mt + v_cs) & 7) ^ v_sw) << 4));
+      const int tok0 = t0 + ta;
+      const bool unmasked = (t0 + C::kTile <= vis_min);
+      bool grew = false;
+      float alpha_o[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
-        if constexpr (SplitP<T>::kOn) mma_16816<T>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float s0 = sacc[nt][cc] * fcol[nt][cc] * ska;
+          float s1 = sacc[nt][2 + cc] * fcol[nt][cc] * skb;
+          if (!unmasked) {
+            s0 = (tok0 < vis[nt][cc]) ? s0 : -INFINITY;
+            s1 = (tok0 + 8 < vis[nt][cc]) ? s1 : -INFINITY;
+          }
+          // the sum l, referenced to m
+          float mx = fmaxf(s0, s1);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m[nt][cc], mx);
+          const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+          l[nt][cc] = fmaf(l[nt][cc], exp2f(m[nt][cc] - mu), exp2f(s0 - mu) + exp2f(s1 - mu));
+          m[nt][cc] = m_new;
+          // the weights of O, referenced to mo: 2^(s + log2 v_scale - mo) <= 1
+          const float w0 = s0 + lva, w1 = s1 + lvb;
+          float mxo = fmaxf(w0, w1);
+          mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 4));
+          mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 8));
+          mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 16));
+          const float mo_new = fmaxf(mo[nt][cc], mxo);
+          const float muo = (mo_new == -INFINITY) ? 0.f : mo_new;
+          alpha_o[nt][cc] = exp2f(mo[nt][cc] - muo);
+          grew |= (mo_new > mo[nt][cc]);
+          mo[nt][cc] = mo_new;
+          sacc[nt][cc] = exp2f(w0 - muo);
+          sacc[nt][2 + cc] = exp2f(w1 - muo);
+        }
+      }
+      if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+        for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            o[mt][nt][0] *= alpha_o[nt][0];
+            o[mt][nt][1] *= alpha_o[nt][1];
+            o[mt][nt][2] *= alpha_o[nt][0];
+            o[mt][nt][3] *= alpha_o[nt][1];
+          }
+      }
+      uint32_t pb[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        pb[nt][0] = movmatrix_trans(f32x2_to_f16x2(sacc[nt][0], sacc[nt][1]));
+        pb[nt][1] = movmatrix_trans(f32x2_to_f16x2(sacc[nt][2], sacc[nt][3]));
+      }
+      // O^T += V^T . P^T; V^T rows of m-tile kp + h come in vt_row_to_d order
+#pragma unroll
+      for (int kp = 0; kp < C::kKSteps; kp += 2) {
+        uint32_t r[4];
+        ldmatrix_x4(r, vb + swz8<D>(k_row, kp + k_cs));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a[4] = {movmatrix_trans(e4m3x2_to_f16x2(r[2 * h])),
+                                 movmatrix_trans(e4m3x2_to_f16x2(r[2 * h] >> 16)),
+                                 movmatrix_trans(e4m3x2_to_f16x2(r[2 * h + 1])),
+                                 movmatrix_trans(e4m3x2_to_f16x2(r[2 * h + 1] >> 16))};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_16816<__half>(o[kp + h][nt], a, pb[nt][0], pb[nt][1]);
+        }
+      }
+    } else {
+      float sacc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < C::kKSteps; ++kk) {
+        uint32_t a[4];
+        ldmatrix_x4(a, kb + k_rp + (kk >> 2) * half_stride + ((((2 * kk + k_cs) & 7) ^ k_sw) << 4));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816<T>(sacc[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+      }
+      const int tok0 = t0 + wrow + (lane >> 2);
+      const bool unmasked = (t0 + C::kTile <= vis_min);
+      bool grew = false;
+      float alpha[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float s0 = sacc[nt][cc] * p.scale_log2;
+          float s1 = sacc[nt][2 + cc] * p.scale_log2;
+          if (!unmasked) {
+            s0 = (tok0 < vis[nt][cc]) ? s0 : -INFINITY;
+            s1 = (tok0 + 8 < vis[nt][cc]) ? s1 : -INFINITY;
+          }
+          float mx = fmaxf(s0, s1);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m[nt][cc], mx);
+          const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+          alpha[nt][cc] = exp2f(m[nt][cc] - mu);
+          grew |= (m_new > m[nt][cc]);
+          m[nt][cc] = m_new;
+          const float p0 = exp2f(s0 - mu);
+          const float p1 = exp2f(s1 - mu);
+          l[nt][cc] = fmaf(l[nt][cc], alpha[nt][cc], p0 + p1);
+          sacc[nt][cc] = p0;
+          sacc[nt][2 + cc] = p1;
+        }
+      }
+      if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+        for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            o[mt][nt][0] *= alpha[nt][0];
+            o[mt][nt][1] *= alpha[nt][1];
+            o[mt][nt][2] *= alpha[nt][0];
+            o[mt][nt][3] *= alpha[nt][1];
+          }
+      }
+      uint32_t pb[NT][2], pl[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t h0 = Elt<T>::pack2(sacc[nt][0], sacc[nt][1]);
+        const uint32_t h1 = Elt<T>::pack2(sacc[nt][2], sacc[nt][3]);
+        pb[nt][0] = movmatrix_trans(h0);
+        pb[nt][1] = movmatrix_trans(h1);
+        if constexpr (SplitP<T>::kOn) {  // bf16: the weights' rounding remainders
+          pl[nt][0] = movmatrix_trans(bf16_remainder2(sacc[nt][0], sacc[nt][1], h0));
+          pl[nt][1] = movmatrix_trans(bf16_remainder2(sacc[nt][2], sacc[nt][3], h1));
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < C::kMTiles; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, vb + v_rp + (mt >> 2) * half_stride + ((((2 * mt + v_cs) & 7) ^ v_sw) << 4));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816<T>(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+          if constexpr (SplitP<T>::kOn) mma_16816<T>(o[mt][nt], a, pl[nt][0], pl[nt][1]);
+        }
       }
     }
 
@@ -936,6 +1148,16 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
       constexpr int kHalfFloats = C::kTileBytes / 4;
       return idx < kHalfFloats ? red_acc + idx : red_acc_hi + (idx - kHalfFloats);
     };
+    // FP8: O referenced to m (O * 2^(mo - m)), its rows in vt_row_to_d order
+    float fo[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc)
+        fo[nt][cc] = !FP8 ? 1.f
+                     : (m[nt][cc] == -INFINITY || mo[nt][cc] == -INFINITY)
+                         ? 0.f
+                         : exp2f(mo[nt][cc] - m[nt][cc]);
 #pragma unroll
     for (int mt = 0; mt < C::kMTiles; ++mt)
 #pragma unroll
@@ -943,8 +1165,9 @@ __global__ void __launch_bounds__(StreamKCfg<D>::kThreads, StreamKCfg<D>::templa
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int row = nt * 8 + (lane & 3) * 2 + (e & 1);
-          const int d = mt * 16 + (lane >> 2) + (e >> 1) * 8;
-          *acc_at(warp, row, d) = o[mt][nt][e];
+          const int rho = (lane >> 2) + (e >> 1) * 8;
+          const int d = mt * 16 + (FP8 ? vt_row_to_d(rho) : rho);
+          *acc_at(warp, row, d) = FP8 ? o[mt][nt][e] * fo[nt][e & 1] : o[mt][nt][e];
         }
     if (lane < 4) {
 #pragma unroll

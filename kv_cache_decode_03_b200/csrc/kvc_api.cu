@@ -79,6 +79,12 @@ constexpr int kEltBytes = 2;
 #ifndef KVC_SPLIT_WAVES
 #define KVC_SPLIT_WAVES 4
 #endif
+#ifndef KVC_FP8_STREAMK  // FP8, 1-8 rows per KV head, no window: the stream-K kernel
+#define KVC_FP8_STREAMK 1
+#endif
+#ifndef KVC_SK_PENALTY_FP8  // its per-piece cost in virtual tiles
+#define KVC_SK_PENALTY_FP8 3
+#endif
 #ifndef KVC_FP8_SPLIT_WAVES  // the FP8 kernel's tiles are cheaper to load: fewer, longer slices
 #define KVC_FP8_SPLIT_WAVES 4
 #endif
@@ -298,22 +304,32 @@ int mma_occ(int D, int NT, bool paged) {
   return paged ? mma_occ_nt<128, T, true>(NT) : mma_occ_nt<128, T, false>(NT);
 }
 
-template <int D, int NT, typename T, bool PAGED>
+template <int D, int NT, typename T, bool PAGED, bool FP8 = false>
 int streamk_occupancy() {
   static int occ = 0;
   static std::once_flag once;
   std::call_once(once, [] {
-    const size_t smem = kvc::StreamKCfg<D>::template smem_bytes<NT>();
-    cudaFuncSetAttribute(kvc::attend_streamk_kernel<D, NT, T, PAGED>,
+    const size_t smem = kvc::StreamKCfg<D, FP8>::template smem_bytes<NT>();
+    cudaFuncSetAttribute(kvc::attend_streamk_kernel<D, NT, T, PAGED, FP8>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, kvc::attend_streamk_kernel<D, NT, T, PAGED>, kvc::StreamKCfg<D>::kThreads,
-            smem) != cudaSuccess)
+            &n, kvc::attend_streamk_kernel<D, NT, T, PAGED, FP8>,
+            kvc::StreamKCfg<D, FP8>::kThreads, smem) != cudaSuccess)
       n = 1;
     occ = std::max(1, n);
   });
   return occ;
+}
+
+// the FP8 variant: one row group of 8, bf16 queries
+int streamk_fp8_occ(int D, bool paged) {
+  using T = __nv_bfloat16;
+  if (D == 64)
+    return paged ? streamk_occupancy<64, 1, T, true, true>()
+                 : streamk_occupancy<64, 1, T, false, true>();
+  return paged ? streamk_occupancy<128, 1, T, true, true>()
+               : streamk_occupancy<128, 1, T, false, true>();
 }
 
 template <typename T>
@@ -558,6 +574,20 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
     pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
     return pl;
   }
+  const int fp8_max_batch = c->D == 64 ? kvc::StreamKCfg<64, true>::kMaxBatch
+                                       : kvc::StreamKCfg<128, true>::kMaxBatch;
+  if (KVC_FP8_STREAMK && pl.fp8 && pl.NT == 1 && c->B <= fp8_max_batch && window == 0) {
+    pl.streamk = true;  // the stream-K kernel with E4M3 stages
+    pl.grid = c->num_sms * streamk_fp8_occ(c->D, c->paged);
+    pl.slots = (size_t)pl.grid * 2;
+    pl.slot_rows = pl.R;
+    pl.split_tokens = 1 << 30;
+    pl.num_splits = 1;
+    pl.ws_partial_floats = pl.slots * pl.slot_rows * (c->D + 1);
+    pl.ws_counters = (size_t)c->B * c->H_kv * pl.row_blocks;
+    pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
+    return pl;
+  }
   const int max_batch = c->D == 64 ? kvc::StreamKCfg<64>::kMaxBatch
                                    : kvc::StreamKCfg<128>::kMaxBatch;
   if (pl.mma && pl.NT <= 2 && c->B <= max_batch && window == 0) {
@@ -679,12 +709,12 @@ static bool dependent_launch_enabled() {
   return on;
 }
 
-template <int D, int NT, typename T, bool PAGED>
+template <int D, int NT, typename T, bool PAGED, bool FP8 = false>
 kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, bool pdl,
                                  const CUtensorMap& tk, const CUtensorMap& tv,
                                  cudaStream_t stream) {
-  using C = kvc::StreamKCfg<D>;
-  streamk_occupancy<D, NT, T, PAGED>();  // sets the shared-memory attribute once
+  using C = kvc::StreamKCfg<D, FP8>;
+  streamk_occupancy<D, NT, T, PAGED, FP8>();  // sets the shared-memory attribute once
   const size_t smem = C::template smem_bytes<NT>();
   // Programmatic stream serialization: the kernel may start while the grid
   // ahead of it retires; it waits for that grid (griddepcontrol.wait) before
@@ -700,7 +730,18 @@ kvc_status launch_attend_streamk(const kvc::AttendParams& p, int grid, bool pdl,
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cuda_status(
-      cudaLaunchKernelEx(&cfg, kvc::attend_streamk_kernel<D, NT, T, PAGED>, p, tk, tv));
+      cudaLaunchKernelEx(&cfg, kvc::attend_streamk_kernel<D, NT, T, PAGED, FP8>, p, tk, tv));
+}
+
+kvc_status dispatch_streamk_fp8(const kvc::AttendParams& p, int D, bool paged, int grid,
+                                bool pdl, const CUtensorMap& tk, const CUtensorMap& tv,
+                                cudaStream_t s) {
+  using T = __nv_bfloat16;
+  if (D == 64)
+    return paged ? launch_attend_streamk<64, 1, T, true, true>(p, grid, pdl, tk, tv, s)
+                 : launch_attend_streamk<64, 1, T, false, true>(p, grid, pdl, tk, tv, s);
+  return paged ? launch_attend_streamk<128, 1, T, true, true>(p, grid, pdl, tk, tv, s)
+               : launch_attend_streamk<128, 1, T, false, true>(p, grid, pdl, tk, tv, s);
 }
 
 template <typename T>
@@ -859,9 +900,15 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
   p.wait_limit_ns = c->wait_limit_ns;
   p.sk_penalty = !pl.streamk ? 0
                  : pl.tc      ? KVC_TC_SK_PENALTY
+                 : pl.fp8     ? KVC_SK_PENALTY_FP8
                  : c->D == 128 ? KVC_SK_PENALTY_D128
                               : KVC_SK_PENALTY_D64;
-  p.sk_blocked = pl.streamk && !pl.tc && c->tma4 ? 1 : 0;
+  p.sk_blocked = pl.streamk && !pl.tc && !pl.fp8 && c->tma4 ? 1 : 0;
+  if (pl.fp8) {
+    p.k_scales = scale_pool(c, layer, 0);
+    p.v_scales = scale_pool(c, layer, 1);
+    p.T_pad = c->T_pad;
+  }
   p.sk_slot_rows = pl.slot_rows;
   p.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
@@ -878,6 +925,9 @@ float* lse_base(const kvc_cache* c, const Plan& pl, float* ws, int H_q, int T_ne
 // Launch the attend kernel a plan chose for layer `layer`.
 kvc_status run_plan(const kvc_cache* c, int layer, const Plan& pl, const kvc::AttendParams& p,
                     cudaStream_t s) {
+  if (pl.fp8 && pl.streamk)
+    return dispatch_streamk_fp8(p, c->D, c->paged, pl.grid, c->dependent_launch, c->tmk[layer],
+                                c->tmv[layer], s);
   if (pl.fp8) {
     const kvc::Fp8Scales sc{scale_pool(c, layer, 0), scale_pool(c, layer, 1), c->T_pad};
     if (c->D == 64)
@@ -1399,7 +1449,7 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
   if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
-  if (!pl.streamk || pl.tc) {  // only the mma.sync stream-K kernel fuses the append
+  if (!pl.streamk || pl.tc || pl.fp8) {  // only the mma.sync stream-K kernel fuses the append
     kvc_status st = kvc_append(c, layer, k_new, v_new, T_new, block_table, max_pages,
                                seq_lens, stream);
     if (st != KVC_OK) return st;

@@ -47,6 +47,9 @@ struct AttendParams {
   int* err;
   unsigned long long wait_limit_ns;  // bound of every pipeline wait (0: the default, 1 s)
   int sk_penalty;  // stream-K: virtual tiles charged for each segment a CTA enters
+  const float* k_scales;  // FP8 cache (stream-K): this layer's K / V scale pools,
+  const float* v_scales;  // contiguous (B, H_kv, T_pad) or paged (num_pages, H_kv, P)
+  int T_pad;
   int sk_slot_rows;  // stream-K: rows of one partial-result slot (the rows of a row block
                      // that can be valid: min(rows per CTA, query rows per KV head))
   int sk_blocked;  // stream-K, paged, D = 128, pages < 64 tokens: the tensor maps are 4-D

@@ -146,6 +146,37 @@ def test_fp8_page_sizes(P):
     run(case)
 
 
+@pytest.mark.parametrize("paged", [False, True])
+def test_fp8_streamk_route_ragged_batch(paged):
+    """1-8 rows per KV head take the persistent stream-K kernel with E4M3 stages: many
+    requests with very different lengths (so that pieces of a segment land on several
+    CTAs and are merged), results within the attention tolerance."""
+    if paged:
+        case = W.paged_case("fp8sk", 16, 16, 4, 128, "bf16", 1, 0, 7000, 16, seed=141,
+                            pool_seed=142)
+    else:
+        case = W.contig_case("fp8sk", 12, 32, 8, 64, "bf16", 1,
+                             [5000, 17, 0, 3100, 64, 63, 1, 4500, 2222, 129, 4999, 700],
+                             seed=143)
+    r = Fp8Run(case)
+    try:
+        ns, split_tokens = r.cache.plan(case.H_q, case.T_new, case.max_pages if paged else 0)
+        assert split_tokens == 0, "expected the persistent stream-K plan"
+        r.append()
+        q = case.q(0)
+        qd = H.to_device(q, "bf16")
+        outs = []
+        for on in (True, False):  # with and without programmatic dependent launch
+            r.cache.set_dependent_launch(on)
+            outs.append(r.cache.attend(0, qd, r.seq_lens, r.bt, scale=case.scale))
+        assert r.cache.get_error() == kvc.KVC_OK
+        assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+        sel, ref = r.reference(q)
+        H.compare(H.out_to_f64(outs[0])[sel], ref, f"{case.name} fp8 stream-K")
+    finally:
+        r.close()
+
+
 def test_fp8_long_context():
     case = W.paged_case("fp8long", 2, 32, 8, 128, "bf16", 1, 20000, 30000, 16, seed=121,
                         pool_seed=122)

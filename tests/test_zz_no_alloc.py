@@ -8,8 +8,9 @@ the synchronisation a free implies.  It runs the same plan and the same kernels 
 kvc_attend with its split-K scratch in a fixed 16 MiB device array of the library.
 
 Here every kernel family an unwindowed attend can take -- persistent stream-K on
-mma.sync and on tcgen05, the CUDA-core kernel and the FP8 kernel (the fixed-split
-mma.sync and tcgen05 kernels serve only windowed calls) -- is called twice in a row
+mma.sync (bf16/fp16 and E4M3 stages) and on tcgen05, the CUDA-core kernel and the
+fixed-split FP8 kernel (the fixed-split mma.sync and tcgen05 kernels serve only
+windowed calls) -- is called twice in a row
 through the new entry point.  Each case first checks that the plan takes
 the intended kernel with more than one slice (so the scratch is really used).  The
 two outputs must be byte-identical to kvc_attend's (same plan, same kernels,
@@ -22,6 +23,8 @@ This file is collected last and needs nothing from the other test files, so it r
 the same alone in a fresh process or after the whole suite.
 """
 from __future__ import annotations
+
+import gc
 
 import numpy as np
 import pytest
@@ -67,8 +70,11 @@ CASES = {
     # CUDA-core kernel (D = 32 has no tensor maps), several slices per head
     "splitk_simt_d32": (lambda: W.contig_case("na_simt", 2, 16, 16, 32, "fp16", 1, 6000,
                                               seed=95), "native", "split"),
-    # FP8 cache: its own fixed-split kernel
-    "splitk_fp8_gqa": (lambda: W.contig_case("na_fp8", 4, 16, 4, 128, "bf16", 1, 3000,
+    # FP8 cache, 4 rows per KV head: the stream-K kernel with E4M3 stages
+    "streamk_fp8_gqa": (lambda: W.contig_case("na_fp8sk", 4, 16, 4, 128, "bf16", 1, 3000,
+                                              seed=98), "fp8", "streamk"),
+    # FP8 cache, 12 rows per KV head: the fixed-split FP8 kernel
+    "splitk_fp8_gqa": (lambda: W.contig_case("na_fp8", 4, 16, 4, 128, "bf16", 3, 3000,
                                              seed=96), "fp8", "split"),
 }
 
@@ -126,10 +132,17 @@ def test_noalloc_matches_attend_twice_in_a_row(name):
         base = torch.empty_like(q)
         _call(kvc.kvc_attend, cache, case, q, seq, bt, base)
         outs = [torch.full_like(q, float("nan")), torch.full_like(q, float("nan"))]
-        before = _device_memory()
-        for out in outs:  # two calls in a row share (and reuse) the static scratch
-            _call(kvc.kvc_attend_noalloc, cache, case, q, seq, bt, out)
-        after = _device_memory()
+        # no collection inside the window: a tensor of an earlier case freed there would
+        # move the counters without any allocation by the calls
+        gc.collect()
+        gc.disable()
+        try:
+            before = _device_memory()
+            for out in outs:  # two calls in a row share (and reuse) the static scratch
+                _call(kvc.kvc_attend_noalloc, cache, case, q, seq, bt, out)
+            after = _device_memory()
+        finally:
+            gc.enable()
         assert cache.get_error() == kvc.KVC_OK
         assert after[:2] == before[:2], "the caching allocator's counters moved"
         # device-wide free memory can also move under other processes: it must not drop
