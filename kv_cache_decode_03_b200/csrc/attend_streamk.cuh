@@ -192,16 +192,21 @@ __device__ __forceinline__ bool length_ok(const AttendParams& p, int L, bool pag
          (!paged || ((L + p.T_new - 1) >> p.page_shift) < p.max_pages);
 }
 
-// Virtual tiles of request b: its segments' tiles plus their penalty tiles.
+// Virtual tiles of request b: its segments' tiles plus their penalty tiles (row-block
+// major: those of one row block, every block having as many).
 template <int R>
 __device__ __forceinline__ int request_tiles(const AttendParams& p, int L) {
   int t = 0;
-  for (int rb = 0; rb < p.row_blocks; ++rb)
+  const int nrb = p.sk_rb_major ? 1 : p.row_blocks;
+  for (int rb = 0; rb < nrb; ++rb)
     t += ceil_div(L + row_block(rb, R, p.rows, p.T_new).imax + 1, 64) + p.sk_penalty;
   return t * p.H_kv;
 }
 
-// Walks the real tiles in the global order: request, KV head, row block, tile.
+// Walks the real tiles in the global order: request, KV head, row block, tile; or, row-block
+// major (p.sk_rb_major), row block, request, KV head, tile -- then the CTAs that stream one
+// K/V tile for different row blocks are a fixed number of ranges apart and stream it at
+// about the same time, so that L2 serves all but the first read.
 template <int R>
 struct TileCursor {
   int b, g, rb, L, k, seg_tiles;
@@ -215,14 +220,22 @@ struct TileCursor {
     if (++k < seg_tiles) return;
     seg_start += seg_tiles + p.sk_penalty;
     k = 0;
-    if (++rb == p.row_blocks) {
-      rb = 0;
+    if (p.sk_rb_major || ++rb == p.row_blocks) {
+      if (!p.sk_rb_major) rb = 0;
       if (++g == p.H_kv) {
         g = 0;
         do {  // requests whose length is invalid contribute no tiles
           ++b;
           L = b < p.B ? lens[b] : 0;
         } while (b < p.B && !length_ok(p, L, paged));
+        if (p.sk_rb_major && b >= p.B && rb + 1 < p.row_blocks) {  // the next row block
+          ++rb;
+          b = -1;
+          do {
+            ++b;
+            L = b < p.B ? lens[b] : 0;
+          } while (b < p.B && !length_ok(p, L, paged));
+        }
       }
     }
     enter_segment(p);

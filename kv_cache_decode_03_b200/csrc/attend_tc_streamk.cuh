@@ -105,28 +105,32 @@ __device__ __forceinline__ SkRange<R> sk_plan(const AttendParams& p, int* P, int
   if (tid == NTH - 1) P[p.B] = base + incl;
   __syncthreads();
   SkRange<R> r{};
-  r.Wt = P[p.B];
+  // row-block major: P covers one row block, repeated row_blocks times
+  const long long W1 = P[p.B];
+  r.Wt = p.sk_rb_major ? W1 * p.row_blocks : W1;
   r.G = (int)(r.Wt < (long long)gridDim.x ? r.Wt : (long long)gridDim.x);
   const int c = blockIdx.x;
   r.work = c < r.G;
   if (r.work) {
     r.lo = (long long)c * r.Wt / r.G;
     r.hi = (long long)(c + 1) * r.Wt / r.G;
-    int a = 0, z = p.B;  // largest b with P[b] <= lo
+    const int rb0 = p.sk_rb_major ? (int)(r.lo / W1) : 0;
+    const long long lo1 = r.lo - rb0 * W1;  // the position within the row block's part
+    int a = 0, z = p.B;  // largest b with P[b] <= lo1
     while (z - a > 1) {
       const int mid = (a + z) >> 1;
-      if (P[mid] <= r.lo) a = mid;
+      if (P[mid] <= lo1) a = mid;
       else z = mid;
     }
     while (P[a + 1] == P[a]) ++a;  // requests with no tiles
     TileCursor<R>& cur = r.cur;
     cur.b = a;
     cur.L = Ls[a];
-    int local = (int)(r.lo - P[a]);
+    int local = (int)(lo1 - P[a]);
     const int per_g = (P[a + 1] - P[a]) / p.H_kv;
     cur.g = local / per_g;
     local -= cur.g * per_g;
-    cur.rb = 0;
+    cur.rb = rb0;  // row-block major: the (b, g) segment of this block; else the first
     while (true) {
       const int t = ceil_div(cur.L + row_block(cur.rb, R, p.rows, p.T_new).imax + 1, 64);
       if (local < t + p.sk_penalty || cur.rb == p.row_blocks - 1) {

@@ -79,6 +79,9 @@ constexpr int kEltBytes = 2;
 #ifndef KVC_SPLIT_WAVES
 #define KVC_SPLIT_WAVES 4
 #endif
+#ifndef KVC_TC_RB_MAJOR
+#define KVC_TC_RB_MAJOR 1
+#endif
 #ifndef KVC_FP8_STREAMK  // FP8, 1-8 rows per KV head, no window: the stream-K kernel
 #define KVC_FP8_STREAMK 1
 #endif
@@ -904,6 +907,13 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
                  : c->D == 128 ? KVC_SK_PENALTY_D128
                               : KVC_SK_PENALTY_D64;
   p.sk_blocked = pl.streamk && !pl.tc && !pl.fp8 && c->tma4 ? 1 : 0;
+  // tcgen05 stream-K over several row blocks: row-block major when every block spans the
+  // same positions (each holds all T_new new-row indices), so a request's K/V tiles are
+  // streamed for all blocks at about the same time
+  if (KVC_TC_RB_MAJOR && pl.tc && pl.streamk && pl.row_blocks > 1 && T_new <= pl.R) {
+    const int last_rows = p.rows - (pl.row_blocks - 1) * pl.R;
+    p.sk_rb_major = last_rows >= T_new ? 1 : 0;
+  }
   if (pl.fp8) {
     p.k_scales = scale_pool(c, layer, 0);
     p.v_scales = scale_pool(c, layer, 1);

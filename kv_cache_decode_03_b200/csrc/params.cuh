@@ -54,6 +54,8 @@ struct AttendParams {
                      // that can be valid: min(rows per CTA, query rows per KV head))
   int sk_blocked;  // stream-K, paged, D = 128, pages < 64 tokens: the tensor maps are 4-D
                    // (64 elements, page tokens, 2 halves, page blocks), one box a page
+  int sk_rb_major;  // stream-K: segments ordered row block first (every block the same
+                   // number of tiles a request)
   int stall;  // failure-detection test: the producers issue no copies, so the first
               // wait runs out (stream-K and tcgen05 kernels)
 };
