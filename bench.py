@@ -374,7 +374,9 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     ns, split_tokens = cache.plan(c.H_q, c.T_new, max_pages)
     stream = torch.cuda.Stream()
     scale = c.scale
-    fused = split_tokens == 0 and not fp8  # kvc_append_attend is one launch
+    # kvc_append_attend is one launch on the mma.sync stream-K kernels (bf16/fp16 and
+    # E4M3 stages: up to 16 rows per KV head); the tcgen05 and fixed-split plans append first
+    fused = split_tokens == 0 and (c.H_q // c.H_kv) * c.T_new <= 16
 
     def step(q=qs, k=ks, v=vs, o=outs):
         for layer in range(c.layers):

@@ -937,6 +937,55 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
         named_barrier_sync(1, NTH);
       }
     }
+    if (FP8 && p.k_new != nullptr) {
+      // FP8: warp w quantises rows (row, K or V) w, w + 4, ... of the new positions in
+      // this tile exactly as the append kernel does, into the stage (codes and scale)
+      // and, first row block, into the cache
+      const int ta = cur.k * C::kTile;
+      const int n_lo = max(cur.L, ta), n_hi = min(cur.L + p.T_new, ta + C::kTile);
+      if (n_lo < n_hi) {  // the same decision in every thread of the CTA
+        constexpr int PER = D / 32;
+        float* ssc = scl + st * 2 * C::kTile;
+#pragma unroll 1
+        for (int task = warp; task < 2 * (n_hi - n_lo); task += W) {
+          const bool is_v = task & 1;
+          const int pos = n_lo + (task >> 1);
+          const __nv_bfloat16* src =
+              static_cast<const __nv_bfloat16*>(is_v ? p.v_new : p.k_new) +
+              (((size_t)cur.b * p.H_kv + cur.g) * p.T_new + (pos - cur.L)) * D;
+          uint32_t codes;
+          const float scale = quantize_row_warp<PER>(src, lane, codes);
+          const int d = lane * PER;  // this lane's first code of the row
+          unsigned char* tile = (is_v ? sv : sk) + st * C::kTileBytes;
+          unsigned char* at = tile + swz8<D>(pos - ta, d >> 4) + (d & 15);
+          if (PER == 4) *reinterpret_cast<uint32_t*>(at) = codes;
+          else *reinterpret_cast<uint16_t*>(at) = (uint16_t)codes;
+          if (lane == 0) ssc[(is_v ? C::kTile : 0) + pos - ta] = scale;
+          if (cur.rb == 0) {
+            long long row, srow;
+            if (PAGED) {
+              const int page = p.block_table[(size_t)cur.b * p.max_pages + (pos >> p.page_shift)];
+              if (page < 0 || page >= p.num_pages) {
+                if (lane == 0) flag_error(p.err, KVC_ERR_BOUNDS);
+                continue;
+              }
+              row = ((long long)page * p.H_kv + cur.g) * (1 << p.page_shift) +
+                    (pos & ((1 << p.page_shift) - 1));
+              srow = row;
+            } else {
+              row = ((long long)cur.b * p.H_kv + cur.g) * p.max_T + pos;
+              srow = ((long long)cur.b * p.H_kv + cur.g) * p.T_pad + pos;
+            }
+            unsigned char* pool =
+                static_cast<unsigned char*>(const_cast<void*>(is_v ? p.v_pool : p.k_pool));
+            if (PER == 4) reinterpret_cast<uint32_t*>(pool + row * D)[lane] = codes;
+            else reinterpret_cast<uint16_t*>(pool + row * D)[lane] = (uint16_t)codes;
+            if (lane == 0) const_cast<float*>(is_v ? p.v_scales : p.k_scales)[srow] = scale;
+          }
+        }
+        named_barrier_sync(1, NTH);
+      }
+    }
 
     const uint32_t kb = sk_addr + st * C::kTileBytes;
     const uint32_t vb = sv_addr + st * C::kTileBytes;

@@ -68,6 +68,29 @@ struct AppendFp8Params {
   int* err;
 };
 
+// Quantises one row of D = 32 * PER bf16 values with a warp: lane `lane` holds values
+// lane*PER .. lane*PER + PER - 1 of `src`; returns the row's scale (every lane) and the
+// lane's PER codes, first value in the low byte.
+template <int PER>
+__device__ __forceinline__ float quantize_row_warp(const __nv_bfloat16* src, int lane,
+                                                   uint32_t& codes) {
+  float x[PER];
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    x[k] = __bfloat162float(src[lane * PER + k]);
+    amax = fmaxf(amax, fabsf(x[k]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float scale = amax > 0.f ? amax / kE4M3Max : 1.f;
+  codes = 0u;
+#pragma unroll
+  for (int k = 0; k < PER; k += 2)
+    codes |= (uint32_t)f32x2_to_e4m3x2(x[k] / scale, x[k + 1] / scale) << (8 * k);
+  return scale;
+}
+
 // One warp per new row (b, g, i) and tensor (K or V): lanes own D/32 values each.
 template <bool PAGED>
 __global__ void append_fp8_kernel(const AppendFp8Params p) {
@@ -103,21 +126,15 @@ __global__ void append_fp8_kernel(const AppendFp8Params p) {
   const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? p.v_new : p.k_new) +
                              (size_t)r * p.D;
   // D = 64 or 128: each lane holds 2 or 4 consecutive values
-  const int per = p.D / 32;
-  float x[4] = {0.f, 0.f, 0.f, 0.f};
-  float amax = 0.f;
-  for (int k = 0; k < per; ++k) {
-    x[k] = __bfloat162float(src[lane * per + k]);
-    amax = fmaxf(amax, fabsf(x[k]));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = amax > 0.f ? amax / kE4M3Max : 1.f;
-  uint8_t* dst = (is_v ? p.v_codes : p.k_codes) + row * p.D + lane * per;
-  for (int k = 0; k < per; k += 2) {
-    const uint16_t c = f32x2_to_e4m3x2(x[k] / scale, x[k + 1] / scale);
-    dst[k] = (uint8_t)(c & 0xFF);
-    dst[k + 1] = (uint8_t)(c >> 8);
+  uint32_t codes;
+  uint8_t* dst = (is_v ? p.v_codes : p.k_codes) + row * p.D;
+  float scale;
+  if (p.D == 128) {
+    scale = quantize_row_warp<4>(src, lane, codes);
+    reinterpret_cast<uint32_t*>(dst)[lane] = codes;
+  } else {
+    scale = quantize_row_warp<2>(src, lane, codes);
+    reinterpret_cast<uint16_t*>(dst)[lane] = (uint16_t)codes;
   }
   if (lane == 0) (is_v ? p.v_scales : p.k_scales)[srow] = scale;
 }

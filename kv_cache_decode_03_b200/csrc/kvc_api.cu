@@ -1459,7 +1459,7 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
   if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
-  if (!pl.streamk || pl.tc || pl.fp8) {  // only the mma.sync stream-K kernel fuses the append
+  if (!pl.streamk || pl.tc) {  // only the mma.sync stream-K kernels fuse the append
     kvc_status st = kvc_append(c, layer, k_new, v_new, T_new, block_table, max_pages,
                                seq_lens, stream);
     if (st != KVC_OK) return st;
@@ -1476,6 +1476,9 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   p.k_new = k_new;
   p.v_new = v_new;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.fp8)
+    return dispatch_streamk_fp8(p, c->D, c->paged, pl.grid, c->dependent_launch, c->tmk[layer],
+                                c->tmv[layer], s);
   const CUtensorMap& tk = p.sk_blocked ? c->tmk4[layer] : c->tmk[layer];
   const CUtensorMap& tv = p.sk_blocked ? c->tmv4[layer] : c->tmv[layer];
   return c->dtype == KVC_BF16

@@ -177,6 +177,38 @@ def test_fp8_streamk_route_ragged_batch(paged):
         r.close()
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("paged", [False, True])
+def test_fp8_append_attend_fused(D, paged):
+    """kvc_append_attend on an FP8 cache is one launch of the stream-K kernel, which
+    quantises the new rows itself: codes and scales bit-exact with the oracle's append
+    (new rows straddling tile boundaries, an empty past), attention within tolerance."""
+    if paged:
+        case = W.paged_case("fp8fz", 5, 16, 4, D, "bf16", 2, 0, 2000, 16, seed=151,
+                            pool_seed=152)
+    else:
+        case = W.contig_case("fp8fz", 5, 16, 4, D, "bf16", 2, [63, 0, 1999, 640, 127],
+                             seed=153, max_T=2100)
+    r = Fp8Run(case)
+    try:
+        mp = case.max_pages if paged else 0
+        ns, split_tokens = r.cache.plan(case.H_q, case.T_new, mp)
+        assert split_tokens == 0, "expected the persistent stream-K plan"
+        q = case.q(0)
+        out = r.cache.append_attend(0, H.to_device(case.k_new(0), "bf16"),
+                                    H.to_device(case.v_new(0), "bf16"),
+                                    H.to_device(q, "bf16"), r.seq_lens, r.bt, scale=case.scale)
+        assert r.cache.get_error() == kvc.KVC_OK
+        bt = case.block_table if paged else None
+        r.o.append_fp8(r.img["kc"], r.img["ks"], case.k_new(0), case.seq_lens, bt)
+        r.o.append_fp8(r.img["vc"], r.img["vs"], case.v_new(0), case.seq_lens, bt)
+        r.check_pools()
+        sel, ref = r.reference(q)
+        H.compare(H.out_to_f64(out)[sel], ref, f"{case.name} fp8 fused append + attend")
+    finally:
+        r.close()
+
+
 def test_fp8_long_context():
     case = W.paged_case("fp8long", 2, 32, 8, 128, "bf16", 1, 20000, 30000, 16, seed=121,
                         pool_seed=122)
