@@ -254,6 +254,17 @@ kvc_status kvc_set_wait_limit(kvc_cache* cache, unsigned long long ns);
  */
 kvc_status kvc_inject_stall(kvc_cache* cache);
 
+/*
+ * kvc_inject_replan -- test hook for the dependent launch.  The persistent stream-K
+ * kernel plans its range from the lengths it reads before its dependency wait and
+ * issues its first copies from that plan right after the wait, while it reads the
+ * lengths again; if they changed, it waits for those copies, resets its pipeline and
+ * plans again.  This hook makes the next attend call on this cache (stream-K only)
+ * take that path whatever the lengths: its results are the same as without it.  The
+ * next call consumes it either way.
+ */
+kvc_status kvc_inject_replan(kvc_cache* cache);
+
 /* kvc_status_string -- static, human-readable name of a status. */
 const char* kvc_status_string(kvc_status status);
 

@@ -79,6 +79,7 @@ def library() -> ctypes.CDLL:
         "kvc_set_dependent_launch": ([P, I], I),
         "kvc_set_wait_limit": ([P, ctypes.c_ulonglong], I),
         "kvc_inject_stall": ([P], I),
+        "kvc_inject_replan": ([P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -238,6 +239,10 @@ def kvc_set_wait_limit(cache: int, ns: int) -> None:
 
 def kvc_inject_stall(cache: int) -> None:
     _check(library().kvc_inject_stall(cache), "kvc_inject_stall")
+
+
+def kvc_inject_replan(cache: int) -> None:
+    _check(library().kvc_inject_replan(cache), "kvc_inject_replan")
 
 
 # ---------------------------------------------------------------------------
@@ -412,6 +417,9 @@ class KVCache:
 
     def inject_stall(self) -> None:
         kvc_inject_stall(self.handle)
+
+    def inject_replan(self) -> None:
+        kvc_inject_replan(self.handle)
 
     def commit(self, seq_lens, accepted, T_new: int, stream=None) -> None:
         """seq_lens[b] += accepted[b] on the device (0 <= accepted[b] <= T_new)."""

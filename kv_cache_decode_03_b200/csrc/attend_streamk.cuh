@@ -607,44 +607,29 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
     }
   }
   griddep_wait();
-  // The lengths now count: keep the speculative plan if none of them changed.
-  bool work;
-  {
-    uint32_t h = 0;
-    for (int b = b_lo; b < b_hi; ++b) {
-      const int L = p.seq_lens[b];
-      h = mix(h, L);
-      if (!length_ok(p, L, PAGED)) flag_error(p.err, KVC_ERR_BOUNDS);
-    }
-    const bool same_first = !spec_work || p.seq_lens[spec_cur.b] == spec_cur.L;
-    if (__syncthreads_or(h != spec_digest || !same_first)) {
-      work = locate(true);
-    } else {
-      work = spec_work;
-      cur = spec_cur;
-    }
-  }
-  if (!work) return;
 
   // ------------------------------------------------------- tile producer
   // Warp 0 issues the copies (lane 0 the barrier and q; lane k box k).
   const bool producer = (warp == 0) && !p.stall;
   const uint64_t pol = l2_policy_evict_first();
-  TileCursor<R> pc = cur;  // producer's own cursor
+  TileCursor<R> pc = spec_cur;  // producer's own cursor
   int issued = 0;
   // Paged: lane k < nbox holds the page ids of box k of the next kLookahead tiles to
   // issue (ids[0] for tile pc); a second cursor, kLookahead - 1 tiles ahead of pc, reads
   // them, so a lookup has that many tiles' time to land.
   constexpr int kLookahead = KVC_SK_LOOKAHEAD;
   int ids[kLookahead];
-  TileCursor<R> pa = cur;
-  if (PAGED && producer) {
+  TileCursor<R> pa = spec_cur;
+  auto prime_lookups = [&]() {
+    if (PAGED && producer) {
+      pa = pc;
 #pragma unroll
-    for (int i = 0; i < kLookahead; ++i) {
-      if (i > 0) pa.next(p, PAGED);
-      ids[i] = lookup_page(pa, lane);
+      for (int i = 0; i < kLookahead; ++i) {
+        if (i > 0) pa.next(p, PAGED);
+        ids[i] = lookup_page(pa, lane);
+      }
     }
-  }
+  };
   auto issue = [&]() {
     const int st = issued % C::kStages;
     const bool first = (issued == 0) || (pc.k == 0);
@@ -723,6 +708,53 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
       ids[kLookahead - 1] = lookup_page(pa, lane);
     }
   };
+  // The first copies of the speculative plan go out now, after the wait (so they read
+  // what the grid ahead wrote), while every thread checks the plan against the lengths
+  // as they now stand; a stale plan drains them and starts over.
+  if (spec_work && producer) {
+    prime_lookups();
+    while (issued < min(C::kStages, ntiles)) issue();
+  }
+  bool work;
+  {
+    uint32_t h = 0;
+    for (int b = b_lo; b < b_hi; ++b) {
+      const int L = p.seq_lens[b];
+      h = mix(h, L);
+      if (!length_ok(p, L, PAGED)) flag_error(p.err, KVC_ERR_BOUNDS);
+    }
+    const bool same_first = !spec_work || p.seq_lens[spec_cur.b] == spec_cur.L;
+    if (__syncthreads_or(h != spec_digest || !same_first || p.replan)) {
+      // every speculative copy lands before the barriers are reset and the ring reused
+      bool drained = true;
+      if (producer && lane == 0)
+#pragma unroll 1
+        for (int j = 0; j < issued && drained; ++j)
+          drained = mbar_wait(&full[j], 0, p.err, p.wait_limit_ns ? p.wait_limit_ns
+                                                                  : kWaitLimitNs);
+      if (__syncthreads_or(!drained)) return;  // a copy that never landed: reported
+      if (tid == 0) {
+#pragma unroll
+        for (int st = 0; st < C::kStages; ++st) {
+          mbar_inval(&full[st]);
+          mbar_inval(&empty[st]);
+          mbar_init(&full[st], 1);
+          mbar_init(&empty[st], W);
+        }
+        fence_barrier_init();
+      }
+      issued = 0;
+      work = locate(true);  // its barriers publish the new barriers too
+      if (work && producer) {
+        pc = cur;
+        prime_lookups();
+      }
+    } else {
+      work = spec_work;
+      cur = spec_cur;
+    }
+  }
+  if (!work) return;
   if (producer)
     while (issued < min(C::kStages, ntiles)) issue();
 

@@ -48,6 +48,7 @@ struct kvc_cache {
   bool dependent_launch;           // stream-K launches with programmatic stream serialization
   unsigned long long wait_limit_ns;  // bound of the kernels' pipeline waits (0: 1 s)
   bool stall_next;                 // failure-detection test: next attend issues no copies
+  bool replan_next;                // dependent-launch test: next stream-K attend replans
 };
 
 namespace {
@@ -922,6 +923,8 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
   p.sk_slot_rows = pl.slot_rows;
   p.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
+  p.replan = c->replan_next ? 1 : 0;
+  c->replan_next = false;
   return p;
 }
 
@@ -1053,6 +1056,7 @@ static kvc_status create_cache(int B, int H_kv, int D, int max_T, kvc_dtype dtyp
   c->dependent_launch = dependent_launch_enabled();
   c->wait_limit_ns = 0;
   c->stall_next = false;
+  c->replan_next = false;
   void* pool = nullptr;
   if (cudaMalloc(&pool, 2 * layer_bytes * (size_t)num_layers) != cudaSuccess) {
     cudaGetLastError();
@@ -1354,6 +1358,12 @@ kvc_status kvc_set_wait_limit(kvc_cache* c, unsigned long long ns) {
 kvc_status kvc_inject_stall(kvc_cache* c) {
   if (!c) return KVC_ERR_INVALID_ARG;
   c->stall_next = true;
+  return KVC_OK;
+}
+
+kvc_status kvc_inject_replan(kvc_cache* c) {
+  if (!c) return KVC_ERR_INVALID_ARG;
+  c->replan_next = true;
   return KVC_OK;
 }
 

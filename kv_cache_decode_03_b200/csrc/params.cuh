@@ -56,6 +56,7 @@ struct AttendParams {
                    // (64 elements, page tokens, 2 halves, page blocks), one box a page
   int sk_rb_major;  // stream-K: segments ordered row block first (every block the same
                    // number of tiles a request)
+  int replan;  // dependent-launch test: the stream-K kernel treats its first plan as stale
   int stall;  // failure-detection test: the producers issue no copies, so the first
               // wait runs out (stream-K and tcgen05 kernels)
 };

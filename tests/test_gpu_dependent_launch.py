@@ -152,3 +152,58 @@ def test_attend_chain_reads_the_previous_output(paged):
     else:
         K, V = kp, vp
     H.compare(first, o.attend(q, K, V, L, case.scale, H.ORACLE_DT[case.dtype]), "first link")
+
+
+REPLAN = {
+    # 4 rows per KV head, contiguous bf16 D 128
+    "gqa_contig": lambda: W.contig_case("rp1", 5, 32, 8, 128, "bf16", 1,
+                                        [4000, 63, 0, 1300, 64], seed=801, max_T=4100),
+    # 2 rows per KV head, paged fp16 D 64, pages of 16 (one box a page) and a verify chunk
+    "paged_d64_t2": lambda: W.paged_case("rp2", 4, 8, 8, 64, "fp16", 2, 0, 1500, 16,
+                                         seed=802, pool_seed=803),
+    # MHA decode, one row per KV head
+    "mha_d64": lambda: W.contig_case("rp3", 4, 12, 12, 64, "fp16", 1, [2047, 1, 900, 4095],
+                                     seed=804, max_T=4100),
+}
+
+
+@pytest.mark.parametrize("kind", sorted(REPLAN))
+def test_replan_after_the_wait_gives_identical_results(kind):
+    """kvc_inject_replan makes the stream-K kernel treat the plan it made before its
+    dependency wait as stale: the copies it issued from that plan are drained, the
+    pipeline barriers reset and the range planned again.  Outputs (attend, and the fused
+    append + attend with the cache it writes) are bit-identical to the ordinary path's."""
+    case = REPLAN[kind]()
+    run = H.GpuRun(case)
+    try:
+        run.load_pools(0, case.k_pool(0), case.v_pool(0))
+        assert_stream_k(run, case)
+        dt = case.dtype
+        q_d = H.to_device(case.q(0), dt)
+        k_d, v_d = H.to_device(case.k_new(0), dt), H.to_device(case.v_new(0), dt)
+        outs, pools = [], []
+        for replan in (False, True, False):
+            if replan:
+                run.cache.inject_replan()
+            out = run.cache.append_attend(0, k_d, v_d, q_d, run.seq_lens, run.block_table,
+                                          scale=case.scale)
+            torch.cuda.synchronize()
+            assert run.cache.get_error() == kvc.KVC_OK
+            outs.append(out)
+            pools.append(run.pools(0))
+        for replan in (True, False):
+            if replan:
+                run.cache.inject_replan()
+            outs.append(run.cache.attend(0, q_d, run.seq_lens, run.block_table,
+                                         scale=case.scale))
+            torch.cuda.synchronize()
+            assert run.cache.get_error() == kvc.KVC_OK
+        for o in outs[1:]:
+            assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+        for kp, vp in pools[1:]:
+            assert np.array_equal(kp, pools[0][0]) and np.array_equal(vp, pools[0][1])
+        kref, vref = H.oracle_pools_after_append(case)
+        sel, ref = H.oracle_attend(case, kref, vref, case.q(0))
+        H.compare(H.out_to_f64(outs[1])[sel], ref, f"{kind} after a replan")
+    finally:
+        run.close()
