@@ -504,11 +504,14 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     call_s = res["call_ms_median"] * 1e-3
     step_call_s = ms * 1e-3 / c.layers  # one layer-step's share of the graph-timed step
     peak, peak_kind = peaks()
-    if kernel.startswith("attend_tc"):
-        tpeak, tpeak_kind = tensor_peak()
+    tpeak, tpeak_kind = tensor_peak()
+    # the binding roof: the longer of the bytes' time at the HBM peak and the attention
+    # flops' time at the dense bf16 peak (the tensor roof binds from about 240 flop/B,
+    # i.e. about 240 query rows per KV head)
+    if flops / (tpeak * 1e12) > call_bytes / (peak * 1e9):
         roof = {"bound": "tensor", "achieved": flops / call_s / 1e12, "peak": tpeak,
-                "unit": "TFLOP/s", "traffic": None, "peak_source": tpeak_kind,
-                "achieved_in_step": flops / step_call_s / 1e12}
+                "unit": "TFLOP/s", "traffic": profiled_traffic(kernel),
+                "peak_source": tpeak_kind, "achieved_in_step": flops / step_call_s / 1e12}
     else:
         roof = {"bound": "hbm", "achieved": call_bytes / call_s / 1e9, "peak": peak,
                 "unit": "GB/s", "traffic": profiled_traffic(kernel), "peak_source": peak_kind,
