@@ -213,6 +213,27 @@ def test_fp8_append_attend_fused(D, paged):
         r.close()
 
 
+def test_fp8_gqa_b16_l4096_one_layer_full_fused():
+    """One layer of the 32-layer GQA decode on an FP8 cache at full size, through the
+    bench's launch (kvc_append_attend: the kernel quantises the new rows): codes and
+    scales bit-exact, every request's attention within tolerance."""
+    case = W.gqa_32layer(layers=1)
+    r = Fp8Run(case)
+    try:
+        q = case.q(0)
+        out = r.cache.append_attend(0, H.to_device(case.k_new(0), "bf16"),
+                                    H.to_device(case.v_new(0), "bf16"),
+                                    H.to_device(q, "bf16"), r.seq_lens, None, scale=case.scale)
+        assert r.cache.get_error() == kvc.KVC_OK
+        r.o.append_fp8(r.img["kc"], r.img["ks"], case.k_new(0), case.seq_lens, None)
+        r.o.append_fp8(r.img["vc"], r.img["vs"], case.v_new(0), case.seq_lens, None)
+        r.check_pools()
+        sel, ref = r.reference(q)
+        H.compare(H.out_to_f64(out)[sel], ref, "fp8 GQA B16 L4096 fused")
+    finally:
+        r.close()
+
+
 def test_fp8_long_context():
     case = W.paged_case("fp8long", 2, 32, 8, 128, "bf16", 1, 20000, 30000, 16, seed=121,
                         pool_seed=122)

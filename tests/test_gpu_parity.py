@@ -260,6 +260,18 @@ def test_gqa_b16_l4096_one_layer_full():
     run_case(W.gqa_32layer(layers=1))
 
 
+def test_gqa_b16_l4096_one_layer_full_fused():
+    """The bench's launch at full size: kvc_append_attend (append fused into the persistent
+    kernel, dependent launch), pools bit-exact and every request checked."""
+    run_case(W.gqa_32layer(layers=1), fused=True)
+
+
+@pytest.mark.parametrize("L", [4096, 8192])
+def test_mha_b4_h12_d64_fused_full(L):
+    """MHA decode at full size through the bench's launch (kvc_append_attend)."""
+    run_case(W.mha_sweep(L), fused=True)
+
+
 def test_gqa_b16_l4096_layer_offsets():
     """Layers are independent pools: layer 3 of a 4-layer cache gives the same check."""
     case = W.gqa_32layer(layers=4)
@@ -273,6 +285,14 @@ def test_paged_gqa_b64_full():
     sh = list(case.shared_requests[:8])
     others = [b for b in range(case.B) if b not in case.shared_requests][:8]
     run_case(case, requests=sorted(sh + others))
+
+
+def test_paged_gqa_b64_full_fused():
+    """Paged GQA decode at full size through the bench's launch (kvc_append_attend)."""
+    case = W.paged_gqa()
+    sh = list(case.shared_requests[:8])
+    others = [b for b in range(case.B) if b not in case.shared_requests][-8:]
+    run_case(case, requests=sorted(sh + others), fused=True)
 
 
 @pytest.mark.parametrize("gamma", [2, 4, 8])
