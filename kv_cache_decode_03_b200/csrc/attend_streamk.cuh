@@ -76,8 +76,11 @@
 #ifndef KVC_SK_LOOKAHEAD
 #define KVC_SK_LOOKAHEAD 1
 #endif
-#ifndef KVC_SK_PREFETCH_TILES
+#ifndef KVC_SK_PREFETCH_TILES  // tiles of its range a CTA warms in L2 before the wait
 #define KVC_SK_PREFETCH_TILES 2
+#endif
+#ifndef KVC_SK_PREFETCH_TILES_PAGED  // the same on a paged cache (measured: 1 beats 2 there)
+#define KVC_SK_PREFETCH_TILES_PAGED 1
 #endif
 
 namespace kvc {
@@ -551,7 +554,7 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
     // only boxes wholly inside the tensor: the cursor may walk off stale lengths
     const long long rows_total =
         PAGED ? (long long)p.num_pages * p.H_kv * Pg : (long long)p.B * p.H_kv * p.max_T;
-    const int pf = min(ntiles, KVC_SK_PREFETCH_TILES);
+    const int pf = min(ntiles, PAGED ? KVC_SK_PREFETCH_TILES_PAGED : KVC_SK_PREFETCH_TILES);
     TileCursor<R> pc = cur;
 #pragma unroll 1
     for (int i = 0; i < max(pf, 1) && pc.b < p.B; ++i) {

@@ -109,7 +109,7 @@ constexpr int kEltBytes = 2;
 #define KVC_SK_PENALTY_D128 3
 #endif
 #ifndef KVC_SK_PENALTY_D64
-#define KVC_SK_PENALTY_D64 2
+#define KVC_SK_PENALTY_D64 4
 #endif
 // tcgen05 rows (64+ per KV head) without a window run on the persistent stream-K
 // tcgen05 kernel; its penalty tiles charge a piece's Q reload, TMEM readout and partial.
