@@ -106,7 +106,7 @@ constexpr int kEltBytes = 2;
 // epilogue, ticket, a fresh q and a ring restart, measured at about two to four tiles'
 // streaming time), so CTAs that cross segment boundaries get fewer real tiles.
 #ifndef KVC_SK_PENALTY_D128
-#define KVC_SK_PENALTY_D128 3
+#define KVC_SK_PENALTY_D128 4
 #endif
 #ifndef KVC_SK_PENALTY_D64
 #define KVC_SK_PENALTY_D64 4
