@@ -458,25 +458,52 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     if cache.get_error() != kvc.KVC_OK:
         raise RuntimeError("device error in the timed region")
 
-    # ---- e2e: pinned host buffers, copies inside the timed region
+    # ---- e2e: pinned host buffers, every step's copies inside the timed region.  Two
+    # device buffer sets and a copy stream, as a serving loop runs it: step i+1's inputs
+    # go in, and step i's output comes out, while the compute stream runs the step.
     if e2e:
         hq = qs.cpu().pin_memory()
         hk = ks.cpu().pin_memory()
         hv = vs.cpu().pin_memory()
         ho = torch.empty(outs.shape, dtype=tdt).pin_memory()
-        dq, dk, dv = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
+        bufs = [(torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs),
+                 torch.empty_like(outs)) for _ in range(2)]
+        copy_stream = torch.cuda.Stream()
         e2e_steps = max(3, steps // 4)
+        ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer set landed
+        ev_run = [torch.cuda.Event() for _ in range(2)]   # step on buffer set finished
+        ev_out = [torch.cuda.Event() for _ in range(2)]   # its output copied out
+        def h2d(i):  # step i's inputs into buffer set i % 2 (copy stream, in order)
+            dq, dk, dv, _ = bufs[i % 2]
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            ev_in[i % 2].record(copy_stream)
+
         reps.barrier()
         torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(e2e_steps):
-                dq.copy_(hq, non_blocking=True)
-                dk.copy_(hk, non_blocking=True)
-                dv.copy_(hv, non_blocking=True)
-                step(dq, dk, dv, outs)
-                ho.copy_(outs, non_blocking=True)
-            e1.record(stream)
+        e0.record(stream)
+        copy_stream.wait_event(e0)
+        with torch.cuda.stream(copy_stream):
+            h2d(0)
+        for i in range(e2e_steps):
+            j = i % 2
+            dq, dk, dv, do = bufs[j]
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev_in[j])
+                step(dq, dk, dv, do)
+                ev_run[j].record(stream)
+            with torch.cuda.stream(copy_stream):
+                # the next step's inputs go in while this step runs (their set was last
+                # used by step i - 1, whose output copy is queued ahead of them) ...
+                if i + 1 < e2e_steps:
+                    h2d(i + 1)
+                # ... and this step's output comes out while the next one runs
+                copy_stream.wait_event(ev_run[j])
+                ho.copy_(do, non_blocking=True)
+                ev_out[j].record(copy_stream)
+        stream.wait_event(ev_out[(e2e_steps - 1) % 2])
+        e1.record(stream)
         e1.synchronize()
         reps.barrier()
         res["e2e_ms"] = reps.max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
