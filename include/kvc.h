@@ -153,13 +153,14 @@ kvc_status kvc_append(kvc_cache* cache, int layer, const void* k_new, const void
  * owned by the cache for split-K partial results; it grows on demand (a device
  * allocation, so the first call with a larger shape should precede any stream capture;
  * kvc_reserve sizes it up front).
- * Launch: when the plan picks the persistent stream-K kernel (D 64/128, 1-16 query rows
- * per KV head, no window), it is launched with programmatic stream serialization.  It
- * may start while the kernel ahead of it on the stream retires, but reads no input that
- * counts and writes nothing before that kernel has completed (before that it only reads
- * seq_lens and the block table to plan, and prefetches K/V lines into L2).  The
- * environment variable KVC_PDL=0 (read at kvc_create) or kvc_set_dependent_launch
- * turns this into a plain launch.
+ * Launch: when the plan picks a persistent kernel (no window; D 64/128; stream-K on
+ * mma.sync for 1-16 query rows per KV head, 1-8 on an FP8 cache; stream-K on tcgen05
+ * for 17 or more), it is launched with programmatic stream serialization.  It may start
+ * while the kernel ahead of it on the stream retires, but reads no input that counts and
+ * writes nothing before that kernel has completed (before that it only reads seq_lens
+ * and the block table to plan, and prefetches K/V lines into L2; if the lengths changed
+ * by then, it plans again).  The environment variable KVC_PDL=0 (read at kvc_create) or
+ * kvc_set_dependent_launch turns this into a plain launch.
  */
 kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
                       const int32_t* block_table, int max_pages, const int32_t* seq_lens,
@@ -184,10 +185,11 @@ kvc_status kvc_attend_window(kvc_cache* cache, int layer, const void* q, int H_q
  * kvc_append_attend -- kvc_append followed by kvc_attend for the same new tokens, in
  * one launch where the kernel allows it ("9. 推理" 9.3: the new token's K/V join the
  * cache and are attended in the same step).  Arguments are those of the two calls.
- * With up to 16 query rows per KV head on the tensor-core path the attend kernel itself
- * writes the new rows into the cache and uses them straight from k_new / v_new; in other
- * cases the two kernels run back to back on `stream`.  Results (cache contents and out)
- * are identical to calling kvc_append then kvc_attend.
+ * On the persistent mma.sync stream-K kernel (up to 16 query rows per KV head, up to 8
+ * on an FP8 cache) the attend kernel itself writes the new rows into the cache (an FP8
+ * cache: quantised exactly as kvc_append does) and uses them straight from k_new /
+ * v_new; in other cases the two kernels run back to back on `stream`.  Results (cache
+ * contents and out) are identical to calling kvc_append then kvc_attend.
  */
 kvc_status kvc_append_attend(kvc_cache* cache, int layer, const void* k_new, const void* v_new,
                              const void* q, int H_q, int T_new, const int32_t* block_table,
@@ -229,7 +231,7 @@ kvc_status kvc_reserve(kvc_cache* cache, int H_q, int T_new, int max_pages);
 kvc_status kvc_get_error(kvc_cache* cache);
 
 /*
- * kvc_set_dependent_launch -- launch this cache's persistent stream-K attend kernel with
+ * kvc_set_dependent_launch -- launch this cache's persistent attend kernels with
  * programmatic stream serialization (on != 0; the default unless the environment
  * variable KVC_PDL=0) or as a plain launch (on == 0).  Results are the same either way;
  * see kvc_attend.
@@ -328,9 +330,10 @@ kvc_status kvc_copy_pages(kvc_cache* cache, const int32_t* src, const int32_t* d
 /*
  * kvc_plan_splits -- how kvc_attend would divide the work for these arguments (for
  * measurement and tests).  Fixed-size split-K: *num_splits slices of *split_tokens tokens
- * per (request, KV head).  Persistent stream-K (up to 16 query rows per KV head with the
- * tensor-core path): *num_splits is the number of persistent CTAs, each streaming an equal
- * share of all K/V tiles, and *split_tokens is 0.
+ * per (request, KV head).  Persistent stream-K (no window, D 64/128, B up to the
+ * kernel's scan capacity; any number of query rows per KV head, at most 8 on an FP8
+ * cache): *num_splits is the number of persistent CTAs, each streaming an equal share of
+ * all K/V tiles, and *split_tokens is 0.
  */
 kvc_status kvc_plan_splits(const kvc_cache* cache, int H_q, int T_new, int max_pages,
                            int* num_splits, int* split_tokens);
