@@ -33,15 +33,19 @@
 //   most two partial pieces (its first and its last); they go to slots
 //   (c, 0) and (c, 1) of the workspace, and the last CTA of a segment to
 //   finish merges the segment's pieces by log-sum-exp ("9. 推理" 9.7:
-//   exact up to rounding); an atomic ticket after a release fence decides
-//   who is last, so nothing ever waits on another CTA.  The merge spreads each
-//   output quad's pieces over up to eight threads, so all of its loads are in
-//   flight at once, and combines them with shuffles.
+//   exact up to rounding); a release-acquire ticket decides who is last (its
+//   result is read only at the CTA's next piece end or after its loop), so
+//   nothing ever waits on another CTA.  The merge spreads each output quad's
+//   pieces over up to eight threads, so all of its loads are in flight at once,
+//   and combines them with shuffles.
 // * Launched with programmatic stream serialization, a CTA sets up its
 //   barriers, plans its tile range from the lengths as they stand and
 //   prefetches the first tiles of that range into L2 while the grid ahead
-//   finishes; after the dependency wait it re-reads the lengths and keeps the
-//   plan when none changed.
+//   finishes; right after the dependency wait it issues its first stages from
+//   that plan while it re-reads the lengths, and if any changed it waits for
+//   those copies, resets its barriers and plans again.
+// * FP8 (a compile-time variant, 1-8 rows): the stages carry E4M3 codes and
+//   per-row scales, and the tile arithmetic is that of attend_fp8.cuh.
 #pragma once
 
 #include <cuda.h>
@@ -68,9 +72,9 @@
 #ifndef KVC_SK_STAGES_D64
 #define KVC_SK_STAGES_D64 KVC_SK_STAGES
 #endif
-// Tiles of its range a CTA prefetches into L2 before the dependency wait (measured:
-// 2 beats 0, 1, 3 and 5: more delays the CTAs that start late and competes with the
-// grid ahead for HBM).
+// Tiles of its range a CTA prefetches into L2 before the dependency wait (measured on
+// contiguous caches: 2 beats 0, 1, 3 and 5: more delays the CTAs that start late and
+// competes with the grid ahead for HBM; paged caches: 1 beats 0 and 2).
 // Paged: tiles ahead of the next copy whose page ids are already being read (measured:
 // 3 is no faster than 1 once a page is one box).
 #ifndef KVC_SK_LOOKAHEAD
