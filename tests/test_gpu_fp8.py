@@ -234,6 +234,32 @@ def test_fp8_gqa_b16_l4096_one_layer_full_fused():
         r.close()
 
 
+def test_fp8_streamk_wait_that_runs_out():
+    """Failure detection on the FP8 stream-K variant: with the next call's copies withheld
+    (kvc_inject_stall) and a 2 ms wait limit, the call returns, KVC_ERR_TIMEOUT is
+    reported, and the next call on the same cache is correct."""
+    case = W.paged_case("fp8stall", 4, 16, 4, 128, "bf16", 1, 100, 1500, 16, seed=161,
+                        pool_seed=162)
+    r = Fp8Run(case)
+    try:
+        ns, split_tokens = r.cache.plan(case.H_q, case.T_new, case.max_pages)
+        assert split_tokens == 0, "expected the persistent stream-K plan"
+        r.append()
+        q = case.q(0)
+        qd = H.to_device(q, "bf16")
+        r.cache.set_wait_limit(2_000_000)
+        r.cache.inject_stall()
+        r.cache.attend(0, qd, r.seq_lens, r.bt, scale=case.scale)
+        assert r.cache.get_error() == kvc.KVC_ERR_TIMEOUT
+        r.cache.set_wait_limit(0)
+        out = r.cache.attend(0, qd, r.seq_lens, r.bt, scale=case.scale)
+        assert r.cache.get_error() == kvc.KVC_OK
+        sel, ref = r.reference(q)
+        H.compare(H.out_to_f64(out)[sel], ref, "fp8 stream-K after a timeout")
+    finally:
+        r.close()
+
+
 def test_fp8_long_context():
     case = W.paged_case("fp8long", 2, 32, 8, 128, "bf16", 1, 20000, 30000, 16, seed=121,
                         pool_seed=122)
