@@ -517,7 +517,12 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     layer_bytes = fp8_algorithmic_bytes(c) if fp8 else c.algorithmic_bytes()
     res["layer_bytes"] = layer_bytes
     res["step_bytes"] = c.layers * layer_bytes
-    res["launches_per_step"] = c.layers * (1 if fused else 2)
+    # tcgen05 stream-K (17+ rows) with large segment merges: append, attend, combine
+    rows = (c.H_q // c.H_kv) * c.T_new
+    segs = c.B * c.H_kv * -(-rows // 128)
+    combine = (split_tokens == 0 and rows > 16 and not fp8 and
+               ns / segs * min(rows, 128) * c.D * 4 > 400 * 1024)
+    res["launches_per_step"] = c.layers * (1 if fused else 3 if combine else 2)
     res["ns"], res["split_tokens"] = ns, split_tokens
     # one call's bytes: K/V read + q read + out written + k_new/v_new read + rows written
     # (the FP8 count already holds both sides of the append)
@@ -546,7 +551,9 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["frac_in_step"] = roof["achieved_in_step"] / roof["peak"]
     roof["kernel"] = (kernel + (", fused: one launch per kvc_append_attend call (append, "
-                                "split attend, merge)" if fused else ", after the append kernel"))
+                                "split attend, merge)" if fused else
+                                ", after the append kernel and before its combine launch"
+                                if combine else ", after the append kernel"))
     roof["duration"] = (f"median of {len(durs)} event-bracketed kvc_append_attend calls "
                         f"({res['call_ms_median'] * 1e3:.2f} us; each call alone, so without "
                         f"the overlap of the dependent launch); achieved_in_step = the "

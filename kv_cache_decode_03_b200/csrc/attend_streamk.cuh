@@ -272,16 +272,15 @@ struct RangeMap {
 // sub, sub + tpq, ..., issuing the lse and the float4 of four pieces before using
 // any, with a running maximum; the group then combines its lanes' (max, sum, acc)
 // with xor shuffles.  A merge is thus about one L2 round trip, not one per piece.
-template <typename T, int D, int R, int NTH>
-__device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const RangeMap& rm,
-                                                    long long rf, long long rl, long long s0,
-                                                    int nr, size_t row_base) {
+// merge_rows_spread merges rows r_off .. r_off + nr - 1 of the npc pieces from range rf
+// (rf_mid: piece 0 sits in its range's second slot) into outputs from row row_base +
+// r_off; merge_pieces_spread merges a whole segment's rows.
+template <typename T, int D, int NTH>
+__device__ __forceinline__ void merge_rows_spread(const AttendParams& p, long long rf, int npc,
+                                                  bool rf_mid, int r_off, int nr,
+                                                  size_t row_base) {
   constexpr int Q4 = D / 4;
   const int tid = threadIdx.x;
-  const int npc = (int)(rl - rf + 1);
-  // range rf streamed real tiles of an earlier segment first iff it began before this
-  // segment's penalty tiles
-  const bool rf_mid = rm.start(rf) < s0 - p.sk_penalty;
   const int items = nr * Q4;
   int tpq = 1;
   while (tpq < 8 && tpq < npc && items * tpq * 2 <= NTH) tpq *= 2;
@@ -305,9 +304,9 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
         const int q = q0 + u * tpq;
         if (q < npc) {
           const size_t slot = (size_t)(rf + q) * 2 + ((q == 0 && rf_mid) ? 1 : 0);
-          ls[u] = __ldcg(p.ws_lse + slot * p.sk_slot_rows + rr);
-          v[u] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (slot * p.sk_slot_rows + rr) * D +
-                                                        d));
+          const size_t srow = slot * p.sk_slot_rows + r_off + rr;
+          ls[u] = __ldcg(p.ws_lse + srow);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + srow * D + d));
         } else {
           ls[u] = -INFINITY;
           v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -355,13 +354,23 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
     }
     if (act && sub == 0) {
       const float inv = den > 0.f ? 1.f / den : 0.f;
-      T* o = out + (row_base + rr) * D + d;
+      T* o = out + (row_base + r_off + rr) * D + d;
       store_elt<T>(o, acc.x * inv);
       store_elt<T>(o + 1, acc.y * inv);
       store_elt<T>(o + 2, acc.z * inv);
       store_elt<T>(o + 3, acc.w * inv);
     }
   }
+}
+
+template <typename T, int D, int R, int NTH>
+__device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const RangeMap& rm,
+                                                    long long rf, long long rl, long long s0,
+                                                    int nr, size_t row_base) {
+  // range rf streamed real tiles of an earlier segment first iff it began before this
+  // segment's penalty tiles
+  const bool rf_mid = rm.start(rf) < s0 - p.sk_penalty;
+  merge_rows_spread<T, D, NTH>(p, rf, (int)(rl - rf + 1), rf_mid, 0, nr, row_base);
 }
 
 // FP8 = true (NT 1, bf16 q and out): the stages carry E4M3 codes and scales and the

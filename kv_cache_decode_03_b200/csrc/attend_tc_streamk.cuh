@@ -38,6 +38,11 @@
 
 namespace kvc {
 
+// ints of a segment's combine descriptor (in the workspace after the lse values):
+// generation, valid rows, first range, pieces, first piece in its range's second slot,
+// output row (2 ints), pad
+constexpr int kCombineDescInts = 8;
+
 template <int D>
 struct TcSkCfg {
   using C = TcCfg<D>;
@@ -259,6 +264,27 @@ __device__ __forceinline__ void tc_merge_final(const AttendParams& p, const Rang
     __syncthreads();  // the window is read: it may be refilled
     if (tid == 0 && win + 2 < nwin) issue(win + 2);
   }
+}
+
+// Combine launch (after attend_tc_streamk_kernel with p.sk_combine != 0): block
+// (segment, 16-row chunk) merges that chunk of the segment's pieces by log-sum-exp
+// ("9. 推理" 9.7) with merge_rows_spread.  A segment whose descriptor does not carry this
+// call's generation was written whole (or has no tiles) and is skipped.  Launched
+// dependently: it waits for the attend grid before reading anything.
+constexpr int kCombineRows = 16;
+template <typename T, int D>
+__global__ void __launch_bounds__(128) combine_kernel(const AttendParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const size_t segi = blockIdx.x;
+  const int* d = p.sk_desc + segi * kCombineDescInts;
+  if (d[0] != p.sk_combine) return;
+  const int nr = d[1];
+  const int r_off = blockIdx.y * kCombineRows;
+  if (r_off >= nr) return;
+  const size_t row_base = (size_t)(uint32_t)d[5] | ((size_t)(uint32_t)d[6] << 32);
+  merge_rows_spread<T, D, 128>(p, d[2], d[3], d[4] != 0, r_off, min(kCombineRows, nr - r_off),
+                               row_base);
 }
 
 template <int D, typename T, bool PAGED>
@@ -643,7 +669,23 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
           nc.next(p, PAGED);
           stage_q(nc);
         }
-        if (!whole) {
+        if (!whole && p.sk_combine) {
+          // a combine launch merges the segment: the piece holding its first tile leaves
+          // the descriptor (read only after this grid has completed)
+          if (tid == 0 && piece_first_j == j - sc.k) {
+            const long long s0 = sc.seg_start, s1 = sc.seg_start + sc.seg_tiles - 1;
+            const long long rf = rm.of(s0), rl = rm.of(s1);
+            const size_t segi = ((size_t)sc.b * p.H_kv + sc.g) * p.row_blocks + sc.rb;
+            int* d = p.sk_desc + segi * kCombineDescInts;
+            d[1] = nr;
+            d[2] = (int)rf;
+            d[3] = (int)(rl - rf + 1);
+            d[4] = rm.start(rf) < s0 - p.sk_penalty ? 1 : 0;
+            d[5] = (int)(row_base & 0xffffffffu);
+            d[6] = (int)(row_base >> 32);
+            d[0] = p.sk_combine;
+          }
+        } else if (!whole) {
           // hand the piece to the segment's last finisher: the barrier orders every
           // row's partial stores before thread 0's release-acquire ticket
           named_barrier_sync(1, NSM);

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -79,6 +80,16 @@ constexpr int kEltBytes = 2;
 // wave's imbalance is a small fraction of the pass.
 #ifndef KVC_SPLIT_WAVES
 #define KVC_SPLIT_WAVES 4
+#endif
+#ifndef KVC_TC_COMBINE  // tcgen05 stream-K: partial pieces merged by a separate combine launch
+#define KVC_TC_COMBINE 1
+#endif
+// ... when a segment's partials average more than this many bytes: one CTA merging them
+// in the attend kernel takes ~20 us at 600 KB (a trace), the combine launch a few us and
+// its own overhead (measured: MQA verify gamma 4, 600 KB a segment, +10 %; gamma 2 and 8,
+// 300 KB, -4 % and +1 %)
+#ifndef KVC_TC_COMBINE_MIN_BYTES
+#define KVC_TC_COMBINE_MIN_BYTES (400 << 10)
 #endif
 #ifndef KVC_TC_RB_MAJOR
 #define KVC_TC_RB_MAJOR 1
@@ -457,6 +468,7 @@ struct Plan {
   bool tc;           // tcgen05 kernel, 128 query rows per CTA
   bool mma;          // mma.sync tensor-core kernel (else the CUDA-core kernel)
   bool streamk;      // mma: persistent stream-K kernel (grid = resident CTAs)
+  bool combine;      // tcgen05 stream-K: segments merged by a separate combine launch
   int grid;          // streamk: persistent CTAs
   size_t slots;      // streamk: partial-result slots (slot_rows rows x D each) in the workspace
   int slot_rows;     // streamk: rows of a slot
@@ -575,7 +587,11 @@ Plan make_plan(const kvc_cache* c, int H_q, int T_new, int max_pages, int window
     pl.num_splits = 1;
     pl.ws_partial_floats = pl.slots * pl.slot_rows * (c->D + 1);
     pl.ws_counters = (size_t)c->B * c->H_kv * pl.row_blocks;
-    pl.ws_bytes = pl.ws_partial_floats * sizeof(float);
+    pl.combine = KVC_TC_COMBINE && (double)pl.grid / pl.ws_counters * pl.slot_rows * c->D *
+                                           sizeof(float) > (double)KVC_TC_COMBINE_MIN_BYTES;
+    // partial outputs, lse, then (combine launch) one descriptor a segment
+    pl.ws_bytes = pl.ws_partial_floats * sizeof(float) +
+                  (pl.combine ? pl.ws_counters * kvc::kCombineDescInts * sizeof(int) : 0);
     return pl;
   }
   const int fp8_max_batch = c->D == 64 ? kvc::StreamKCfg<64, true>::kMaxBatch
@@ -828,14 +844,35 @@ kvc_status launch_attend_tc_streamk(const kvc::AttendParams& p, int grid, bool p
       cudaLaunchKernelEx(&cfg, kvc::attend_tc_streamk_kernel<D, T, PAGED>, p, tk, tv));
 }
 
+// The combine launch after a tcgen05 stream-K attend (p.sk_combine != 0): one block
+// per (segment, 16-row chunk), dependent on the attend grid.
+template <int D, typename T>
+kvc_status launch_combine(const kvc::AttendParams& p, bool pdl, cudaStream_t stream) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  const int segs = p.B * p.H_kv * p.row_blocks;
+  cfg.gridDim = dim3(segs, kvc::ceil_div(p.sk_slot_rows, kvc::kCombineRows));
+  cfg.blockDim = dim3(128);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kvc::combine_kernel<T, D>, p));
+}
+
 template <typename T>
 kvc_status dispatch_tc_streamk(const kvc::AttendParams& p, int D, bool paged, int grid, bool pdl,
                                const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  kvc_status st;
   if (D == 64)
-    return paged ? launch_attend_tc_streamk<64, T, true>(p, grid, pdl, tk, tv, s)
-                 : launch_attend_tc_streamk<64, T, false>(p, grid, pdl, tk, tv, s);
-  return paged ? launch_attend_tc_streamk<128, T, true>(p, grid, pdl, tk, tv, s)
+    st = paged ? launch_attend_tc_streamk<64, T, true>(p, grid, pdl, tk, tv, s)
+               : launch_attend_tc_streamk<64, T, false>(p, grid, pdl, tk, tv, s);
+  else
+    st = paged ? launch_attend_tc_streamk<128, T, true>(p, grid, pdl, tk, tv, s)
                : launch_attend_tc_streamk<128, T, false>(p, grid, pdl, tk, tv, s);
+  if (st != KVC_OK || p.sk_combine == 0) return st;
+  return D == 64 ? launch_combine<64, T>(p, pdl, s) : launch_combine<128, T>(p, pdl, s);
 }
 
 template <typename T>
@@ -925,6 +962,17 @@ kvc::AttendParams attend_params(kvc_cache* c, int layer, const void* q, int H_q,
   c->stall_next = false;
   p.replan = c->replan_next ? 1 : 0;
   c->replan_next = false;
+  if (pl.combine) {
+    // nonzero and new for every call of the process: descriptors left by another call
+    // (of any cache: kvc_attend_noalloc shares one scratch) never match
+    static std::atomic<int> gen{0};
+    int g = gen.fetch_add(1) + 1;
+    if (g <= 0) {  // wrapped
+      gen.store(1);
+      g = 1;
+    }
+    p.sk_combine = g;
+  }
   return p;
 }
 
@@ -933,6 +981,11 @@ float* lse_base(const kvc_cache* c, const Plan& pl, float* ws, int H_q, int T_ne
   if (!ws) return nullptr;
   return pl.streamk ? ws + pl.slots * pl.slot_rows * c->D
                     : ws + (size_t)c->B * H_q * T_new * pl.num_splits * c->D;
+}
+
+// Where the combine descriptors start (tcgen05 stream-K): after the slots' lse values.
+int* desc_base(const Plan& pl, float* lse) {
+  return (lse && pl.combine) ? reinterpret_cast<int*>(lse + pl.slots * pl.slot_rows) : nullptr;
 }
 
 // Launch the attend kernel a plan chose for layer `layer`.
@@ -1314,6 +1367,7 @@ kvc_status kvc_attend_window(kvc_cache* c, int layer, const void* q, int H_q, in
   p.sink = sink;
   p.ws_o = c->ws;
   p.ws_lse = lse_base(c, pl, c->ws, H_q, T_new);
+  p.sk_desc = desc_base(pl, p.ws_lse);
   p.counters = c->tickets;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return run_plan(c, layer, pl, p, s);
@@ -1444,6 +1498,7 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
       attend_params(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, out, pl);
   p.ws_o = ws;
   p.ws_lse = lse_base(c, pl, ws, H_q, T_new);
+  p.sk_desc = desc_base(pl, p.ws_lse);
   p.counters = static_cast<int*>(base);
   return run_plan(c, layer, pl, p, s);
 }
@@ -1482,6 +1537,7 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
       attend_params(c, layer, q, H_q, T_new, block_table, max_pages, seq_lens, scale, out, pl);
   p.ws_o = c->ws;
   p.ws_lse = lse_base(c, pl, c->ws, H_q, T_new);
+  p.sk_desc = desc_base(pl, p.ws_lse);
   p.counters = c->tickets;
   p.k_new = k_new;
   p.v_new = v_new;

@@ -56,6 +56,10 @@ struct AttendParams {
                    // (64 elements, page tokens, 2 halves, page blocks), one box a page
   int sk_rb_major;  // stream-K: segments ordered row block first (every block the same
                    // number of tiles a request)
+  int sk_combine;  // tcgen05 stream-K: partial pieces are merged by a separate combine
+                   // launch (combine_kernel); the value is this call's generation, which the
+                   // segment descriptors in sk_desc carry (0: last-finisher merges)
+  int* sk_desc;    // tcgen05 stream-K with sk_combine: kCombineDescInts ints a segment
   int replan;  // dependent-launch test: the stream-K kernel treats its first plan as stale
   int stall;  // failure-detection test: the producers issue no copies, so the first
               // wait runs out (stream-K and tcgen05 kernels)
