@@ -160,7 +160,9 @@ kvc_status kvc_append(kvc_cache* cache, int layer, const void* k_new, const void
  * writes nothing before that kernel has completed (before that it only reads seq_lens
  * and the block table to plan, and prefetches K/V lines into L2; if the lengths changed
  * by then, it plans again).  The environment variable KVC_PDL=0 (read at kvc_create) or
- * kvc_set_dependent_launch turns this into a plain launch.
+ * kvc_set_dependent_launch turns this into a plain launch.  On the tcgen05 path a
+ * segment whose partial results are large is merged by a second, dependent launch on
+ * `stream` (the combine); callers see one call either way.
  */
 kvc_status kvc_attend(kvc_cache* cache, int layer, const void* q, int H_q, int T_new,
                       const int32_t* block_table, int max_pages, const int32_t* seq_lens,
