@@ -45,7 +45,8 @@
 //   that plan while it re-reads the lengths, and if any changed it waits for
 //   those copies, resets its barriers and plans again.
 // * FP8 (a compile-time variant, 1-8 rows): the stages carry E4M3 codes and
-//   per-row scales, and the tile arithmetic is that of attend_fp8.cuh.
+//   per-row scales; the codes are converted in registers as in attend_fp8.cuh, and
+//   one running reference per row serves both the sum and the V-scaled weights.
 #pragma once
 
 #include <cuda.h>
@@ -374,8 +375,9 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
 }
 
 // FP8 = true (NT 1, bf16 q and out): the stages carry E4M3 codes and scales and the
-// tile arithmetic is that of attend_fp8.cuh (codes converted in registers, two running
-// maxima); planning, the ring, pieces, epilogue and merge are the same.
+// codes are converted in registers as in attend_fp8.cuh, with one running reference per
+// row (the maximum of s + max(log2 v_scale, -64)) for the sum and the weights; planning,
+// the ring, pieces, epilogue and merge are the same.
 template <int D, int NT, typename T, bool PAGED, bool FP8 = false>
 __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
                                   StreamKCfg<D, FP8>::template min_blocks<NT>())
@@ -827,7 +829,6 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
   int vis[NT][2];
   int r0 = 0, nr = 0, vis_min = 0, piece_first_j = 0;
   float m[NT][2], l[NT][2];
-  float mo[NT][2];    // FP8: the running maximum of s + log2(v_scale), the weights' reference
   float fcol[NT][2];  // FP8: score factor of the column's row: scale * log2(e) * 2^e_row
   float o[C::kMTiles][NT][4];
   // fresh running state; reset again at the end of every piece
@@ -837,7 +838,6 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         m[nt][cc] = -INFINITY;
-        mo[nt][cc] = -INFINITY;
         l[nt][cc] = 0.f;
       }
 #pragma unroll
@@ -1039,11 +1039,15 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
     const uint32_t vb = sv_addr + st * C::kTileBytes;
     const int t0 = cur.k * C::kTile;
     if constexpr (FP8) {
-      // E4M3 tile: scores and weights as in attend_fp8.cuh
+      // E4M3 tile: the codes converted as in attend_fp8.cuh
       const float* ssc = scl + st * 2 * C::kTile;
       const int ta = wrow + (lane >> 2);  // this thread's two tokens: ta and ta + 8
       const float ska = ssc[ta], skb = ssc[ta + 8];
       const float lva = __log2f(ssc[C::kTile + ta]), lvb = __log2f(ssc[C::kTile + ta + 8]);
+      // the reference of the row: the running maximum of s + max(log2 v_scale, -64), so
+      // the f16 weights 2^(s + log2 v_scale - m) stay <= 1 and the sum's terms 2^(s - m)
+      // stay below 2^64
+      const float lca = fmaxf(lva, -64.f), lcb = fmaxf(lvb, -64.f);
       // KVC_SK_FP8_CHAINS independent accumulator chains (chunk % chains), summed after:
       // shorter dependent MMA chains for the one n-tile
       constexpr int NCH = KVC_SK_FP8_CHAINS;
@@ -1092,28 +1096,19 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
             s0 = (tok0 < vis[nt][cc]) ? s0 : -INFINITY;
             s1 = (tok0 + 8 < vis[nt][cc]) ? s1 : -INFINITY;
           }
-          // the sum l, referenced to m
-          float mx = fmaxf(s0, s1);
+          float mx = fmaxf(s0 + lca, s1 + lcb);
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           const float m_new = fmaxf(m[nt][cc], mx);
           const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-          l[nt][cc] = fmaf(l[nt][cc], exp2f(m[nt][cc] - mu), exp2f(s0 - mu) + exp2f(s1 - mu));
+          alpha_o[nt][cc] = exp2f(m[nt][cc] - mu);
+          grew |= (m_new > m[nt][cc]);
           m[nt][cc] = m_new;
-          // the weights of O, referenced to mo: 2^(s + log2 v_scale - mo) <= 1
-          const float w0 = s0 + lva, w1 = s1 + lvb;
-          float mxo = fmaxf(w0, w1);
-          mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 4));
-          mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 8));
-          mxo = fmaxf(mxo, __shfl_xor_sync(0xffffffffu, mxo, 16));
-          const float mo_new = fmaxf(mo[nt][cc], mxo);
-          const float muo = (mo_new == -INFINITY) ? 0.f : mo_new;
-          alpha_o[nt][cc] = exp2f(mo[nt][cc] - muo);
-          grew |= (mo_new > mo[nt][cc]);
-          mo[nt][cc] = mo_new;
-          sacc[nt][cc] = exp2f(w0 - muo);
-          sacc[nt][2 + cc] = exp2f(w1 - muo);
+          // the sum l and the weights of O, both referenced to m
+          l[nt][cc] = fmaf(l[nt][cc], alpha_o[nt][cc], exp2f(s0 - mu) + exp2f(s1 - mu));
+          sacc[nt][cc] = exp2f(s0 + lva - mu);
+          sacc[nt][2 + cc] = exp2f(s1 + lvb - mu);
         }
       }
       if (__any_sync(0xffffffffu, grew)) {
@@ -1258,16 +1253,7 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
       constexpr int kHalfFloats = C::kTileBytes / 4;
       return idx < kHalfFloats ? red_acc + idx : red_acc_hi + (idx - kHalfFloats);
     };
-    // FP8: O referenced to m (O * 2^(mo - m)), its rows in vt_row_to_d order
-    float fo[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc)
-        fo[nt][cc] = !FP8 ? 1.f
-                     : (m[nt][cc] == -INFINITY || mo[nt][cc] == -INFINITY)
-                         ? 0.f
-                         : exp2f(mo[nt][cc] - m[nt][cc]);
+    // FP8: the rows of O come in vt_row_to_d order
 #pragma unroll
     for (int mt = 0; mt < C::kMTiles; ++mt)
 #pragma unroll
@@ -1277,7 +1263,7 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
           const int row = nt * 8 + (lane & 3) * 2 + (e & 1);
           const int rho = (lane >> 2) + (e >> 1) * 8;
           const int d = mt * 16 + (FP8 ? vt_row_to_d(rho) : rho);
-          *acc_at(warp, row, d) = FP8 ? o[mt][nt][e] * fo[nt][e & 1] : o[mt][nt][e];
+          *acc_at(warp, row, d) = o[mt][nt][e];
         }
     if (lane < 4) {
 #pragma unroll
