@@ -34,7 +34,7 @@ def out_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-class GpuRun:
+class DeviceCase:
     """A cache with the case's initial pools loaded, plus device copies of the per-step inputs."""
 
     def __init__(self, case: Case, layers: int = 1):

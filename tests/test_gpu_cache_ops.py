@@ -65,7 +65,7 @@ def test_commit_and_rollback_match_oracle():
 def test_copy_pages_bit_exact_all_layers():
     B, H_kv, D, P, layers = 4, 2, 128, 16, 3
     case = W.paged_case("copy", B, 8, H_kv, D, "bf16", 1, 100, 600, P, seed=41, pool_seed=42)
-    g = H.GpuRun(case, layers=layers)
+    g = H.DeviceCase(case, layers=layers)
     o = oracle.get()
     try:
         pools = []
@@ -126,7 +126,7 @@ def test_speculative_round_end_to_end(H_q, H_kv):
     nk = W.normal_bits((B, H_kv, 1, D), dtype, 55, "nk")
     nv = W.normal_bits((B, H_kv, 1, D), dtype, 55, "nv")
     nq = W.normal_bits((B, H_q, 1, D), dtype, 55, "nq")
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         kp, vp = case.k_pool(0), case.v_pool(0)
         g.load_pools(0, kp, vp)
@@ -183,7 +183,7 @@ def test_copy_on_write_then_append():
     nk = W.normal_bits((B, H_kv, 1, D), dtype, 63, "nk")
     nv = W.normal_bits((B, H_kv, 1, D), dtype, 63, "nv")
     q = W.normal_bits((B, H_q, 1, D), dtype, 63, "q")
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         g.load_pools(0, pool_k, pool_v)
         src = np.full(B - 1, n_shared - 1, np.int32)

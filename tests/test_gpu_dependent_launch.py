@@ -41,7 +41,7 @@ def make_case(paged: bool, seed: int) -> W.Case:
                          max_T=int(L.max()) + GAMMA + 2)
 
 
-def assert_stream_k(run: H.GpuRun, case: W.Case) -> None:
+def assert_stream_k(run: H.DeviceCase, case: W.Case) -> None:
     """The plan of a one-token step is the persistent stream-K kernel (the one launched
     dependently): no fixed split, a grid of at least one CTA per SM."""
     ns, split_tokens = run.cache.plan(case.H_q, 1, case.max_pages if case.paged else 0)
@@ -83,7 +83,7 @@ def test_length_kernel_then_attend(op, paged):
     nv = W.normal_bits((B, case.H_kv, 1, case.D), dt, case.seed + 2, "nv")
     nq = W.normal_bits((B, case.H_q, 1, case.D), dt, case.seed + 2, "nq")
     kp, vp = case.k_pool(0), case.v_pool(0)
-    run = H.GpuRun(case)
+    run = H.DeviceCase(case)
     try:
         run.load_pools(0, kp, vp)
         assert_stream_k(run, case)
@@ -119,7 +119,7 @@ def test_attend_chain_reads_the_previous_output(paged):
     q = W.normal_bits((case.B, case.H_q, 1, case.D), case.dtype, case.seed + 3, "q")
     kp, vp = case.k_pool(0), case.v_pool(0)
     links = 3
-    run = H.GpuRun(case)
+    run = H.DeviceCase(case)
     try:
         run.load_pools(0, kp, vp)
         assert_stream_k(run, case)
@@ -174,7 +174,7 @@ def test_replan_after_the_wait_gives_identical_results(kind):
     pipeline barriers reset and the range planned again.  Outputs (attend, and the fused
     append + attend with the cache it writes) are bit-identical to the ordinary path's."""
     case = REPLAN[kind]()
-    run = H.GpuRun(case)
+    run = H.DeviceCase(case)
     try:
         run.load_pools(0, case.k_pool(0), case.v_pool(0))
         assert_stream_k(run, case)

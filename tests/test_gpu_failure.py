@@ -41,7 +41,7 @@ CASES = {
 def test_wait_that_runs_out_reports_timeout(kind):
     case = CASES[kind]()
     ns, split_tokens = None, None
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         mp = case.max_pages if case.paged else 0
         ns, split_tokens = g.cache.plan(case.H_q, case.T_new, mp)
@@ -77,7 +77,7 @@ def test_wait_that_runs_out_reports_timeout(kind):
 def test_stall_is_consumed_by_one_call():
     """A stall affects only the next attend: a second call is unaffected."""
     case = CASES["streamk"]()
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         g.load_pools()
         g.append(0, case.k_new(0), case.v_new(0))
@@ -99,7 +99,7 @@ def test_dependent_launch_switch_gives_identical_results():
     """kvc_set_dependent_launch changes how the stream-K kernel is launched, not what it
     computes: outputs are bit-identical with and without programmatic serialization."""
     case = W.contig_case("pdl_switch", 4, 12, 12, 64, "fp16", 1, 3000, seed=95)
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         g.load_pools()
         g.append(0, case.k_new(0), case.v_new(0))

@@ -27,7 +27,7 @@ def run_case(case: W.Case, layer: int = 0, requests=None, check_pools: bool = Tr
              nthreads: int = 0, twice: bool = False, fused: bool = False):
     """Append + attend on the GPU (two calls, or kvc_append_attend when fused); compare
     pools bit-exactly and outputs within tolerance."""
-    g = H.GpuRun(case, layers=layer + 1)
+    g = H.DeviceCase(case, layers=layer + 1)
     try:
         kp0, vp0 = case.k_pool(layer), case.v_pool(layer)
         g.load_pools(layer, kp0, vp0)
@@ -191,7 +191,7 @@ def test_mha_b1_token_by_token_matches_full_causal():
     K = W.normal_bits((1, 16, T, 32), "fp16", case.seed, "tbt_k")
     V = W.normal_bits((1, 16, T, 32), "fp16", case.seed, "tbt_v")
     Q = W.normal_bits((1, 16, T, 32), "fp16", case.seed, "tbt_q")
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         rows = []
         for t in range(T):
@@ -226,7 +226,7 @@ def test_mha_b4_h12_d64_chunked_prefill(T, chunk):
     K = W.normal_bits((B, Hh, T, D), "fp16", 2, "prefill_k", T)
     V = W.normal_bits((B, Hh, T, D), "fp16", 2, "prefill_v", T)
     Q = W.normal_bits((B, Hh, T, D), "fp16", 2, "prefill_q", T)
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     out = np.empty((B, Hh, T, D))
     try:
         for s0 in range(0, T, chunk):
@@ -334,7 +334,7 @@ def test_device_bounds_flag_on_bad_page_id():
     bt = case.block_table.copy()
     bt[1, 1] = case.num_pages + 5  # outside the pool
     case.block_table = bt
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         g.load_pools(0)
         g.attend(0, case.q(0))
@@ -356,7 +356,7 @@ def test_device_bounds_flag_on_bad_page_id():
 
 def test_device_bounds_flag_on_capacity_overflow():
     case = W.contig_case("overflow", 2, 4, 4, 32, "fp16", 2, [10, 15], seed=22, max_T=16)
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         g.load_pools(0)
         before = g.pools(0)
@@ -402,7 +402,7 @@ def test_alternating_plans_share_one_cache():
     again on the same cache: each kernel's slice tickets must be left clean for the next."""
     import oracle
     base = W.paged_case("alt", 6, 32, 8, 128, "bf16", 8, 300, 6000, 16, seed=31, pool_seed=32)
-    g = H.GpuRun(base)
+    g = H.DeviceCase(base)
     try:
         kp, vp = base.k_pool(0), base.v_pool(0)
         g.load_pools(0, kp, vp)

@@ -23,7 +23,7 @@ if not torch.cuda.is_available():  # collected on CPU, skipped there
 
 
 def run_window(case: W.Case, window: int, sink: int, requests=None):
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         kp0, vp0 = case.k_pool(0), case.v_pool(0)
         g.load_pools(0, kp0, vp0)
@@ -94,7 +94,7 @@ def test_window_long_context(route):
 
 def test_window_zero_is_full_attention():
     case = W.paged_case("win0", 2, 8, 2, 128, "bf16", 2, 100, 900, 16, seed=73, pool_seed=74)
-    g = H.GpuRun(case)
+    g = H.DeviceCase(case)
     try:
         g.load_pools(0)
         g.append(0, case.k_new(0), case.v_new(0))
