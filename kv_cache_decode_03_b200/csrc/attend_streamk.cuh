@@ -376,8 +376,8 @@ __device__ __forceinline__ void merge_pieces_spread(const AttendParams& p, const
 
 // FP8 = true (NT 1, bf16 q and out): the stages carry E4M3 codes and scales and the
 // codes are converted in registers as in attend_fp8.cuh, with one running reference per
-// row (the maximum of s + max(log2 v_scale, -64)) for the sum and the weights; planning,
-// the ring, pieces, epilogue and merge are the same.
+// row (the maximum of s + max(exponent of v_scale, -64)) for the sum and the weights
+// v_scale * 2^(s - m); planning, the ring, pieces, epilogue and merge are the same.
 template <int D, int NT, typename T, bool PAGED, bool FP8 = false>
 __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
                                   StreamKCfg<D, FP8>::template min_blocks<NT>())
@@ -1043,11 +1043,13 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
       const float* ssc = scl + st * 2 * C::kTile;
       const int ta = wrow + (lane >> 2);  // this thread's two tokens: ta and ta + 8
       const float ska = ssc[ta], skb = ssc[ta + 8];
-      const float lva = __log2f(ssc[C::kTile + ta]), lvb = __log2f(ssc[C::kTile + ta + 8]);
-      // the reference of the row: the running maximum of s + max(log2 v_scale, -64), so
-      // the f16 weights 2^(s + log2 v_scale - m) stay <= 1 and the sum's terms 2^(s - m)
-      // stay below 2^64
-      const float lca = fmaxf(lva, -64.f), lcb = fmaxf(lvb, -64.f);
+      const float vsa = ssc[C::kTile + ta], vsb = ssc[C::kTile + ta + 8];
+      // the reference of the row: the running maximum of s + max(e_v, -64), e_v the binary
+      // exponent of the V scale (read off its bits: 2^e_v <= v_scale < 2^(e_v + 1)), so
+      // the f16 weights v_scale * 2^(s - m) stay below 2 and the sum's terms 2^(s - m)
+      // below 2^64
+      const float lca = fmaxf((float)(int)((__float_as_uint(vsa) >> 23) & 0xFFu) - 127.f, -64.f);
+      const float lcb = fmaxf((float)(int)((__float_as_uint(vsb) >> 23) & 0xFFu) - 127.f, -64.f);
       // KVC_SK_FP8_CHAINS independent accumulator chains (chunk % chains), summed after:
       // shorter dependent MMA chains for the one n-tile
       constexpr int NCH = KVC_SK_FP8_CHAINS;
@@ -1106,9 +1108,10 @@ __global__ void __launch_bounds__(StreamKCfg<D, FP8>::kThreads,
           grew |= (m_new > m[nt][cc]);
           m[nt][cc] = m_new;
           // the sum l and the weights of O, both referenced to m
-          l[nt][cc] = fmaf(l[nt][cc], alpha_o[nt][cc], exp2f(s0 - mu) + exp2f(s1 - mu));
-          sacc[nt][cc] = exp2f(s0 + lva - mu);
-          sacc[nt][2 + cc] = exp2f(s1 + lvb - mu);
+          const float e0 = exp2f(s0 - mu), e1 = exp2f(s1 - mu);
+          l[nt][cc] = fmaf(l[nt][cc], alpha_o[nt][cc], e0 + e1);
+          sacc[nt][cc] = e0 * vsa;
+          sacc[nt][2 + cc] = e1 * vsb;
         }
       }
       if (__any_sync(0xffffffffu, grew)) {
