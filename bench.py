@@ -517,11 +517,12 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     layer_bytes = fp8_algorithmic_bytes(c) if fp8 else c.algorithmic_bytes()
     res["layer_bytes"] = layer_bytes
     res["step_bytes"] = c.layers * layer_bytes
-    # tcgen05 stream-K (17+ rows) with large segment merges: append, attend, combine
+    # tcgen05 stream-K (17+ rows) with large segment merges: append, attend, combine (the
+    # library's default threshold: partials above 64 KB a segment on average)
     rows = (c.H_q // c.H_kv) * c.T_new
     segs = c.B * c.H_kv * -(-rows // 128)
     combine = (split_tokens == 0 and rows > 16 and not fp8 and
-               ns / segs * min(rows, 128) * c.D * 4 > 400 * 1024)
+               ns / segs * min(rows, 128) * c.D * 4 > 64 * 1024)
     res["launches_per_step"] = c.layers * (1 if fused else 3 if combine else 2)
     res["ns"], res["split_tokens"] = ns, split_tokens
     # one call's bytes: K/V read + q read + out written + k_new/v_new read + rows written

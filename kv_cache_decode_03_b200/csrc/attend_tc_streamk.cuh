@@ -267,11 +267,17 @@ __device__ __forceinline__ void tc_merge_final(const AttendParams& p, const Rang
 }
 
 // Combine launch (after attend_tc_streamk_kernel with p.sk_combine != 0): block
-// (segment, 16-row chunk) merges that chunk of the segment's pieces by log-sum-exp
-// ("9. 推理" 9.7) with merge_rows_spread.  A segment whose descriptor does not carry this
-// call's generation was written whole (or has no tiles) and is skipped.  Launched
-// dependently: it waits for the attend grid before reading anything.
-constexpr int kCombineRows = 16;
+// (segment, chunk of KVC_TC_COMBINE_ROWS rows) merges that chunk of the segment's pieces
+// by log-sum-exp ("9. 推理" 9.7) with merge_rows_spread.  A segment whose descriptor does
+// not carry this call's generation was written whole (or has no tiles) and is skipped.
+// Launched dependently: it waits for the attend grid before reading anything.  Small
+// chunks keep each thread's chain of dependent partial loads short (4 rows: one quad of
+// one row a thread, about nine pieces in three rounds of four loads; 16 rows took four
+// such items in sequence: gamma 4 MQA verify 0.216 -> 0.185 ms a step).
+#ifndef KVC_TC_COMBINE_ROWS
+#define KVC_TC_COMBINE_ROWS 4
+#endif
+constexpr int kCombineRows = KVC_TC_COMBINE_ROWS;
 template <typename T, int D>
 __global__ void __launch_bounds__(128) combine_kernel(const AttendParams p) {
   griddep_launch_dependents();

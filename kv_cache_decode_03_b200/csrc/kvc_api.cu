@@ -85,11 +85,11 @@ constexpr int kEltBytes = 2;
 #define KVC_TC_COMBINE 1
 #endif
 // ... when a segment's partials average more than this many bytes: one CTA merging them
-// in the attend kernel takes ~20 us at 600 KB (a trace), the combine launch a few us and
-// its own overhead (measured: MQA verify gamma 4, 600 KB a segment, +10 %; gamma 2 and 8,
-// 300 KB, -4 % and +1 %)
+// in the attend kernel takes ~20 us at 600 KB (a trace); the combine launch, with 4 rows a
+// block, was measured on MQA verify at gamma 2 / 4 / 8 (300 / 600 / 300 KB a segment):
+// +12 / +14 / +5 % a step, and flat on GQA verify gamma 8 (19 KB a segment)
 #ifndef KVC_TC_COMBINE_MIN_BYTES
-#define KVC_TC_COMBINE_MIN_BYTES (400 << 10)
+#define KVC_TC_COMBINE_MIN_BYTES (64 << 10)
 #endif
 #ifndef KVC_TC_RB_MAJOR
 #define KVC_TC_RB_MAJOR 1
