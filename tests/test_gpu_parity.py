@@ -90,12 +90,15 @@ def test_page_sizes(P):
 
 
 # ---------------------------------------------------------------------------
-# 64 or more query rows per KV head (the 128-row tcgen05 blocks): MQA decode,
+# 17 or more query rows per KV head (the 128-row tcgen05 blocks): MQA decode,
 # verify chunks, prefill chunks; row counts that leave a ragged last block and
-# blocks that cut one head's chunk in two
+# blocks that cut one head's chunk in two.  At these lengths the partial pieces of a
+# segment are merged by the combine launch in 4-row chunks; 18 rows (4 x 4 + 2) and a
+# last block of 7 rows (135 = 128 + 4 + 3) leave a short chunk.
 # ---------------------------------------------------------------------------
 
-TC_HEADS = [(64, 1, 1), (16, 2, 8), (8, 1, 25), (32, 1, 9), (12, 12, 128)]
+TC_HEADS = [(64, 1, 1), (16, 2, 8), (8, 1, 25), (32, 1, 9), (12, 12, 128), (6, 1, 3),
+            (3, 1, 45)]
 
 
 @pytest.mark.parametrize("D", [64, 128])
