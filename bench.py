@@ -374,9 +374,10 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     ns, split_tokens = cache.plan(c.H_q, c.T_new, max_pages)
     stream = torch.cuda.Stream()
     scale = c.scale
-    # kvc_append_attend is one launch on the mma.sync stream-K kernels (bf16/fp16 and
-    # E4M3 stages: up to 16 rows per KV head); the tcgen05 and fixed-split plans append first
-    fused = split_tokens == 0 and (c.H_q // c.H_kv) * c.T_new <= 16
+    # kvc_append_attend is one attend launch on the persistent stream-K kernels (mma.sync
+    # with bf16/fp16 or E4M3 stages, tcgen05 for 17+ rows: the append fused into it, a
+    # tcgen05 plan's combine launch after it); the fixed-split plans append first
+    fused = split_tokens == 0
 
     def step(q=qs, k=ks, v=vs, o=outs):
         for layer in range(c.layers):
@@ -523,7 +524,7 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     segs = c.B * c.H_kv * -(-rows // 128)
     combine = (split_tokens == 0 and rows > 16 and not fp8 and
                ns / segs * min(rows, 128) * c.D * 4 > 64 * 1024)
-    res["launches_per_step"] = c.layers * (1 if fused else 3 if combine else 2)
+    res["launches_per_step"] = c.layers * ((1 if fused else 2) + (1 if combine else 0))
     res["ns"], res["split_tokens"] = ns, split_tokens
     # one call's bytes: K/V read + q read + out written + k_new/v_new read + rows written
     # (the FP8 count already holds both sides of the append)
@@ -552,9 +553,9 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["frac_in_step"] = roof["achieved_in_step"] / roof["peak"]
     roof["kernel"] = (kernel + (", fused: one launch per kvc_append_attend call (append, "
-                                "split attend, merge)" if fused else
-                                ", after the append kernel and before its combine launch"
-                                if combine else ", after the append kernel"))
+                                "split attend, merge)" if fused and not combine else
+                                ", fused: append and split attend in one launch, then the "
+                                "combine launch" if fused else ", after the append kernel"))
     roof["duration"] = (f"median of {len(durs)} event-bracketed kvc_append_attend calls "
                         f"({res['call_ms_median'] * 1e3:.2f} us; each call alone, so without "
                         f"the overlap of the dependent launch); achieved_in_step = the "

@@ -187,11 +187,16 @@ kvc_status kvc_attend_window(kvc_cache* cache, int layer, const void* q, int H_q
  * kvc_append_attend -- kvc_append followed by kvc_attend for the same new tokens, in
  * one launch where the kernel allows it ("9. 推理" 9.3: the new token's K/V join the
  * cache and are attended in the same step).  Arguments are those of the two calls.
- * On the persistent mma.sync stream-K kernel (up to 16 query rows per KV head, up to 8
- * on an FP8 cache) the attend kernel itself writes the new rows into the cache (an FP8
- * cache: quantised exactly as kvc_append does) and uses them straight from k_new /
- * v_new; in other cases the two kernels run back to back on `stream`.  Results (cache
- * contents and out) are identical to calling kvc_append then kvc_attend.
+ * On the persistent stream-K kernels the attend kernel itself writes the new rows into
+ * the cache: on mma.sync (up to 16 query rows per KV head, up to 8 on an FP8 cache; an
+ * FP8 cache quantised exactly as kvc_append does) it also uses them straight from
+ * k_new / v_new; on tcgen05 (17 or more rows) its copy warps store them into the cache
+ * before they load those tiles (the combine launch, where the plan has one, follows).
+ * The fixed-split plans (sliding windows, 9+ rows on an FP8 cache, batches beyond the
+ * stream-K scan) run the two kernels back to back on `stream`.  Results (cache contents
+ * and out) are identical to calling kvc_append then kvc_attend for valid inputs; a
+ * request whose new rows would overflow its capacity is flagged KVC_ERR_BOUNDS, and the
+ * fused kernels then write none of its rows.
  */
 kvc_status kvc_append_attend(kvc_cache* cache, int layer, const void* k_new, const void* v_new,
                              const void* q, int H_q, int T_new, const int32_t* block_table,

@@ -434,9 +434,45 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
         if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
       unsigned char* dst = ring + st * C::kTileBytes;
+      const int t0 = pc.k * C::kTile;
+      if (p.k_new != nullptr) {
+        // Fused append: the new positions of this tile go into the pool (this warp's K
+        // or V) before its copy reads them.  Every CTA that loads such a tile writes them
+        // (the row blocks of a segment write the same bytes), after the dependency wait;
+        // each lane's proxy fence, then the warp barrier, order the stores before the
+        // copies' async-proxy reads.
+        const int n_lo = max(pc.L, t0), n_hi = min(pc.L + p.T_new, t0 + C::kTile);
+        if (n_lo < n_hi) {  // the same decision in every lane
+          constexpr int CH = D / 8;  // 16-byte chunks a row
+          const char* src = static_cast<const char*>(is_k ? p.k_new : p.v_new);
+          char* pool = static_cast<char*>(const_cast<void*>(is_k ? p.k_pool : p.v_pool));
+#pragma unroll 1
+          for (int idx = lane_id; idx < (n_hi - n_lo) * CH; idx += 32) {
+            const int rr = idx / CH;
+            const int ch = idx - rr * CH;
+            const int pos = n_lo + rr;
+            long long row;
+            if (PAGED) {
+              const int page = p.block_table[(size_t)pc.b * p.max_pages + (pos >> p.page_shift)];
+              if (page < 0 || page >= p.num_pages) {
+                flag_error(p.err, KVC_ERR_BOUNDS);
+                continue;
+              }
+              row = ((long long)page * p.H_kv + pc.g) * Pg + (pos & (Pg - 1));
+            } else {
+              row = ((long long)pc.b * p.H_kv + pc.g) * p.max_T + pos;
+            }
+            const size_t s_off =
+                ((((size_t)pc.b * p.H_kv + pc.g) * p.T_new + (pos - pc.L)) * D + ch * 8) *
+                sizeof(T);
+            st_global_v4(pool + (row * D + ch * 8) * (long long)sizeof(T),
+                         ld_global_nc_v4(src + s_off));
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+      }
       if (lane_id == 0) mbar_arrive_expect_tx(&full[st], C::kTileBytes);
       __syncwarp();
-      const int t0 = pc.k * C::kTile;
       if (!PAGED) {
         if (lane_id < C::kHalves)
           tma_load_2d(dst + lane_id * C::kBoxBytes, tm, lane_id * 64,

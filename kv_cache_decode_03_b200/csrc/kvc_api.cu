@@ -845,7 +845,7 @@ kvc_status launch_attend_tc_streamk(const kvc::AttendParams& p, int grid, bool p
 }
 
 // The combine launch after a tcgen05 stream-K attend (p.sk_combine != 0): one block
-// per (segment, 16-row chunk), dependent on the attend grid.
+// per (segment, chunk of kCombineRows rows), dependent on the attend grid.
 template <int D, typename T>
 kvc_status launch_combine(const kvc::AttendParams& p, bool pdl, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
@@ -1504,10 +1504,12 @@ extern "C" kvc_status kvc_attend_noalloc(kvc_cache* c, int layer, const void* q,
 }
 
 // ---------------------------------------------------------------------------
-// Append and attend in one call.  With the persistent stream-K kernel this is one
-// launch: the tile holding the new positions takes them from k_new / v_new and
-// the kernel writes them into the cache.  Other kernels run the append kernel
-// and then the attend kernel on the same stream.
+// Append and attend in one call.  With the persistent stream-K kernels this is one
+// attend launch (plus the combine launch of a tcgen05 plan that uses one): on mma.sync
+// the tile holding the new positions takes them from k_new / v_new and the kernel
+// writes them into the cache; on tcgen05 the producer warps write them into the cache
+// before the copies of those tiles.  The fixed-split kernels run the append kernel and
+// then the attend kernel on the same stream.
 extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_new,
                                         const void* v_new, const void* q, int H_q, int T_new,
                                         const int32_t* block_table, int max_pages,
@@ -1524,7 +1526,7 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   if (!c->paged && block_table) return KVC_ERR_INVALID_ARG;
   if (!(scale == scale)) return KVC_ERR_INVALID_ARG;
   const Plan pl = make_plan(c, H_q, T_new, max_pages);
-  if (!pl.streamk || pl.tc) {  // only the mma.sync stream-K kernels fuse the append
+  if (!pl.streamk) {  // the fixed-split kernels do not fuse the append
     kvc_status st = kvc_append(c, layer, k_new, v_new, T_new, block_table, max_pages,
                                seq_lens, stream);
     if (st != KVC_OK) return st;
@@ -1545,6 +1547,13 @@ extern "C" kvc_status kvc_append_attend(kvc_cache* c, int layer, const void* k_n
   if (pl.fp8)
     return dispatch_streamk_fp8(p, c->D, c->paged, pl.grid, c->dependent_launch, c->tmk[layer],
                                 c->tmv[layer], s);
+  if (pl.tc)
+    return c->dtype == KVC_BF16
+               ? dispatch_tc_streamk<__nv_bfloat16>(p, c->D, c->paged, pl.grid,
+                                                    c->dependent_launch, c->tmk[layer],
+                                                    c->tmv[layer], s)
+               : dispatch_tc_streamk<__half>(p, c->D, c->paged, pl.grid, c->dependent_launch,
+                                             c->tmk[layer], c->tmv[layer], s);
   const CUtensorMap& tk = p.sk_blocked ? c->tmk4[layer] : c->tmk[layer];
   const CUtensorMap& tv = p.sk_blocked ? c->tmv4[layer] : c->tmv[layer];
   return c->dtype == KVC_BF16

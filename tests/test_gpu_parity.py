@@ -443,10 +443,21 @@ FUSED = {
                                               seed=51, pool_seed=52),
     "gqa2_d64_paged": lambda: W.paged_case("fz9", 3, 8, 4, 64, "bf16", 1, 0, 900, 8,
                                            seed=53, pool_seed=54),
+    # tcgen05 stream-K (17+ rows): the copy warps store the new rows before loading their
+    # tiles; MQA verify (then the combine launch), new rows straddling tile boundaries in
+    # two row blocks, 8-token pages, and a prefill chunk whose later positions only the
+    # second row block sees
+    "mqa_tc_paged": lambda: W.paged_case("fz6", 2, 32, 1, 128, "bf16", 4, 100, 2000, 16,
+                                         seed=48, pool_seed=49),
+    "mqa_tc_straddle_two_blocks": lambda: W.contig_case("fz10", 3, 32, 1, 128, "bf16", 8,
+                                                        [60, 125, 1021], seed=55,
+                                                        max_T=1100),
+    "gqa_tc_d64_fp16_pages8": lambda: W.paged_case("fz11", 3, 16, 2, 64, "fp16", 8, 0, 900,
+                                                   8, seed=56, pool_seed=57),
+    "mha_tc_prefill_chunk": lambda: W.contig_case("fz12", 2, 2, 2, 64, "bf16", 200,
+                                                  [0, 300], seed=58, max_T=520),
     # other kernels: append then attend, two launches
     "mha_simt_d32": lambda: W.contig_case("fz5", 2, 8, 8, 32, "fp16", 1, [700, 33], seed=47),
-    "mqa_splitk": lambda: W.paged_case("fz6", 2, 32, 1, 128, "bf16", 4, 100, 2000, 16,
-                                       seed=48, pool_seed=49),
 }
 
 
