@@ -265,12 +265,13 @@ kvc_status kvc_inject_stall(kvc_cache* cache);
 
 /*
  * kvc_inject_replan -- test hook for the dependent launch.  The persistent stream-K
- * kernel plans its range from the lengths it reads before its dependency wait and
- * issues its first copies from that plan right after the wait, while it reads the
- * lengths again; if they changed, it waits for those copies, resets its pipeline and
- * plans again.  This hook makes the next attend call on this cache (stream-K only)
- * take that path whatever the lengths: its results are the same as without it.  The
- * next call consumes it either way.
+ * kernels plan their range from the lengths they read before the dependency wait and
+ * read the lengths again after it; if they changed, they plan again.  The mma.sync
+ * kernel issues its first copies from the first plan right after the wait, so it also
+ * waits for those copies and resets its pipeline first; the tcgen05 kernel issues
+ * nothing before the check.  This hook makes the next attend call on this cache
+ * (stream-K only) take that path whatever the lengths: its results are the same as
+ * without it.  The next call consumes it either way.
  */
 kvc_status kvc_inject_replan(kvc_cache* cache);
 

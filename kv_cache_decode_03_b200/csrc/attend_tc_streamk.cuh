@@ -73,21 +73,31 @@ struct SkRange {
   TileCursor<R> cur;
 };
 
+// Mixes one length into a thread's digest of the lengths it scanned.
+__device__ __forceinline__ uint32_t len_mix(uint32_t h, int L) {
+  return (h ^ (uint32_t)L) * 0x9E3779B1u + 0x7F4A7C15u;
+}
+
 // Plans this CTA's range from seq_lens with a block scan over the requests; every one of
 // the NTH threads calls it.  P and Ls: 2B + 1 ints of shared memory, wsum: NTH/32 ints.
-// Lengths outside the cache flag KVC_ERR_BOUNDS and contribute no tiles.
+// Lengths outside the cache contribute no tiles (and flag KVC_ERR_BOUNDS when
+// `authoritative`); `digest` receives this thread's digest of the lengths it read
+// (requests tid * ceil(B / NTH) onwards).
 template <int R, int NTH, bool PAGED>
-__device__ __forceinline__ SkRange<R> sk_plan(const AttendParams& p, int* P, int* Ls, int* wsum) {
+__device__ __forceinline__ SkRange<R> sk_plan(const AttendParams& p, int* P, int* Ls, int* wsum,
+                                              bool authoritative, uint32_t& digest) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = ceil_div(p.B, NTH);
   const int b_lo = min(p.B, tid * per), b_hi = min(p.B, b_lo + per);
   int sum = 0;
+  digest = 0;
   for (int b = b_lo; b < b_hi; ++b) {
     const int L = p.seq_lens[b];
+    digest = len_mix(digest, L);
     Ls[b] = L;
     int t = 0;
     if (length_ok(p, L, PAGED)) t = request_tiles<R>(p, L);
-    else flag_error(p.err, KVC_ERR_BOUNDS);
+    else if (authoritative) flag_error(p.err, KVC_ERR_BOUNDS);
     P[b] = t;
     sum += t;
   }
@@ -362,9 +372,27 @@ __global__ void __launch_bounds__(TcCfg<D>::kThreads, 2)
     fence_barrier_init();
   }
   tc_fence_before();
-  griddep_wait();
+  // Plan from the lengths as they stand while the grid ahead finishes (shared memory
+  // only); after the dependency wait every thread reads the lengths it scanned again and
+  // the block plans once more if any changed (or a test asked for it: p.replan).
   int* Pscan = reinterpret_cast<int*>(smem);
-  const SkRange<R> rg = sk_plan<R, C::kThreads, PAGED>(p, Pscan, Pscan + p.B + 1, flags + 8);
+  SkRange<R> rg;
+#pragma unroll 1
+  for (int pass = 0;; ++pass) {  // pass 0 before the wait, pass 1 only if it was stale
+    uint32_t digest;
+    rg = sk_plan<R, C::kThreads, PAGED>(p, Pscan, Pscan + p.B + 1, flags + 8, pass > 0, digest);
+    if (pass > 0) break;
+    griddep_wait();
+    const int per = ceil_div(p.B, C::kThreads);
+    const int b_lo = min(p.B, tid * per), b_hi = min(p.B, b_lo + per);
+    uint32_t h = 0;
+    for (int b = b_lo; b < b_hi; ++b) {
+      const int L = p.seq_lens[b];
+      h = len_mix(h, L);
+      if (!length_ok(p, L, PAGED)) flag_error(p.err, KVC_ERR_BOUNDS);
+    }
+    if (!__syncthreads_or(h != digest || p.replan != 0)) break;
+  }
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t tO = tmem + C::kOCol;

@@ -164,15 +164,23 @@ REPLAN = {
     # MHA decode, one row per KV head
     "mha_d64": lambda: W.contig_case("rp3", 4, 12, 12, 64, "fp16", 1, [2047, 1, 900, 4095],
                                      seed=804, max_T=4100),
+    # tcgen05 stream-K (17+ rows): MQA verify (then the combine launch), and paged GQA
+    # verify with 64 rows per KV head
+    "mqa_tc_t4": lambda: W.contig_case("rp4", 4, 32, 1, 128, "bf16", 4, [4000, 2100, 0, 2500],
+                                       seed=805, max_T=4100),
+    "gqa_tc_paged_t8": lambda: W.paged_case("rp5", 3, 16, 2, 128, "bf16", 8, 1500, 3000, 16,
+                                            seed=806, pool_seed=807),
 }
 
 
 @pytest.mark.parametrize("kind", sorted(REPLAN))
 def test_replan_after_the_wait_gives_identical_results(kind):
     """kvc_inject_replan makes the stream-K kernel treat the plan it made before its
-    dependency wait as stale: the copies it issued from that plan are drained, the
-    pipeline barriers reset and the range planned again.  Outputs (attend, and the fused
-    append + attend with the cache it writes) are bit-identical to the ordinary path's."""
+    dependency wait as stale: on mma.sync the copies it issued from that plan are
+    drained, the pipeline barriers reset and the range planned again; on tcgen05 (which
+    issues nothing before the check) the range is planned again.  Outputs (attend, and
+    the fused append + attend with the cache it writes) are bit-identical to the ordinary
+    path's."""
     case = REPLAN[kind]()
     run = H.DeviceCase(case)
     try:
