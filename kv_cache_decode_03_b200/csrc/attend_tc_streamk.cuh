@@ -1,5 +1,5 @@
 // attend_tc_streamk.cuh -- N2 + N3 (tcgen05, persistent): stream-K split attention for
-// 64 or more query rows per KV head (MQA verify chunks, large GQA groups, chunked prefill).
+// 17 or more query rows per KV head (MQA verify chunks, large GQA groups, chunked prefill).
 //
 // The per-tile arithmetic is that of attend_tc.cuh (S = Q.K^T and O += P.V on tcgen05
 // with fp32 accumulators in TMEM, one softmax thread per query row, lazy rescaling,
@@ -18,7 +18,13 @@
 // * A piece that covers its whole segment writes the output rows directly; otherwise
 //   it writes a normalised partial (o / l, base-2 log-sum-exp) to one of its CTA's two
 //   workspace slots and takes a release-acquire ticket; the segment's last finisher
-//   merges the pieces by log-sum-exp ("9. 推理" 9.7: exact up to rounding).
+//   merges the pieces by log-sum-exp ("9. 推理" 9.7: exact up to rounding), or, when the
+//   plan's segments carry large partials (p.sk_combine), leaves a descriptor for the
+//   dependent combine_kernel launch, which merges them over many CTAs.
+// * The range is planned before the dependency wait (shared memory only) and checked
+//   against the lengths after it; it is planned again if any changed.
+// * With k_new / v_new (kvc_append_attend) the K and V copy warps store a tile's new
+//   rows into the pool before its TMA copy reads them (the append, fused).
 //
 // Roles (224 threads): warps 0-3 softmax (thread t = TMEM lane t = query row t of the
 // block; they also load Q and run the epilogue and the merge), warp 4 lane 0 issues the
