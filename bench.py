@@ -43,6 +43,10 @@ METRIC = ("decode-attention KV HBM GB/s (% of B200 peak) and tokens/s per layer-
 
 # The sources each profiled kernel is compiled from: a committed ncu summary stays
 # valid while these files are unchanged.
+# The library's default threshold for the tcgen05 combine launch (KVC_TC_COMBINE_MIN_BYTES
+# in csrc/kvc_api.cu): segments whose partials average more take a second launch.
+TC_COMBINE_MIN_BYTES = 64 * 1024
+
 KERNEL_SOURCES = {
     "attend_streamk_kernel": ("attend_streamk.cuh", "attend_fp8.cuh", "fp8.cuh",
                               "splitk_epilogue.cuh", "device_common.cuh", "params.cuh"),
@@ -518,12 +522,11 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     layer_bytes = fp8_algorithmic_bytes(c) if fp8 else c.algorithmic_bytes()
     res["layer_bytes"] = layer_bytes
     res["step_bytes"] = c.layers * layer_bytes
-    # tcgen05 stream-K (17+ rows) with large segment merges: append, attend, combine (the
-    # library's default threshold: partials above 64 KB a segment on average)
+    # tcgen05 stream-K (17+ rows) with large segment merges: attend (append fused), combine
     rows = (c.H_q // c.H_kv) * c.T_new
     segs = c.B * c.H_kv * -(-rows // 128)
     combine = (split_tokens == 0 and rows > 16 and not fp8 and
-               ns / segs * min(rows, 128) * c.D * 4 > 64 * 1024)
+               ns / segs * min(rows, 128) * c.D * 4 > TC_COMBINE_MIN_BYTES)
     res["launches_per_step"] = c.layers * ((1 if fused else 2) + (1 if combine else 0))
     res["ns"], res["split_tokens"] = ns, split_tokens
     # one call's bytes: K/V read + q read + out written + k_new/v_new read + rows written

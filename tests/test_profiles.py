@@ -1,4 +1,5 @@
-"""The committed ncu summaries that bench.py reads (CPU only).
+"""The committed ncu summaries that bench.py reads, and its mirror of a library
+default (CPU only).
 
 bench.py takes `roofline.traffic` from a summary's machine-readable block only
 while the kernel's sources hash to the value recorded there; these checks keep
@@ -52,3 +53,12 @@ def test_traffic_is_used_only_while_the_sources_match():
         else:
             assert got is None, f.name
     assert bench.profiled_traffic("no_such_kernel<1>") is None
+
+
+def test_bench_mirrors_the_combine_threshold():
+    """bench.py counts a tcgen05 plan's combine launch with the library's default
+    threshold; the two must not drift apart."""
+    src = (ROOT / "kv_cache_decode_03_b200" / "csrc" / "kvc_api.cu").read_text()
+    m = re.search(r"#define KVC_TC_COMBINE_MIN_BYTES \((\d+) << (\d+)\)", src)
+    assert m, "KVC_TC_COMBINE_MIN_BYTES default not found"
+    assert bench.TC_COMBINE_MIN_BYTES == int(m.group(1)) << int(m.group(2))
