@@ -380,7 +380,8 @@ def measure(case: W.Case, kv_format: str, steps: int, warmup: int, samples: int,
     scale = c.scale
     # kvc_append_attend is one attend launch on the persistent stream-K kernels (mma.sync
     # with bf16/fp16 or E4M3 stages, tcgen05 for 17+ rows: the append fused into it, a
-    # tcgen05 plan's combine launch after it); the fixed-split plans append first
+    # tcgen05 plan's combine launch after it); the fixed-split plans append in a launch of
+    # its own first
     fused = split_tokens == 0
 
     def step(q=qs, k=ks, v=vs, o=outs):

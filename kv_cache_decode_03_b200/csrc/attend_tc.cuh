@@ -3,9 +3,10 @@
 //
 // Same contract as the other attend kernels: for every query row (query head h
 // of KV head g, new row i) of request b, exact-softmax attention over positions
-// 0 .. L_b + i ("项目 9-16" projects 11/15; "9. 推理" 9.7).  With 64 or more rows
-// sharing each K/V row the work is a real dense contraction, so a CTA takes a
-// block of 128 query rows as the MMA M dimension:
+// 0 .. L_b + i ("项目 9-16" projects 11/15; "9. 推理" 9.7).  With many rows sharing
+// each K/V row the work is a real dense contraction, so a CTA takes a block of 128
+// query rows as the MMA M dimension (the library routes 17 or more rows per KV head
+// here; with fewer than 128 the rest of the block idles and it still pays):
 //     S[128 x 64]  = Q[128 x D] . K_tile^T        tcgen05.mma, fp32 in TMEM
 //     O[128 x D]  += P[128 x 64] . V_tile          tcgen05.mma, fp32 in TMEM
 // Roles (warp-specialised, 224 threads):
